@@ -1,0 +1,275 @@
+"""fp64 CPU oracle of the DeepSeek-V2 MLA decode step (weight-absorbed and not).
+
+TEST INFRASTRUCTURE. Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` may import this module. The product (the CUDA library and its Python
+binding) never imports it, and this module imports nothing from the product package: the
+two share no code. Everything here is plain numpy in float64; a matrix product is the only
+library primitive used as a step.
+
+Sources, cited by page title and section:
+
+[V2-walk]  "DeepSeek-V2 paper walkthrough" (2kiu.com/news/6085339)
+           §2.1 MHA cache arithmetic and the kv_cache_bytes estimate;
+           §2.2 low-rank joint KV compression; §2.3 matrix absorption (displayed equation);
+           §2.4 decoupled RoPE; §5.2 position-path check; §6 validation recipe.
+[V2-arch]  "Transformer-15: DeepSeek-V2 architecture, MLA, DeepSeekMoE" (zeeklog.com)
+           MHA equations (per-head softmax attention, W^O), eqs. 9-11, cache table.
+[V2-notes] "DeepSeek-V2" paper notes (process-cxr.github.io ai-library), section
+           "Multi-Head Latent Attention": shared k^R, cache = d_c + d_h^R = 4.5 d_h l.
+[V3-walk]  "DeepSeek-V3 technical report walkthrough" (2kiu.com/news/6340724)
+           §2.2 KV-side forward (only c^KV and k^R are cached); §2.3 absorption, RoPE R_p.
+
+What the decode step computes, for sequence b with L = kv_len[b] cached tokens and
+head i (non-absorbed definition, [V2-arch] MHA equations with [V2-arch] eqs. 9-11 and the
+decoupled key of [V2-notes] / [V3-walk] §2.3):
+
+    k_j,i = [ W_UK,i c_j ; k^R_j ]            c_j = c^KV_j (d_c), k^R_j shared by all heads
+    v_j,i =   W_UV,i c_j
+    q_i   = [ q^C_i ; RoPE_{L-1}(q^R_i) ]
+    s_j   = scale * q_i . k_j,i               j = 0 .. L-1
+    o_i   = sum_j softmax_j(s)_j v_j,i        (d_h)
+
+The absorbed form ([V2-walk] §2.3 displayed equation, [V3-walk] §2.3) reaches the same
+o_i through q'_i = W_UK,i^T q^C_i, a latent output sum_j p_j c_j, and W_UV,i last.
+
+Readings where the pages are silent (each is also listed in the design doc):
+  * scale = 1/sqrt(d_h + d_h^R). The pages print only the MHA 1/sqrt(d_h); the MLA
+    equations that would fix it are omitted or lost in extraction.
+  * RoPE: interleaved pairs (x[2m], x[2m+1]), theta_m = base^(-2m/d_R), angle pos*theta_m,
+    0-based positions. base == 0 means "no rotation" (RoPE off).
+  * The query of the new token sits at position L-1 and attends to all L cached rows,
+    its own included ([V2-arch]: the new token's K/V is appended, then attended). So the
+    causal mask has no interior holes, only the end at L.
+  * k^R in the cache is already rotated (it is rotated when it is written, [V3-walk]
+    §2.2); the decode step reads it as it is.
+  * kv_len == 0: the output is 0 and the log-sum-exp is -inf.
+
+Cache layouts accepted (the row is [c^KV (d_c) ; k^R (d_R)], 576 values):
+  * contiguous: array [B, Lmax, d_c + d_R];
+  * paged: array [num_pages, page_size, d_c + d_R] plus page_table[B, max_pages]; token j
+    of sequence b sits at page page_table[b, j // page_size], slot j % page_size.
+A cache given as uint16 is read as bf16 bit patterns and widened exactly to float64.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+D_HEAD = 128      # d_h
+D_LATENT = 512    # d_c
+D_ROPE = 64       # d_h^R
+
+
+# ---------------------------------------------------------------------------
+# cache-size arithmetic  ([V2-walk] §2.1, [V2-arch] cache table, [V2-notes] MLA)
+# ---------------------------------------------------------------------------
+
+def mha_cache_elements_per_token(n_heads: int, d_head: int) -> int:
+    """Elements an MHA layer caches per token: one key and one value per head."""
+    return 2 * n_heads * d_head
+
+
+def mla_cache_elements_per_token(d_latent: int, d_rope: int) -> int:
+    """Elements an MLA layer caches per token: the latent c^KV plus the shared k^R."""
+    return d_latent + d_rope
+
+
+def kv_cache_bytes(seq_len: int, n_layers: int, elems_per_token_per_layer: int,
+                   dtype_bytes: int = 2) -> int:
+    """Bytes one request's KV cache takes: tokens x layers x elements x element size."""
+    return seq_len * n_layers * elems_per_token_per_layer * dtype_bytes
+
+
+# ---------------------------------------------------------------------------
+# input widening and row gathering
+# ---------------------------------------------------------------------------
+
+def widen(x) -> np.ndarray:
+    """Return x as float64. uint16 input is taken as bf16 bit patterns (exact widening:
+    a bf16 is the top 16 bits of an IEEE binary32)."""
+    a = np.asarray(x)
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def token_rows(cache, b: int, kv_len: int, page_table=None, page_size: int = 0) -> np.ndarray:
+    """The kv_len cached rows of sequence b, in token order, as float64 [kv_len, 576]."""
+    cache = np.asarray(cache)
+    if kv_len == 0:
+        return np.zeros((0, cache.shape[-1]), dtype=np.float64)
+    if page_table is None or page_size == 0:
+        return widen(cache[b, :kv_len, :])
+    pt = np.asarray(page_table)
+    j = np.arange(kv_len)
+    pages = pt[b, j // page_size]
+    slots = j % page_size
+    return widen(cache[pages, slots, :])
+
+
+# ---------------------------------------------------------------------------
+# RoPE on the decoupled query  ([V2-walk] §2.4, [V3-walk] §2.3; convention: module doc)
+# ---------------------------------------------------------------------------
+
+def rope_angles(pos: int, d_rope: int, base: float) -> np.ndarray:
+    """Angles pos * theta_m for the d_rope/2 pairs, theta_m = base^(-2m/d_rope)."""
+    m = np.arange(d_rope // 2, dtype=np.float64)
+    theta = base ** (-2.0 * m / d_rope)
+    return float(pos) * theta
+
+
+def rope_rotate(x, pos: int, base: float) -> np.ndarray:
+    """Rotate each interleaved pair (x[2m], x[2m+1]) of the last axis by pos * theta_m.
+    base == 0 leaves x unchanged (RoPE off)."""
+    x = widen(x)
+    if base == 0:
+        return x.copy()
+    ang = rope_angles(pos, x.shape[-1], base)
+    c, s = np.cos(ang), np.sin(ang)
+    even, odd = x[..., 0::2], x[..., 1::2]
+    y = np.empty_like(x)
+    y[..., 0::2] = even * c - odd * s
+    y[..., 1::2] = even * s + odd * c
+    return y
+
+
+# ---------------------------------------------------------------------------
+# softmax with its log-sum-exp  ([V2-arch] MHA equation: Softmax_j over j = 1..t)
+# ---------------------------------------------------------------------------
+
+def softmax_lse(s: np.ndarray, axis: int = 0):
+    """Two-pass softmax along `axis`: subtract the max, exponentiate, normalise.
+    Returns (p, lse) with lse = log(sum(exp(s))). An empty axis gives lse = -inf."""
+    s = np.asarray(s, dtype=np.float64)
+    if s.shape[axis] == 0:
+        shape = list(s.shape)
+        del shape[axis]
+        return s.copy(), np.full(shape, -np.inf)
+    m = np.max(s, axis=axis, keepdims=True)
+    e = np.exp(s - m)
+    z = np.sum(e, axis=axis, keepdims=True)
+    p = e / z
+    lse = np.squeeze(m + np.log(z), axis=axis)
+    return p, lse
+
+
+def default_scale(d_head: int = D_HEAD, d_rope: int = D_ROPE) -> float:
+    """1/sqrt(d_h + d_h^R): the reading of the softmax scale (see module doc)."""
+    return 1.0 / math.sqrt(d_head + d_rope)
+
+
+# ---------------------------------------------------------------------------
+# the absorbed path, one stage at a time
+# ---------------------------------------------------------------------------
+
+def absorb_query(q_c, q_r, w_uk, kv_lens, rope_base: float) -> np.ndarray:
+    """Absorbed query rows [B, n_h, d_c + d_R] in float64.
+
+    q'_{b,i} = W_UK,i^T q^C_{b,i}   ([V2-walk] §2.3 displayed equation; [V3-walk] §2.3)
+    followed by RoPE_{L_b - 1}(q^R_{b,i}) in the last d_R slots ([V2-walk] §2.4).
+    w_uk is [n_h, d_h, d_c]: W_UK,i maps a latent c (d_c) to the head's content key (d_h).
+    """
+    q_c, q_r, w_uk = widen(q_c), widen(q_r), widen(w_uk)
+    kv_lens = np.asarray(kv_lens)
+    B, H, _ = q_c.shape
+    d_c = w_uk.shape[2]
+    d_r = q_r.shape[2]
+    out = np.zeros((B, H, d_c + d_r))
+    for b in range(B):
+        pos = max(int(kv_lens[b]) - 1, 0)
+        for i in range(H):
+            out[b, i, :d_c] = w_uk[i].T @ q_c[b, i]
+            out[b, i, d_c:] = rope_rotate(q_r[b, i], pos, rope_base)
+    return out
+
+
+def latent_attention(q_abs, cache, kv_lens, scale: float, page_table=None,
+                     page_size: int = 0, d_latent: int = D_LATENT):
+    """Attention over the shared latent cache for every (sequence, head).
+
+    s_{i,j} = scale * q'_i . [c_j ; k^R_j], p = softmax_j(s), latent_i = sum_j p_j c_j.
+    Returns (latent [B, n_h, d_c], lse [B, n_h]); lse is log sum_j exp(s_{i,j}).
+    The score uses the full 576-wide row, the weighted sum only the first d_c values
+    ([V2-walk] §2.3: the weighted sum stays in the latent space).
+    """
+    q_abs = widen(q_abs)
+    kv_lens = np.asarray(kv_lens)
+    B, H, _ = q_abs.shape
+    latent = np.zeros((B, H, d_latent))
+    lse = np.full((B, H), -np.inf)
+    for b in range(B):
+        L = int(kv_lens[b])
+        if L == 0:
+            continue
+        rows = token_rows(cache, b, L, page_table, page_size)      # [L, 576]
+        s = (rows @ q_abs[b].T) * scale                              # [L, H]
+        p, lse[b] = softmax_lse(s, axis=0)
+        latent[b] = p.T @ rows[:, :d_latent]
+    return latent, lse
+
+
+def apply_wuv(latent, w_uv) -> np.ndarray:
+    """o_{b,i} = W_UV,i latent_{b,i}; w_uv is [n_h, d_h, d_c] ([V2-arch] eq. 11)."""
+    latent, w_uv = widen(latent), widen(w_uv)
+    B, H, _ = latent.shape
+    out = np.zeros((B, H, w_uv.shape[1]))
+    for i in range(H):
+        out[:, i, :] = latent[:, i, :] @ w_uv[i].T
+    return out
+
+
+# ---------------------------------------------------------------------------
+# the non-absorbed definition: plain MHA over materialised keys and values
+# ---------------------------------------------------------------------------
+
+def mla_decode_nonabsorbed(q_c, q_r, w_uk, w_uv, cache, kv_lens, scale: float,
+                           rope_base: float, page_table=None, page_size: int = 0,
+                           pairs=None) -> np.ndarray:
+    """Head outputs o [B, n_h, d_h] by the non-absorbed definition (module doc).
+
+    Per (b, i): k^C_j = W_UK,i c_j and v_j = W_UV,i c_j are materialised for every cached
+    token ([V2-arch] eqs. 9-11), the key gets the shared k^R_j appended and the query its
+    rotated q^R ([V2-notes] decoupled RoPE), and ordinary softmax attention follows
+    ([V2-arch] MHA equation). `pairs` restricts the work to a list of (b, i); the other
+    outputs are left at NaN.
+    """
+    q_c, q_r = widen(q_c), widen(q_r)
+    w_uk, w_uv = widen(w_uk), widen(w_uv)
+    kv_lens = np.asarray(kv_lens)
+    B, H, d_h = q_c.shape
+    d_c = w_uk.shape[2]
+    out = np.full((B, H, d_h), np.nan)
+    if pairs is None:
+        pairs = [(b, i) for b in range(B) for i in range(H)]
+    by_seq: dict[int, list[int]] = {}
+    for b, i in pairs:
+        by_seq.setdefault(int(b), []).append(int(i))
+    for b, heads in by_seq.items():
+        L = int(kv_lens[b])
+        if L == 0:
+            for i in heads:
+                out[b, i] = 0.0
+            continue
+        rows = token_rows(cache, b, L, page_table, page_size)
+        c, k_r = rows[:, :d_c], rows[:, d_c:]
+        for i in heads:
+            k_content = c @ w_uk[i].T                                   # [L, d_h]
+            v = c @ w_uv[i].T                                           # [L, d_h]
+            q = np.concatenate([q_c[b, i], rope_rotate(q_r[b, i], L - 1, rope_base)])
+            keys = np.concatenate([k_content, k_r], axis=1)             # [L, d_h + d_R]
+            p, _ = softmax_lse((keys @ q) * scale, axis=0)
+            out[b, i] = p @ v
+    return out
+
+
+def mla_decode_absorbed(q_c, q_r, w_uk, w_uv, cache, kv_lens, scale: float,
+                        rope_base: float, page_table=None, page_size: int = 0):
+    """The absorbed path in float64: absorb_query -> latent_attention -> apply_wuv.
+    Returns (out [B, n_h, d_h], latent [B, n_h, d_c], lse [B, n_h])."""
+    d_latent = np.asarray(w_uk).shape[2]
+    q_abs = absorb_query(q_c, q_r, w_uk, kv_lens, rope_base)
+    latent, lse = latent_attention(q_abs, cache, kv_lens, scale, page_table, page_size,
+                                   d_latent=d_latent)
+    return apply_wuv(latent, w_uv), latent, lse

@@ -1,0 +1,321 @@
+"""Pins of the fp64 oracle to facts the pages and the mathematics fix (CPU only).
+
+Each test is chosen so that a plausible slip in the oracle (a dropped k^R term, a
+transposed W_UK, a wrong RoPE sign or frequency, a softmax over the wrong axis, a
+page-table index error) fails at least one of them; test_planted_mistakes_are_caught
+plants such slips and checks exactly that.
+"""
+
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import mla_oracle as om
+from tests import _bruteforce
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "cache_sizes.txt")
+
+
+def _golden():
+    vals = {}
+    with open(GOLDEN) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, value, tol = line.split()[:3]
+            vals[key] = (float(value), float(tol))
+    return vals
+
+
+def _tiny(seed=0, B=2, H=2, d_h=4, d_c=8, d_r=4, L=(5, 3), scale=0.37, base=10.0):
+    rng = np.random.default_rng(seed)
+    Lmax = max(L)
+    return dict(
+        q_c=rng.standard_normal((B, H, d_h)), q_r=rng.standard_normal((B, H, d_r)),
+        w_uk=rng.standard_normal((H, d_h, d_c)), w_uv=rng.standard_normal((H, d_h, d_c)),
+        cache=rng.standard_normal((B, Lmax, d_c + d_r)), kv_lens=np.array(L),
+        scale=scale, rope_base=base)
+
+
+# --- cache arithmetic ------------------------------------------------------------
+
+def test_cache_closed_forms_match_printed_figures():
+    g = _golden()
+    mha = oracle.mha_cache_elements_per_token(128, 128)
+    mla = oracle.mla_cache_elements_per_token(512, 64)
+
+    def close(key, got):
+        v, tol = g[key]
+        assert abs(got - v) <= tol, (key, got, v)
+
+    close("mha_elements_per_token_per_layer", mha)
+    close("mla_elements_per_token_per_layer", mla)
+    close("mha_elements_per_token_60_layers", mha * 60)
+    close("mla_elements_per_token_60_layers", mla * 60)
+    close("mha_over_mla_ratio", mha / mla)
+    close("mla_cache_in_units_of_d_h", mla / 128)
+    close("mha_bytes_per_token_per_layer_bf16", oracle.kv_cache_bytes(1, 1, mha, 2))
+    close("mha_request_bytes_128k_60_layers", oracle.kv_cache_bytes(131072, 60, mha))
+    close("mla_request_bytes_128k_60_layers", oracle.kv_cache_bytes(131072, 60, mla))
+    # d_c = 4 d_h and d_h^R = d_h / 2 give the 2.25-group GQA equivalence (2 * 2.25 d_h)
+    assert mla == 2 * 2.25 * 128
+
+
+# --- RoPE --------------------------------------------------------------------------
+
+def test_rope_identity_at_position_zero_and_off_switch():
+    x = np.random.default_rng(1).standard_normal(64)
+    np.testing.assert_array_equal(oracle.rope_rotate(x, 0, 10000.0), x)
+    np.testing.assert_array_equal(oracle.rope_rotate(x, 12345, 0.0), x)
+
+
+def test_rope_matches_complex_product_and_preserves_norm():
+    rng = np.random.default_rng(2)
+    for pos in (1, 7, 4095, 131071):
+        x = rng.standard_normal(64)
+        y = oracle.rope_rotate(x, pos, 10000.0)
+        z = (x[0::2] + 1j * x[1::2]) * np.exp(1j * pos * 10000.0 ** (-np.arange(32) / 32.0))
+        np.testing.assert_allclose(y[0::2], z.real, atol=1e-12)
+        np.testing.assert_allclose(y[1::2], z.imag, atol=1e-12)
+        assert abs(np.linalg.norm(y) - np.linalg.norm(x)) < 1e-12
+
+
+def test_rope_first_pair_turns_by_one_radian_per_position():
+    # theta_0 = base^0 = 1: position p turns the first pair by p radians; the second pair
+    # turns by base^(-2/64) radians per position (10000^(-1/32) = 0.74989420933245...).
+    e0 = np.zeros(64)
+    e0[0] = 1.0
+    y = oracle.rope_rotate(e0, 1, 10000.0)
+    assert abs(y[0] - 0.5403023058681398) < 1e-15 and abs(y[1] - 0.8414709848078965) < 1e-15
+    e1 = np.zeros(64)
+    e1[2] = 1.0
+    y = oracle.rope_rotate(e1, 1, 10000.0)
+    assert abs(math.atan2(y[3], y[2]) - 0.7498942093324559) < 1e-14
+
+
+def test_rope_scores_depend_only_on_relative_position():
+    rng = np.random.default_rng(3)
+    q, k = rng.standard_normal(64), rng.standard_normal(64)
+    ref = oracle.rope_rotate(q, 100, 10000.0) @ oracle.rope_rotate(k, 37, 10000.0)
+    for shift in (-37, 5, 1000, 50000):
+        got = oracle.rope_rotate(q, 100 + shift, 10000.0) @ oracle.rope_rotate(k, 37 + shift, 10000.0)
+        assert abs(got - ref) < 1e-9
+
+
+# --- softmax -----------------------------------------------------------------------
+
+def test_softmax_rows_sum_to_one_shift_invariance_and_lse():
+    rng = np.random.default_rng(4)
+    s = rng.standard_normal((37, 5)) * 20
+    p, lse = oracle.softmax_lse(s, axis=0)
+    np.testing.assert_allclose(p.sum(axis=0), 1.0, atol=1e-14)
+    p2, lse2 = oracle.softmax_lse(s + 123.0, axis=0)
+    np.testing.assert_allclose(p2, p, atol=1e-14)
+    np.testing.assert_allclose(lse2, lse + 123.0, atol=1e-12)
+    for h in range(5):
+        direct = math.log(math.fsum(math.exp(v) for v in s[:, h]))
+        assert abs(lse[h] - direct) < 1e-12
+    _, lse_empty = oracle.softmax_lse(np.zeros((0, 3)), axis=0)
+    assert np.all(np.isneginf(lse_empty))
+
+
+# --- the decode step -----------------------------------------------------------------
+
+def test_absorbed_equals_nonabsorbed_tiny():
+    """The absorption identity q.(W_UK c) = (W_UK^T q).c, through the whole step
+    (DeepSeek-V2 walkthrough section 2.3 displayed equation; section 6 check 2)."""
+    t = _tiny()
+    ref = oracle.mla_decode_nonabsorbed(**t)
+    out, latent, lse = oracle.mla_decode_absorbed(**t)
+    assert np.max(np.abs(out - ref)) <= 1e-12 * max(1.0, np.max(np.abs(ref)))
+    # the latent output, up-projected, is the head output
+    np.testing.assert_allclose(oracle.apply_wuv(latent, t["w_uv"]), ref, atol=1e-12)
+
+
+def test_score_identity_per_token():
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal(128)
+    w = rng.standard_normal((128, 512))
+    c = rng.standard_normal(512)
+    q_abs = oracle.absorb_query(q[None, None], np.zeros((1, 1, 64)), w[None],
+                                np.array([1]), 0.0)[0, 0, :512]
+    assert abs(q @ (w @ c) - q_abs @ c) < 1e-10 * np.abs(q).sum() * np.abs(w).max() * 10
+
+
+def _bruteforce_case(paged):
+    rng = np.random.default_rng(6)
+    B, H, L = 2, 2, [5, 3]
+    q_c = rng.standard_normal((B, H, 128))
+    q_r = rng.standard_normal((B, H, 64))
+    w_uk = rng.standard_normal((H, 128, 512)) / math.sqrt(512)
+    w_uv = rng.standard_normal((H, 128, 512)) / math.sqrt(512)
+    logical = [rng.standard_normal((n, 576)) for n in L]
+    if not paged:
+        cache = np.full((B, max(L), 576), np.nan)
+        for b in range(B):
+            cache[b, :L[b]] = logical[b]
+        pt, ps = None, 0
+    else:
+        ps = 2
+        npages = [(n + ps - 1) // ps for n in L]
+        total = sum(npages) + 1
+        perm = rng.permutation(total)
+        cache = np.full((total, ps, 576), np.nan)
+        pt = np.full((B, 3), -1)
+        off = 0
+        for b in range(B):
+            for k in range(npages[b]):
+                page = perm[off + k]
+                pt[b, k] = page
+                for s in range(ps):
+                    j = k * ps + s
+                    if j < L[b]:
+                        cache[page, s] = logical[b][j]
+            off += npages[b]
+    return q_c, q_r, w_uk, w_uv, cache, np.array(L), pt, ps, logical
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_bruteforce_python_loops_agree(paged):
+    q_c, q_r, w_uk, w_uv, cache, L, pt, ps, logical = _bruteforce_case(paged)
+    scale = 1 / math.sqrt(192)
+    ref, ref_lse = _bruteforce.decode(q_c.tolist(), q_r.tolist(), w_uk.tolist(), w_uv.tolist(),
+                                      lambda b: logical[b].tolist(), L.tolist(), scale, 10000.0)
+    got = oracle.mla_decode_nonabsorbed(q_c, q_r, w_uk, w_uv, cache, L, scale, 10000.0, pt, ps)
+    np.testing.assert_allclose(got, np.array(ref), atol=1e-12)
+    out, _, lse = oracle.mla_decode_absorbed(q_c, q_r, w_uk, w_uv, cache, L, scale, 10000.0, pt, ps)
+    np.testing.assert_allclose(out, np.array(ref), atol=1e-12)
+    np.testing.assert_allclose(lse, np.array(ref_lse), atol=1e-12)
+
+
+def test_one_token_gives_the_up_projected_latent():
+    t = _tiny(L=(1, 1))
+    out = oracle.mla_decode_nonabsorbed(**t)
+    for b in range(2):
+        for i in range(2):
+            np.testing.assert_allclose(out[b, i], t["w_uv"][i] @ t["cache"][b, 0, :8], atol=1e-13)
+
+
+def test_zero_query_gives_the_mean_latent():
+    t = _tiny()
+    t["q_c"][:] = 0.0
+    t["q_r"][:] = 0.0
+    out = oracle.mla_decode_nonabsorbed(**t)
+    for b, L in enumerate(t["kv_lens"]):
+        mean_c = t["cache"][b, :L, :8].mean(axis=0)
+        for i in range(2):
+            np.testing.assert_allclose(out[b, i], t["w_uv"][i] @ mean_c, atol=1e-13)
+
+
+def test_identical_rows_make_the_query_irrelevant():
+    t = _tiny()
+    t["cache"][:] = t["cache"][:, :1, :]
+    out = oracle.mla_decode_nonabsorbed(**t)
+    for b in range(2):
+        for i in range(2):
+            np.testing.assert_allclose(out[b, i], t["w_uv"][i] @ t["cache"][b, 0, :8], atol=1e-12)
+
+
+def test_zero_position_query_ignores_the_rope_key():
+    """DeepSeek-V2 walkthrough section 5.2: with the position path zeroed, the output no
+    longer depends on the positional key."""
+    t = _tiny()
+    t["q_r"][:] = 0.0
+    a = oracle.mla_decode_nonabsorbed(**t)
+    t["cache"][:, :, 8:] = np.random.default_rng(9).standard_normal(t["cache"][:, :, 8:].shape)
+    b = oracle.mla_decode_nonabsorbed(**t)
+    np.testing.assert_allclose(a, b, atol=1e-14)
+    # and with the position path live, the positional key does matter
+    t2 = _tiny()
+    a2 = oracle.mla_decode_nonabsorbed(**t2)
+    # (a per-token change: adding one vector to every k^R shifts all of a head's scores
+    # equally, which the softmax ignores)
+    t2["cache"][:, :, 8:] += np.random.default_rng(11).standard_normal(t2["cache"][:, :, 8:].shape)
+    assert np.max(np.abs(oracle.mla_decode_nonabsorbed(**t2) - a2)) > 1e-3
+
+
+def test_empty_sequence_and_unread_rows():
+    t = _tiny(L=(4, 0))
+    t["cache"][0, 4:] = np.nan          # rows past kv_len are never read
+    out = oracle.mla_decode_nonabsorbed(**t)
+    assert np.all(np.isfinite(out))
+    np.testing.assert_array_equal(out[1], 0.0)
+    _, latent, lse = oracle.mla_decode_absorbed(**t)
+    np.testing.assert_array_equal(latent[1], 0.0)
+    assert np.all(np.isneginf(lse[1])) and np.all(np.isfinite(lse[0]))
+
+
+def test_paged_layout_equals_contiguous():
+    q_c, q_r, w_uk, w_uv, cache_p, L, pt, ps, logical = _bruteforce_case(True)
+    cache_c = np.full((2, 5, 576), np.nan)
+    for b in range(2):
+        cache_c[b, :L[b]] = logical[b]
+    s = 1 / math.sqrt(192)
+    a = oracle.mla_decode_nonabsorbed(q_c, q_r, w_uk, w_uv, cache_p, L, s, 10000.0, pt, ps)
+    b = oracle.mla_decode_nonabsorbed(q_c, q_r, w_uk, w_uv, cache_c, L, s, 10000.0)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_scale_gives_unit_variance_scores_on_the_workload_distributions():
+    """With the workloads' distributions (weights std 1/sqrt(512), inputs N(0,1)) the
+    scaled scores have variance (128*512/512 + 64)/192 = 1."""
+    rng = np.random.default_rng(10)
+    H, L = 8, 4000
+    q_c = rng.standard_normal((1, H, 128))
+    q_r = rng.standard_normal((1, H, 64))
+    w_uk = rng.standard_normal((H, 128, 512)) / math.sqrt(512)
+    cache = rng.standard_normal((1, L, 576))
+    q_abs = oracle.absorb_query(q_c, q_r, w_uk, np.array([L]), 10000.0)
+    s = (cache[0] @ q_abs[0].T) * oracle.default_scale()
+    assert 0.85 < s.var() < 1.15
+
+
+def test_bf16_widening_is_exact():
+    vals = np.array([1.0, -2.5, 3.140625, 2.0 ** -100, -1.5 * 2.0 ** 120], dtype=np.float32)
+    bits = (vals.view(np.uint32) >> 16).astype(np.uint16)
+    np.testing.assert_array_equal(oracle.widen(bits), vals.astype(np.float64))
+
+
+# --- the pins above catch plausible slips -------------------------------------------
+
+def test_planted_mistakes_are_caught(monkeypatch):
+    """Plant typical slips into the oracle (CPU only) and check that the brute-force
+    cross-check notices each one."""
+    q_c, q_r, w_uk, w_uv, cache, L, pt, ps, logical = _bruteforce_case(True)
+    scale = 1 / math.sqrt(192)
+    ref, _ = _bruteforce.decode(q_c.tolist(), q_r.tolist(), w_uk.tolist(), w_uv.tolist(),
+                                lambda b: logical[b].tolist(), L.tolist(), scale, 10000.0)
+    ref = np.array(ref)
+    good_rotate, good_rows = om.rope_rotate, om.token_rows
+
+    def wrong_sign(x, pos, base):
+        return good_rotate(x, -pos, base)
+
+    def off_by_one(x, pos, base):
+        return good_rotate(x, pos + 1, base)
+
+    def wrong_slot(cache, b, kv_len, page_table=None, page_size=0):
+        # slot index off by one inside each page (the order of the rows alone would not
+        # matter: attention does not depend on the order of its keys)
+        j = np.arange(kv_len)
+        return om.widen(np.asarray(cache)[np.asarray(page_table)[b, j // page_size],
+                                          (j + 1) % page_size, :])
+
+    def no_rope_key(cache, b, kv_len, page_table=None, page_size=0):
+        r = good_rows(cache, b, kv_len, page_table, page_size)
+        r[:, 512:] = 0.0
+        return r
+
+    for name, fn in [("rope_rotate", wrong_sign), ("rope_rotate", off_by_one),
+                     ("token_rows", wrong_slot), ("token_rows", no_rope_key)]:
+        with monkeypatch.context() as m:
+            m.setattr(om, name, fn)
+            got = om.mla_decode_nonabsorbed(q_c, q_r, w_uk, w_uv, cache, L, scale, 10000.0, pt, ps)
+        assert not np.allclose(got, ref, atol=1e-6), f"planted {fn.__name__} not caught"
+    # the two up-projections swapped (W_UK where W_UV belongs)
+    got = om.mla_decode_nonabsorbed(q_c, q_r, w_uk, w_uk, cache, L, scale, 10000.0, pt, ps)
+    assert not np.allclose(got, ref, atol=1e-6)

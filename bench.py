@@ -1,0 +1,448 @@
+"""Benchmark of the MLA absorbed-decode step on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch: query absorption + RoPE, the
+split-KV decode attention over the latent cache (plan, split kernel, combine), and the W_UV
+up-projection, through the C ABI. Inputs are resident in HBM before the timed region;
+every step reads a different one of several cache copies whose total exceeds L2 four times,
+so no step finds its cache in L2. Multi-GPU (torchrun, one process per GPU): every rank runs
+its own replica of the workload (sequences are independent; no data-path collective), the
+timing is the max over ranks, and `value` counts the tokens of all ranks (weak scaling).
+
+--impl reference times the fp64 CPU oracle on the host cores (rank 0 only), each step one
+(sequence, head) output of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mla_latent_kv_28_b200 import workloads as wl  # noqa: E402
+
+METRIC = "MLA decode tokens/s & latent-KV GB/s on 1 B200; % of binding roofline"
+DEFAULT_WORKLOAD = "v2_b32_l4096"
+L2_BYTES = 126 * 2**20
+ROW_BYTES = 576 * 2
+KERNEL_SOURCES = ["decode_split.cu", "decode_simple.cu", "tcgen05.cuh"]
+
+
+# --------------------------------------------------------------------------- ranks
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world: int, local: int, backend: str):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        kw = {}
+        if backend == "nccl":
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120), **kw)
+    return dist
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The max of x over all ranks (the timing rule for multi-GPU numbers)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, local: int, cuda: bool):
+    if world > 1:
+        import torch.distributed as dist
+        if cuda:
+            dist.barrier(device_ids=[local])
+        else:
+            dist.barrier()
+
+
+def replica_seed(rank: int) -> int:
+    """Each rank draws its own replica of the workload."""
+    return rank
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML every few ms on a thread."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.ok = False
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.ok = True
+        except Exception as e:  # NVML missing: report no clocks rather than guess
+            self.err = repr(e)
+        self.period = period_s
+        self.t = threading.Thread(target=self._run, daemon=True)
+
+    def _handle(self, idx):
+        nv = self.nv
+        try:
+            p = torch.cuda.get_device_properties(idx)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            if vis:
+                idx = int(vis.split(",")[idx])
+            return nv.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = int(self._reasons(self.h))
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t.start()
+
+    def stop(self):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        win = [s for s in self.samples if t0 <= s[0] <= t1] or self.samples[-3:]
+        reasons = set()
+        for _, _, rs in win:
+            for bit, name in self.REASONS.items():
+                if rs & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[1] for s in win) if win else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons), "samples": len(win)}
+
+
+# --------------------------------------------------------------------------- roofline
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def kernel_sources_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mla_latent_kv_28_b200", "csrc")
+    for name in KERNEL_SOURCES:
+        p = os.path.join(csrc, name)
+        if os.path.exists(p):
+            with open(p, "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on the
+    current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"decode_attn_{workload}.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_sources_sha") != kernel_sources_sha():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def _np(t):
+    """torch tensor -> numpy; bf16 as uint16 bit patterns (the oracle widens them)."""
+    import numpy as np
+    t = t.detach().cpu()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+def workload_np(w):
+    return dict(q_c=_np(w.q_c), q_r=_np(w.q_r), w_uk=_np(w.w_uk), w_uv=_np(w.w_uv),
+                cache=_np(w.cache), kv_lens=_np(w.kv_lens),
+                page_table=None if w.page_table is None else _np(w.page_table),
+                page_size=w.page_size)
+
+
+def oracle_tokens_per_s(w, budget_s: float = 15.0, max_tokens: int = 4):
+    """Time the fp64 oracle (non-absorbed definition) on whole decode tokens: every head of
+    sequence 0, then 1, ... until the budget is spent. Returns (tokens/s, tokens, seconds)."""
+    import oracle
+    a = workload_np(w)
+    scale = oracle.default_scale()
+    done, t0 = 0, time.perf_counter()
+    for b in range(min(max_tokens, w.batch)):
+        pairs = [(b, i) for i in range(w.n_heads)]
+        oracle.mla_decode_nonabsorbed(a["q_c"], a["q_r"], a["w_uk"], a["w_uv"], a["cache"],
+                                      a["kv_lens"], scale, w.rope_base, a["page_table"],
+                                      a["page_size"], pairs=pairs)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done / dt, done, dt
+
+
+def blas_threads() -> int:
+    try:
+        import numpy  # noqa: F401
+        from threadpoolctl import threadpool_info
+        n = [d["num_threads"] for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args):
+    rank, world, local = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    w = wl.config_workload(args.workload, seed=0)
+    a = workload_np(w)
+    scale = oracle.default_scale()
+    pairs = [(b, i) for b in range(w.batch) for i in range(w.n_heads)]
+
+    def one(k):
+        b, i = pairs[k % len(pairs)]
+        oracle.mla_decode_nonabsorbed(a["q_c"], a["q_r"], a["w_uk"], a["w_uv"], a["cache"],
+                                      a["kv_lens"], scale, w.rope_base, a["page_table"],
+                                      a["page_size"], pairs=[(b, i)])
+    for k in range(args.warmup):
+        one(k)
+    t0 = time.perf_counter()
+    for k in range(args.steps):
+        one(args.warmup + k)
+    dt = time.perf_counter() - t0
+    tokens = args.steps / w.n_heads
+    value = tokens / dt
+    cores = blas_threads()
+    sample = (f"{args.steps} (sequence, head) outputs of {args.workload}, one per step "
+              f"({w.n_heads} make one decode token)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, args.workload),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- ours
+def workload_config(w, name):
+    lens = w.kv_lens
+    return {"workload": name, "batch": w.batch, "n_heads": w.n_heads,
+            "kv_len": int(lens[0]) if bool((lens == lens[0]).all()) else
+            f"ragged {int(lens.min())}..{int(lens.max())}",
+            "cached_tokens_per_gpu": w.cached_tokens,
+            "layout": f"paged {w.page_size}" if w.page_size else "contiguous",
+            "rope_base": w.rope_base, "d_c": 512, "d_rope": 64, "d_head": 128}
+
+
+def run_ours(args):
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, local, "nccl")
+    from mla_latent_kv_28_b200 import binding
+
+    w = wl.config_workload(args.workload, seed=replica_seed(rank))
+    g = w.to(dev)
+    cache_bytes = w.cached_tokens * ROW_BYTES              # algorithmic bytes per step
+    alloc_bytes = g.cache.numel() * g.cache.element_size()
+    copies = max(1, math.ceil(4 * L2_BYTES / alloc_bytes))
+    caches = [g.cache] + [g.cache.clone() for _ in range(copies - 1)]
+
+    h = binding.MlaDecode(w.n_heads, w.batch, w.max_kv_len, page_size=w.page_size,
+                          rope_base=w.rope_base)
+    B, H = w.batch, w.n_heads
+    bufs = {"q_abs": torch.empty((B, H, 576), dtype=torch.bfloat16, device=dev),
+            "latent": torch.empty((B, H, 512), dtype=torch.bfloat16, device=dev),
+            "out": torch.empty((B, H, 128), dtype=torch.bfloat16, device=dev)}
+    stream = torch.cuda.current_stream(dev)
+
+    def step(k, ev=None):
+        q_abs = h.absorb_q(g.q_c, g.q_r, g.w_uk, g.kv_lens, bufs["q_abs"], stream)
+        if ev is not None:
+            ev[0].record(stream)
+        h.decode_attn(q_abs, caches[k % copies], g.kv_lens, g.page_table, bufs["latent"],
+                      None, want_lse=False, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        h.apply_wuv(bufs["latent"], g.w_uv, bufs["out"], stream)
+
+    for k in range(args.warmup):
+        step(k)
+    h.check_device_errors(stream)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, local, True)
+    torch.cuda.synchronize(dev)
+    w0 = time.perf_counter()
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(k, attn_ev[k])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    w1 = time.perf_counter()
+    barrier(world, local, True)
+    h.check_device_errors(stream)
+    ms = t_start.elapsed_time(t_end) / args.steps
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in attn_ev)
+    ms_max = max_over_ranks(ms, world, dev)
+
+    # end to end through the public API: per step the step's inputs come from pinned host
+    # memory and the head outputs go back to pinned host memory
+    hq_c = g.q_c.cpu().pin_memory()
+    hq_r = g.q_r.cpu().pin_memory()
+    hlens = g.kv_lens.cpu().pin_memory()
+    hout = torch.empty((B, H, 128), dtype=torch.bfloat16).pin_memory()
+    dq_c, dq_r, dlens = torch.empty_like(g.q_c), torch.empty_like(g.q_r), torch.empty_like(g.kv_lens)
+    h2d = hq_c.numel() * 2 + hq_r.numel() * 2 + hlens.numel() * 4
+    d2h = hout.numel() * 2
+
+    def e2e_step(k):
+        dq_c.copy_(hq_c, non_blocking=True)
+        dq_r.copy_(hq_r, non_blocking=True)
+        dlens.copy_(hlens, non_blocking=True)
+        out = h.step(dq_c, dq_r, g.w_uk, g.w_uv, caches[k % copies], dlens, g.page_table,
+                     stream, bufs)
+        hout.copy_(out, non_blocking=True)
+
+    for k in range(args.warmup):
+        e2e_step(k)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, local, True)
+    torch.cuda.synchronize(dev)
+    e_start.record(stream)
+    for k in range(args.steps):
+        e2e_step(k)
+    e_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, local, True)
+    h.check_device_errors(stream)
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / args.steps, world, dev)
+    clocks.stop()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, toks, secs = oracle_tokens_per_s(w)
+        cpu = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{toks} decode token(s) of {args.workload} (all {H} heads of sequences "
+                         f"0..{toks - 1}, non-absorbed fp64), {secs:.1f} s"}
+
+    hbm_gbs, bf16_tf, peak_kind = measured_peaks()
+    achieved = cache_bytes / (attn_ms * 1e-3) / 1e9
+    value = world * B / (ms_max * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; workload shapes of the DeepSeek-V2 MLA layer)",
+        "config": dict(workload_config(w, args.workload),
+                       l2=f"inputs larger than L2: {copies} rotating cache copies of "
+                          f"{alloc_bytes / 1e6:.0f} MB per GPU, one per step",
+                       parallelism=f"replicas x{world} (one per GPU, no data-path collective)"),
+        "kv_gbs": world * cache_bytes / (ms_max * 1e-3) / 1e9,
+        "attn_us": attn_ms * 1e3,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                     "frac": achieved / hbm_gbs, "traffic": profiled_traffic(args.workload),
+                     "kernel": "mla_decode_attn (plan + split-KV + combine)",
+                     "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes": cache_bytes,
+                     "tensor_frac_of_measured": (cache_bytes / ROW_BYTES * 2 * 1088 * H)
+                     / (attn_ms * 1e-3) / (bf16_tf * 1e12)},
+        "e2e": {"value": world * B / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 5 * args.steps,
+        "clocks": clocks.summary(w0, w1),
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    h.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wl.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, world, _ = dist_env()
+    if world != args.gpus and not (world == 1 and args.gpus == 1):
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    return run_reference(args) if args.impl == "reference" else run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,157 @@
+/*
+ * mla_decode.h — C ABI of the B200 (sm_100a) MLA absorbed-decode library.
+ *
+ * The operation is the decode step of DeepSeek-V2's Multi-head Latent Attention with
+ * weight absorption. Sources, by page title and section:
+ *   [V2-walk]  "DeepSeek-V2 paper walkthrough" (2kiu.com/news/6085339): §2.3 matrix
+ *              absorption (displayed equation), §2.4 decoupled RoPE.
+ *   [V2-arch]  "Transformer-15: DeepSeek-V2 architecture" (zeeklog.com): MHA equations,
+ *              eqs. 9-11 (c^KV, k^C = W^UK c^KV, v^C = W^UV c^KV), cache table.
+ *   [V2-notes] "DeepSeek-V2" paper notes (process-cxr.github.io): shared k^R, cache of
+ *              d_c + d_h^R values per token.
+ *   [V3-walk]  "DeepSeek-V3 technical report walkthrough" (2kiu.com/news/6340724):
+ *              §2.2 only c^KV and k^R are cached, §2.3 absorption and RoPE.
+ *
+ * Shapes: n_h heads (1..128), d_h = 128, d_c = 512, d_R = d_h^R = 64; one cache row is
+ * [c^KV (512) ; k^R (64)] = 576 bf16 values, one copy for all heads. bf16 means IEEE
+ * bfloat16; every bf16 output is rounded to nearest-even from fp32.
+ *
+ * Conventions for every call:
+ *   - Memory: the caller owns every input and output buffer; all of them are DEVICE
+ *     pointers on the handle's device unless stated. The handle owns only its workspace
+ *     (split partials, work list, device error word), allocated in mla_decode_create;
+ *     the compute calls never allocate.
+ *   - Asynchrony: every compute call enqueues kernels on `stream` and returns at once.
+ *     The returned status covers argument checks and launch errors only. A device-side
+ *     problem (a page-table entry out of range, a bounded wait that ran out) sets the
+ *     handle's device error word; read it with mla_check_device_errors.
+ *   - Threads: a handle may be used by one stream at a time (its workspace is shared by
+ *     the calls enqueued on it).
+ *   - Alignment: every pointer must be 16-byte aligned.
+ *   - Status codes are the MLA_* values below; mla_status_string names them.
+ */
+#ifndef MLA_DECODE_H
+#define MLA_DECODE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct mla_decode_s* mla_handle_t;
+typedef struct CUstream_st* mla_stream_t; /* same object as cudaStream_t; NULL = legacy default stream */
+
+enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = -1,  /* a pointer, size or layout argument is invalid          */
+  MLA_ERR_UNSUPPORTED = -2,  /* valid, but outside what this build implements           */
+  MLA_ERR_CUDA = -3,         /* a CUDA runtime/driver call failed (launch, alloc, ...)  */
+  MLA_ERR_OOM = -4,          /* workspace allocation failed in mla_decode_create        */
+  MLA_ERR_DEVICE_CHECK = -5  /* the device error word was set (bad page id, timeout)    */
+};
+
+typedef struct {
+  int32_t n_heads;       /* n_h, 1..128                                               */
+  int32_t d_head;        /* d_h, must be 128                                          */
+  int32_t d_latent;      /* d_c, must be 512                                          */
+  int32_t d_rope;        /* d_h^R, must be 64                                         */
+  int32_t page_size;     /* 0 = contiguous cache; else tokens per page, must be 64    */
+  int32_t max_batch;     /* largest batch any call will pass (>= 1)                   */
+  int64_t max_kv_len;    /* largest kv_len any call will pass (>= 1)                  */
+  float softmax_scale;   /* 0 => 1/sqrt(d_h + d_h^R) = 1/sqrt(192)                    */
+  float rope_base;       /* RoPE base (10000 for DeepSeek-V2); 0 => q^R not rotated   */
+  int32_t max_splits;    /* upper bound on KV splits per sequence; 0 => automatic     */
+} mla_config_t;
+
+/*
+ * Check a configuration without touching any GPU: MLA_OK if mla_decode_create would accept
+ * it, else the status it would return (MLA_ERR_INVALID_ARG / MLA_ERR_UNSUPPORTED).
+ */
+int mla_check_config(const mla_config_t* cfg);
+
+/*
+ * Create a handle on CUDA device `device` and allocate its workspace there (sized from
+ * cfg->max_batch, cfg->max_kv_len and n_heads). On success *out is the handle and the
+ * return is MLA_OK; on failure *out is NULL. Makes `device` current on the calling thread.
+ */
+int mla_decode_create(const mla_config_t* cfg, int device, mla_handle_t* out);
+
+/* Free the workspace and the handle. Synchronises the device first. NULL is a no-op. */
+int mla_destroy(mla_handle_t h);
+
+/*
+ * Query absorption and RoPE ([V2-walk] §2.3 displayed equation: q^T W_UK c = (W_UK^T q)^T c;
+ * [V3-walk] §2.3; [V2-walk] §2.4 decoupled query):
+ *   q_abs[b,i,0:512]   = W_UK,i^T q^C_{b,i}                     (fp32 accumulation)
+ *   q_abs[b,i,512:576] = RoPE_{kv_lens[b]-1}(q^R_{b,i})         (pairs (2m,2m+1),
+ *                        angle (kv_len-1) * base^(-2m/64); identity if rope_base == 0)
+ * q_c   bf16 [batch, n_h, 128]  the content query (W^UQ c^Q, computed upstream)
+ * q_r   bf16 [batch, n_h, 64]   the decoupled query, not yet rotated
+ * w_uk  bf16 [n_h, 128, 512]    W_UK,i maps a latent (512) to head i's content key (128);
+ *                               this is the nn.Linear weight [n_h*128, 512] reshaped
+ * kv_lens int32 [batch]         cached tokens per sequence (the new token included); the
+ *                               query sits at position kv_lens[b]-1 (0 if kv_lens[b] == 0)
+ * q_abs bf16 [batch, n_h, 576]  output
+ * Errors: MLA_ERR_INVALID_ARG for NULL pointers or batch outside 1..max_batch.
+ */
+int mla_absorb_q(mla_handle_t h, int32_t batch, const void* q_c, const void* q_r,
+                 const void* w_uk, const int32_t* kv_lens, void* q_abs, mla_stream_t stream);
+
+/*
+ * Split-KV decode attention over the shared latent cache ([V2-walk] §2.3: the weighted
+ * sum stays in the latent space; [V2-notes] shared k^R; [V3-walk] §2.2 cached rows):
+ *   s_{b,i,j}  = scale * q_abs[b,i,:] . [c^KV_j ; k^R_j]          j = 0 .. kv_lens[b]-1
+ *   out_latent[b,i,:] = sum_j softmax_j(s)_j c^KV_j                (512, bf16)
+ *   lse[b,i]   = log sum_j exp(s_{b,i,j})                         (natural log, fp32)
+ * q_abs  bf16 [batch, n_h, 576] (from mla_absorb_q)
+ * c_kv   bf16 cache rows, row r at c_kv + r*row_stride (512 values each)
+ * k_r    bf16 cache rows, row r at k_r + r*row_stride (64 values each); the usual fused
+ *        layout is k_r = c_kv + 512 with row_stride = 576
+ * row_stride  elements between consecutive rows; a multiple of 8, >= 512
+ * seq_stride  contiguous cache (page_size 0): token j of sequence b is row b*seq_stride+j,
+ *             seq_stride >= max kv_len; ignored for a paged cache
+ * kv_lens int32 [batch], each 0..max_kv_len. kv_len 0 gives latent 0 and lse = -inf.
+ * page_table  paged cache only (else NULL): int32 [batch, max_pages]; token j of sequence b
+ *             is row page_table[b*max_pages + j/page_size]*page_size + j%page_size. Only the
+ *             first ceil(kv_len/page_size) entries of a row are read. An entry outside
+ *             0..num_pages-1 sets the device error word; its tokens are skipped.
+ * max_pages, num_pages  table width and physical pages in the pool (paged only)
+ * out_latent bf16 [batch, n_h, 512]  output
+ * lse   fp32 [batch, n_h] output, or NULL to skip
+ * Errors: MLA_ERR_INVALID_ARG for NULL pointers, bad strides or alignment, a page table
+ * given to a contiguous handle (or missing for a paged one), max_pages too small for
+ * max_kv_len.
+ */
+int mla_decode_attn(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
+                    const void* k_r, int64_t row_stride, int64_t seq_stride,
+                    const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                    int32_t num_pages, void* out_latent, float* lse, mla_stream_t stream);
+
+/*
+ * V up-projection ([V2-walk] §2.3: W_UV is applied last; [V2-arch] eq. 11 v^C = W^UV c^KV):
+ *   out[b,i,:] = W_UV,i latent[b,i,:]                               (fp32 accumulation)
+ * latent bf16 [batch, n_h, 512]; w_uv bf16 [n_h, 128, 512]; out bf16 [batch, n_h, 128].
+ */
+int mla_apply_wuv(mla_handle_t h, int32_t batch, const void* latent, const void* w_uv,
+                  void* out, mla_stream_t stream);
+
+/*
+ * Synchronise `stream`, then read and clear the handle's device error word. Returns MLA_OK
+ * if it was clear, MLA_ERR_DEVICE_CHECK if a kernel set it (*detail, if not NULL, gets the
+ * word: bit 0 = page-table entry out of range, bit 1 = a bounded wait ran out), or
+ * MLA_ERR_CUDA if the synchronisation itself failed.
+ */
+int mla_check_device_errors(mla_handle_t h, mla_stream_t stream, uint32_t* detail);
+
+/* Bytes of device workspace the handle holds. */
+int64_t mla_workspace_bytes(mla_handle_t h);
+
+/* A static, human-readable name for a status code. */
+const char* mla_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_DECODE_H */

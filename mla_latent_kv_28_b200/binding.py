@@ -1,0 +1,237 @@
+"""ctypes binding of libmla_decode.so (include/mla_decode.h).
+
+Argument marshalling only: tensors are passed as raw device pointers with their strides,
+and every step of the decode path runs in the library's CUDA kernels. torch is used for
+device memory and streams. Loading fails loudly if the library has not been built.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla_decode.so")
+
+MLA_OK = 0
+MLA_ERR_INVALID_ARG = -1
+MLA_ERR_UNSUPPORTED = -2
+MLA_ERR_CUDA = -3
+MLA_ERR_OOM = -4
+MLA_ERR_DEVICE_CHECK = -5
+
+ERR_BAD_PAGE = 1 << 0
+ERR_TIMEOUT = 1 << 1
+ERR_BAD_KV_LEN = 1 << 2
+
+ROW = 576
+D_LATENT = 512
+
+
+class MlaConfig(ctypes.Structure):
+    _fields_ = [
+        ("n_heads", ctypes.c_int32),
+        ("d_head", ctypes.c_int32),
+        ("d_latent", ctypes.c_int32),
+        ("d_rope", ctypes.c_int32),
+        ("page_size", ctypes.c_int32),
+        ("max_batch", ctypes.c_int32),
+        ("max_kv_len", ctypes.c_int64),
+        ("softmax_scale", ctypes.c_float),
+        ("rope_base", ctypes.c_float),
+        ("max_splits", ctypes.c_int32),
+    ]
+
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+
+# name -> (restype, argtypes); every function include/mla_decode.h declares
+SIGNATURES = {
+    "mla_check_config": (ctypes.c_int, [ctypes.POINTER(MlaConfig)]),
+    "mla_decode_create": (ctypes.c_int, [ctypes.POINTER(MlaConfig), ctypes.c_int, ctypes.POINTER(_P)]),
+    "mla_destroy": (ctypes.c_int, [_P]),
+    "mla_absorb_q": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P, _P, _P]),
+    "mla_decode_attn": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32, _P, _P, _P]),
+    "mla_apply_wuv": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P]),
+    "mla_check_device_errors": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
+    "mla_workspace_bytes": (ctypes.c_int64, [_P]),
+    "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+}
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libmla_decode.so once and declare its functions."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build the CUDA library first "
+            "(python -m mla_latent_kv_28_b200.build, or __graft_entry__.build())")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+class MlaError(RuntimeError):
+    def __init__(self, status: int, what: str, detail: int = 0):
+        name = load_library().mla_status_string(status).decode()
+        super().__init__(f"{what}: {name} ({status})" + (f", device error word {detail:#x}" if detail else ""))
+        self.status = status
+        self.detail = detail
+
+
+def _check(status: int, what: str) -> None:
+    if status != MLA_OK:
+        raise MlaError(status, what)
+
+
+def make_config(n_heads: int, max_batch: int, max_kv_len: int, page_size: int = 0,
+                softmax_scale: float = 0.0, rope_base: float = 10000.0,
+                max_splits: int = 0) -> MlaConfig:
+    return MlaConfig(n_heads, 128, 512, 64, page_size, max_batch, max_kv_len,
+                     softmax_scale, rope_base, max_splits)
+
+
+def check_config(cfg: MlaConfig) -> int:
+    return load_library().mla_check_config(ctypes.byref(cfg))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype, name: str) -> None:
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor, got "
+                         f"{t.dtype} on {t.device} (contiguous={t.is_contiguous()})")
+
+
+class MlaDecode:
+    """One handle of the library: its configuration plus its device workspace."""
+
+    def __init__(self, n_heads: int, max_batch: int, max_kv_len: int, page_size: int = 0,
+                 softmax_scale: float = 0.0, rope_base: float = 10000.0, max_splits: int = 0,
+                 device: Optional[int] = None):
+        self._lib = load_library()
+        self.cfg = make_config(n_heads, max_batch, max_kv_len, page_size, softmax_scale,
+                               rope_base, max_splits)
+        self.device = torch.cuda.current_device() if device is None else int(device)
+        h = ctypes.c_void_p()
+        _check(self._lib.mla_decode_create(ctypes.byref(self.cfg), self.device, ctypes.byref(h)),
+               "mla_decode_create")
+        self._h = h
+
+    # -- lifetime ----------------------------------------------------------------------
+    def close(self) -> None:
+        if getattr(self, "_h", None) is not None and self._h.value is not None:
+            _check(self._lib.mla_destroy(self._h), "mla_destroy")
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    @property
+    def workspace_bytes(self) -> int:
+        return int(self._lib.mla_workspace_bytes(self._h))
+
+    # -- the three steps ---------------------------------------------------------------
+    def absorb_q(self, q_c: torch.Tensor, q_r: torch.Tensor, w_uk: torch.Tensor,
+                 kv_lens: torch.Tensor, q_abs: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+        B, H = q_c.shape[0], q_c.shape[1]
+        for t, n in ((q_c, "q_c"), (q_r, "q_r"), (w_uk, "w_uk")):
+            _need(t, torch.bfloat16, n)
+        _need(kv_lens, torch.int32, "kv_lens")
+        if q_abs is None:
+            q_abs = torch.empty((B, H, ROW), dtype=torch.bfloat16, device=q_c.device)
+        _need(q_abs, torch.bfloat16, "q_abs")
+        _check(self._lib.mla_absorb_q(self._h, B, _ptr(q_c), _ptr(q_r), _ptr(w_uk), _ptr(kv_lens),
+                                      _ptr(q_abs), _stream(stream)), "mla_absorb_q")
+        return q_abs
+
+    def decode_attn(self, q_abs: torch.Tensor, cache: torch.Tensor, kv_lens: torch.Tensor,
+                    page_table: Optional[torch.Tensor] = None,
+                    out_latent: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                    want_lse: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+        """cache: contiguous [B, Lmax, 576] or paged [num_pages, page_size, 576] bf16 rows
+        [c^KV ; k^R]. Returns (out_latent [B, n_h, 512] bf16, lse [B, n_h] fp32 or None)."""
+        B, H = q_abs.shape[0], q_abs.shape[1]
+        _need(q_abs, torch.bfloat16, "q_abs")
+        _need(kv_lens, torch.int32, "kv_lens")
+        if not cache.is_cuda or cache.dtype != torch.bfloat16 or cache.dim() != 3 or cache.stride(-1) != 1:
+            raise ValueError("cache: expected a CUDA bf16 [*, *, 576] tensor with unit inner stride")
+        row_stride = cache.stride(1)
+        seq_stride = cache.stride(0) // row_stride
+        c_kv = cache.data_ptr()
+        k_r = c_kv + D_LATENT * cache.element_size()
+        max_pages = num_pages = 0
+        if page_table is not None:
+            _need(page_table, torch.int32, "page_table")
+            max_pages = page_table.shape[1]
+            num_pages = cache.shape[0]
+            seq_stride = 0
+        if out_latent is None:
+            out_latent = torch.empty((B, H, D_LATENT), dtype=torch.bfloat16, device=q_abs.device)
+        if lse is None and want_lse:
+            lse = torch.empty((B, H), dtype=torch.float32, device=q_abs.device)
+        _check(self._lib.mla_decode_attn(
+            self._h, B, _ptr(q_abs), ctypes.c_void_p(c_kv), ctypes.c_void_p(k_r), row_stride,
+            seq_stride, _ptr(kv_lens), _ptr(page_table), max_pages, num_pages, _ptr(out_latent),
+            _ptr(lse), _stream(stream)), "mla_decode_attn")
+        return out_latent, lse
+
+    def apply_wuv(self, latent: torch.Tensor, w_uv: torch.Tensor,
+                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        B, H = latent.shape[0], latent.shape[1]
+        _need(latent, torch.bfloat16, "latent")
+        _need(w_uv, torch.bfloat16, "w_uv")
+        if out is None:
+            out = torch.empty((B, H, 128), dtype=torch.bfloat16, device=latent.device)
+        _need(out, torch.bfloat16, "out")
+        _check(self._lib.mla_apply_wuv(self._h, B, _ptr(latent), _ptr(w_uv), _ptr(out),
+                                       _stream(stream)), "mla_apply_wuv")
+        return out
+
+    def step(self, q_c, q_r, w_uk, w_uv, cache, kv_lens, page_table=None, stream=None,
+             bufs: Optional[dict] = None):
+        """One decode step: absorb -> split-KV attention -> W_UV. Returns the head
+        outputs [B, n_h, 128] bf16. `bufs` may hold preallocated q_abs / latent / out."""
+        bufs = bufs or {}
+        q_abs = self.absorb_q(q_c, q_r, w_uk, kv_lens, bufs.get("q_abs"), stream)
+        latent, _ = self.decode_attn(q_abs, cache, kv_lens, page_table, bufs.get("latent"),
+                                     bufs.get("lse"), want_lse=False, stream=stream)
+        return self.apply_wuv(latent, w_uv, bufs.get("out"), stream)
+
+    def check_device_errors(self, stream=None) -> int:
+        """Synchronise the stream; raise MlaError if a kernel set the device error word."""
+        word = ctypes.c_uint32(0)
+        st = self._lib.mla_check_device_errors(self._h, _stream(stream), ctypes.byref(word))
+        if st != MLA_OK:
+            raise MlaError(st, "device check", int(word.value))
+        return 0

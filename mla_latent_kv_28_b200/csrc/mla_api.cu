@@ -1,0 +1,206 @@
+// The C ABI of libmla_decode.so: argument checks, the workspace, and the launches.
+// Every compute call validates on the host, then enqueues kernels on the caller's stream;
+// nothing here allocates after mla_decode_create.
+#include <cmath>
+#include <cstring>
+#include <new>
+
+#include "mla_internal.cuh"
+
+namespace {
+
+using mla::kDHead;
+using mla::kDLatent;
+using mla::kDRope;
+
+constexpr int kCacheAlign = 16;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & (kCacheAlign - 1)) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int config_status(const mla_config_t* c) {
+  if (c == nullptr) return MLA_ERR_INVALID_ARG;
+  if (c->n_heads < 1 || c->max_batch < 1 || c->max_kv_len < 1 || c->max_splits < 0 ||
+      c->page_size < 0 || !(c->softmax_scale >= 0.f) || !std::isfinite(c->softmax_scale) ||
+      !(c->rope_base >= 0.f) || !std::isfinite(c->rope_base))
+    return MLA_ERR_INVALID_ARG;
+  if (c->d_head != kDHead || c->d_latent != kDLatent || c->d_rope != kDRope)
+    return MLA_ERR_UNSUPPORTED;
+  if (c->n_heads > mla::kMaxHeads || c->max_batch > mla::kMaxBatch) return MLA_ERR_UNSUPPORTED;
+  if (c->page_size != 0 && c->page_size != 64) return MLA_ERR_UNSUPPORTED;
+  if (c->max_kv_len > (int64_t)1 << 30) return MLA_ERR_UNSUPPORTED;
+  if (c->max_splits > 64) return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_status_string(int status) {
+  switch (status) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_OOM: return "MLA_ERR_OOM";
+    case MLA_ERR_DEVICE_CHECK: return "MLA_ERR_DEVICE_CHECK";
+    default: return "MLA_ERR_UNKNOWN";
+  }
+}
+
+int mla_check_config(const mla_config_t* cfg) { return config_status(cfg); }
+
+int mla_decode_create(const mla_config_t* cfg, int device, mla_handle_t* out) {
+  if (out == nullptr) return MLA_ERR_INVALID_ARG;
+  *out = nullptr;
+  const int st = config_status(cfg);
+  if (st != MLA_OK) return st;
+  if (cudaSetDevice(device) != cudaSuccess) return MLA_ERR_CUDA;
+  int major = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (major != 10) return MLA_ERR_UNSUPPORTED;  // built for sm_100a only
+
+  mla_decode_s* h = new (std::nothrow) mla_decode_s;
+  if (h == nullptr) return MLA_ERR_OOM;
+  h->cfg = *cfg;
+  h->device = device;
+  h->num_sms = sms;
+  h->scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale
+                                      : (float)(1.0 / std::sqrt((double)(kDHead + kDRope)));
+  h->units = sms;
+
+  const int B = cfg->max_batch;
+  const int max_units = cfg->max_splits > 0 ? B * cfg->max_splits : h->units;
+  const int max_slots = max_units + B;
+  size_t off = 0;
+  const size_t o_err = off;       off = round_up(off + 4, 256);
+  const size_t o_hdr = off;       off = round_up(off + 4 * 4, 256);
+  const size_t o_seq_tile = off;  off = round_up(off + 4 * (B + 1), 256);
+  const size_t o_seq_slot = off;  off = round_up(off + 4 * (B + 1), 256);
+  const size_t o_seq_len = off;   off = round_up(off + 4 * B, 256);
+  const size_t o_seq_unit = off;  off = round_up(off + 4 * B, 256);
+  const size_t o_ubegin = off;    off = round_up(off + 4 * (max_units + 1), 256);
+  const size_t o_useq = off;      off = round_up(off + 4 * max_units, 256);
+  const size_t o_plse = off;      off = round_up(off + 4 * (size_t)max_slots * cfg->n_heads, 256);
+  const size_t o_po = off;        off = round_up(off + 4 * (size_t)max_slots * cfg->n_heads * kDLatent, 256);
+
+  void* base = nullptr;
+  if (cudaMalloc(&base, off) != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return MLA_ERR_OOM;
+  }
+  if (cudaMemset(base, 0, off) != cudaSuccess) {
+    cudaFree(base);
+    delete h;
+    return MLA_ERR_CUDA;
+  }
+  char* p = static_cast<char*>(base);
+  h->ws.base = base;
+  h->ws.bytes = off;
+  h->ws.err = reinterpret_cast<uint32_t*>(p + o_err);
+  h->ws.plan.header = reinterpret_cast<int32_t*>(p + o_hdr);
+  h->ws.plan.seq_tile = reinterpret_cast<int32_t*>(p + o_seq_tile);
+  h->ws.plan.seq_slot = reinterpret_cast<int32_t*>(p + o_seq_slot);
+  h->ws.plan.seq_len = reinterpret_cast<int32_t*>(p + o_seq_len);
+  h->ws.plan.seq_unit = reinterpret_cast<int32_t*>(p + o_seq_unit);
+  h->ws.plan.unit_begin = reinterpret_cast<int32_t*>(p + o_ubegin);
+  h->ws.plan.unit_seq = reinterpret_cast<int32_t*>(p + o_useq);
+  h->ws.part_lse = reinterpret_cast<float*>(p + o_plse);
+  h->ws.part_o = reinterpret_cast<float*>(p + o_po);
+  h->ws.max_units = max_units;
+  h->ws.max_slots = max_slots;
+  *out = h;
+  return MLA_OK;
+}
+
+int mla_destroy(mla_handle_t h) {
+  if (h == nullptr) return MLA_OK;
+  int st = MLA_OK;
+  if (cudaSetDevice(h->device) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+    st = MLA_ERR_CUDA;
+  if (h->ws.base != nullptr && cudaFree(h->ws.base) != cudaSuccess) st = MLA_ERR_CUDA;
+  delete h;
+  return st;
+}
+
+int64_t mla_workspace_bytes(mla_handle_t h) { return h == nullptr ? -1 : (int64_t)h->ws.bytes; }
+
+int mla_absorb_q(mla_handle_t h, int32_t batch, const void* q_c, const void* q_r,
+                 const void* w_uk, const int32_t* kv_lens, void* q_abs, mla_stream_t stream) {
+  if (h == nullptr || q_c == nullptr || q_r == nullptr || w_uk == nullptr ||
+      kv_lens == nullptr || q_abs == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > h->cfg.max_batch) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_c) || !aligned16(q_r) || !aligned16(w_uk) || !aligned16(q_abs))
+    return MLA_ERR_INVALID_ARG;
+  const cudaError_t e = mla::launch_absorb_q(
+      *h, batch, static_cast<const __nv_bfloat16*>(q_c), static_cast<const __nv_bfloat16*>(q_r),
+      static_cast<const __nv_bfloat16*>(w_uk), kv_lens, static_cast<__nv_bfloat16*>(q_abs), stream);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_decode_attn(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
+                    const void* k_r, int64_t row_stride, int64_t seq_stride,
+                    const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                    int32_t num_pages, void* out_latent, float* lse, mla_stream_t stream) {
+  if (h == nullptr || q_abs == nullptr || c_kv == nullptr || k_r == nullptr ||
+      kv_lens == nullptr || out_latent == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > h->cfg.max_batch) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_abs) || !aligned16(c_kv) || !aligned16(k_r) || !aligned16(out_latent) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3) != 0))
+    return MLA_ERR_INVALID_ARG;
+  if (row_stride < kDLatent || row_stride % 8 != 0) return MLA_ERR_INVALID_ARG;
+  mla::CacheView cv{};
+  cv.c_kv = static_cast<const __nv_bfloat16*>(c_kv);
+  cv.k_r = static_cast<const __nv_bfloat16*>(k_r);
+  cv.row_stride = row_stride;
+  cv.page_size = h->cfg.page_size;
+  if (h->cfg.page_size == 0) {
+    if (page_table != nullptr || seq_stride < h->cfg.max_kv_len) return MLA_ERR_INVALID_ARG;
+    cv.seq_stride = seq_stride;
+  } else {
+    const int64_t need = (h->cfg.max_kv_len + h->cfg.page_size - 1) / h->cfg.page_size;
+    if (page_table == nullptr || max_pages < need || num_pages < 1) return MLA_ERR_INVALID_ARG;
+    cv.page_table = page_table;
+    cv.max_pages = max_pages;
+    cv.num_pages = num_pages;
+  }
+  cudaError_t e = mla::launch_split_plan(*h, batch, kv_lens, stream);
+  if (e == cudaSuccess)
+    e = mla::launch_decode_split(*h, batch, static_cast<const __nv_bfloat16*>(q_abs), cv, stream);
+  if (e == cudaSuccess)
+    e = mla::launch_combine(*h, batch, static_cast<__nv_bfloat16*>(out_latent), lse, stream);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_apply_wuv(mla_handle_t h, int32_t batch, const void* latent, const void* w_uv,
+                  void* out, mla_stream_t stream) {
+  if (h == nullptr || latent == nullptr || w_uv == nullptr || out == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > h->cfg.max_batch) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(latent) || !aligned16(w_uv) || !aligned16(out)) return MLA_ERR_INVALID_ARG;
+  const cudaError_t e = mla::launch_apply_wuv(
+      *h, batch, static_cast<const __nv_bfloat16*>(latent),
+      static_cast<const __nv_bfloat16*>(w_uv), static_cast<__nv_bfloat16*>(out), stream);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_check_device_errors(mla_handle_t h, mla_stream_t stream, uint32_t* detail) {
+  if (h == nullptr) return MLA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MLA_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, h->ws.err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (detail != nullptr) *detail = word;
+  if (word == 0) return MLA_OK;
+  if (cudaMemset(h->ws.err, 0, sizeof(word)) != cudaSuccess) return MLA_ERR_CUDA;
+  return MLA_ERR_DEVICE_CHECK;
+}
+
+}  // extern "C"

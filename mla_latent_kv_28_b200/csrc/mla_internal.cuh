@@ -1,0 +1,94 @@
+// Internal declarations shared by the kernels and the C-ABI layer of libmla_decode.so.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/mla_decode.h"
+
+namespace mla {
+
+constexpr int kDHead = 128;    // d_h
+constexpr int kDLatent = 512;  // d_c
+constexpr int kDRope = 64;     // d_h^R
+constexpr int kRow = kDLatent + kDRope;  // one cache row: [c^KV ; k^R]
+constexpr int kMaxHeads = 128;
+constexpr int kMaxBatch = 1024;
+constexpr int kTileTokens = 64;  // tokens per KV tile: the unit of the work plan
+
+// Device error word bits (see mla_check_device_errors).
+constexpr uint32_t kErrBadPage = 1u << 0;
+constexpr uint32_t kErrTimeout = 1u << 1;
+constexpr uint32_t kErrBadKvLen = 1u << 2;
+
+// Work plan, written on the device by the plan kernel from kv_lens, read by the decode
+// and combine kernels. The cache tokens of all sequences, cut into 64-token tiles and laid
+// end to end (sequence 0's tiles first), form one "tile space" of `total_tiles` tiles.
+// A unit is a contiguous range of that space [unit_begin[u], unit_begin[u+1]); the decode
+// kernel's CTAs (or CTA pairs) take units in turn. A unit may span several sequences; each
+// (unit, sequence) overlap is a segment with its own partial-result slot. The slots of
+// sequence b are seq_slot[b] .. seq_slot[b+1]-1, in token order.
+struct PlanView {
+  int32_t* header;      // [0] total_tiles, [1] n_units
+  int32_t* seq_tile;    // [B+1]  first tile of each sequence (prefix sum of tiles)
+  int32_t* seq_slot;    // [B+1]  first slot of each sequence
+  int32_t* seq_len;     // [B]    kv_len as used (clamped to 0..max_kv_len)
+  int32_t* seq_unit;    // [B]    the unit that holds the sequence's first tile
+  int32_t* unit_begin;  // [max_units+1]
+  int32_t* unit_seq;    // [max_units] first sequence that unit u touches
+};
+
+struct Workspace {
+  void* base = nullptr;
+  size_t bytes = 0;
+  uint32_t* err = nullptr;   // device error word
+  PlanView plan{};
+  float* part_o = nullptr;   // [max_slots, n_h, 512] partial latent outputs (normalised)
+  float* part_lse = nullptr; // [max_slots, n_h]     their log-sum-exp
+  int max_units = 0;
+  int max_slots = 0;
+};
+
+}  // namespace mla
+
+struct mla_decode_s {
+  mla_config_t cfg;
+  int device = 0;
+  int num_sms = 0;
+  float scale = 0.f;
+  int units = 0;  // units the balanced plan cuts the tile space into
+  mla::Workspace ws;
+};
+
+namespace mla {
+
+// Launchers (each returns the cudaGetLastError() of its launch).
+cudaError_t launch_absorb_q(const mla_decode_s& h, int batch, const __nv_bfloat16* q_c,
+                            const __nv_bfloat16* q_r, const __nv_bfloat16* w_uk,
+                            const int32_t* kv_lens, __nv_bfloat16* q_abs, cudaStream_t s);
+
+cudaError_t launch_split_plan(const mla_decode_s& h, int batch, const int32_t* kv_lens,
+                              cudaStream_t s);
+
+struct CacheView {
+  const __nv_bfloat16* c_kv;
+  const __nv_bfloat16* k_r;
+  int64_t row_stride;   // elements between rows
+  int64_t seq_stride;   // contiguous layout: rows between sequences
+  const int32_t* page_table;  // nullptr = contiguous
+  int32_t max_pages;
+  int32_t num_pages;
+  int32_t page_size;
+};
+
+cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfloat16* q_abs,
+                                const CacheView& cache, cudaStream_t s);
+
+cudaError_t launch_combine(const mla_decode_s& h, int batch, __nv_bfloat16* out_latent,
+                           float* lse, cudaStream_t s);
+
+cudaError_t launch_apply_wuv(const mla_decode_s& h, int batch, const __nv_bfloat16* latent,
+                             const __nv_bfloat16* w_uv, __nv_bfloat16* out, cudaStream_t s);
+
+}  // namespace mla

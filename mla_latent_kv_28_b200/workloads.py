@@ -173,3 +173,19 @@ CONFIGS = {
 def config_workload(name: str, seed: int = 0) -> Workload:
     kw = dict(CONFIGS[name])
     return make_workload(seed=seed, name=name, **kw)
+
+
+def draw_q_abs(batch: int, n_heads: int, seed: int = 1) -> torch.Tensor:
+    """A stand-alone absorbed-query input [B, n_h, 576] bf16 for testing the attention call
+    by itself: the first 512 values N(0, 0.5^2) (the spread of W_UK^T q^C under the weight
+    recipe above), the last 64 N(0, 1)."""
+    gen = torch.Generator().manual_seed(seed)
+    q = torch.randn((batch, n_heads, ROW), generator=gen)
+    q[..., :D_LATENT] *= 0.5
+    return q.to(torch.bfloat16)
+
+
+def draw_latent(batch: int, n_heads: int, seed: int = 2) -> torch.Tensor:
+    """A stand-alone latent input [B, n_h, 512] bf16 ~ N(0, 1) for testing the W_UV call."""
+    gen = torch.Generator().manual_seed(seed)
+    return torch.randn((batch, n_heads, D_LATENT), generator=gen).to(torch.bfloat16)

@@ -137,9 +137,42 @@ int mla_apply_wuv(mla_handle_t h, int32_t batch, const void* latent, const void*
                   void* out, mla_stream_t stream);
 
 /*
+ * mla_decode_attn for callers that cannot allocate device memory. The pages have no
+ * counterpart to this call: it exists for library users whose device memory is owned by
+ * someone else (a serving engine that has reserved nearly all of HBM for its own KV-cache
+ * pool and allocates only from it, a plugin host whose memory manager forbids cudaMalloc)
+ * or whose hot path cannot afford cudaMalloc/cudaFree and the synchronisation they may
+ * bring. Such callers cannot create a handle, so the configuration comes as arguments and
+ * the scratch (work plan, split partials, error word) lives in one fixed 32 MiB array of
+ * device memory inside the library, which every GPU that loads the library holds until the
+ * process exits. The call allocates nothing.
+ *
+ * Arguments and results are those of mla_decode_attn, with n_heads, softmax_scale (0 =>
+ * 1/sqrt(192)), page_size (0 or 64) and max_kv_len in place of the handle, and:
+ *   err_word  device uint32, or NULL: set to 0 at the start of the call, then OR-ed with the
+ *             device error bits of mla_check_device_errors; with NULL the bits stay in the
+ *             library's array and are not reported.
+ * Uses the current device. Limits: batch <= 64 and n_heads <= 128; beyond them the call
+ * returns MLA_ERR_UNSUPPORTED and enqueues nothing. The split count adapts to what fits in
+ * the array, so results can differ from mla_decode_attn by floating-point reassociation.
+ * All calls on a device share the array and it keeps the last call's contents: calls whose
+ * kernels overlap on the GPU (different streams or host threads) race, so serialise them.
+ * The first call on a device looks up the array's device address; make it before any
+ * stream capture.
+ */
+int mla_decode_attn_noalloc(int32_t n_heads, float softmax_scale, int32_t page_size,
+                            int64_t max_kv_len, int32_t batch, const void* q_abs,
+                            const void* c_kv, const void* k_r, int64_t row_stride,
+                            int64_t seq_stride, const int32_t* kv_lens,
+                            const int32_t* page_table, int32_t max_pages, int32_t num_pages,
+                            void* out_latent, float* lse, uint32_t* err_word,
+                            mla_stream_t stream);
+
+/*
  * Synchronise `stream`, then read and clear the handle's device error word. Returns MLA_OK
  * if it was clear, MLA_ERR_DEVICE_CHECK if a kernel set it (*detail, if not NULL, gets the
- * word: bit 0 = page-table entry out of range, bit 1 = a bounded wait ran out), or
+ * word: bit 0 = page-table entry out of range, bit 1 = a bounded wait ran out, bit 2 = a
+ * kv_len outside 0..max_kv_len, clamped), or
  * MLA_ERR_CUDA if the synchronisation itself failed.
  */
 int mla_check_device_errors(mla_handle_t h, mla_stream_t stream, uint32_t* detail);

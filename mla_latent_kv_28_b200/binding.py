@@ -57,6 +57,8 @@ SIGNATURES = {
     "mla_absorb_q": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P, _P, _P]),
     "mla_decode_attn": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32, _P, _P, _P]),
     "mla_apply_wuv": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P]),
+    "mla_decode_attn_noalloc": (ctypes.c_int, [_I32, ctypes.c_float, _I32, _I64, _I32, _P, _P, _P,
+                                               _I64, _I64, _P, _P, _I32, _I32, _P, _P, _P, _P]),
     "mla_check_device_errors": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "mla_workspace_bytes": (ctypes.c_int64, [_P]),
     "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),

@@ -38,7 +38,7 @@ METRIC = "MLA decode tokens/s & latent-KV GB/s on 1 B200; % of binding roofline"
 DEFAULT_WORKLOAD = "v2_b32_l4096"
 L2_BYTES = 126 * 2**20
 ROW_BYTES = 576 * 2
-KERNEL_SOURCES = ["decode_split.cu", "decode_simple.cu", "tcgen05.cuh"]
+KERNEL_SOURCES = ["decode_split.cu", "sm100.cuh"]
 
 
 # --------------------------------------------------------------------------- ranks

@@ -1,0 +1,510 @@
+// Split-KV decode attention over the latent cache on the sm_100a tensor core.
+//
+// Per (sequence, split) segment, for all 128 heads at once (heads are the MMA's M = 128):
+//   S = Q_abs [128 x 576] . [c ; k^R]^T [576 x 64 tokens]     (tcgen05, fp32 in TMEM)
+//   online softmax over the tokens (exp2, running max with lazy rescale)
+//   O += P [128 x 64] . c [64 x 512]                            (tcgen05, fp32 in TMEM)
+// and the segment's partial O / l and log-sum-exp go to the split slots.
+//
+// Why a 2-CTA cluster: O alone (128 heads x 512 fp32) is the whole 256 KB of one SM's
+// tensor memory, leaving no room for S. So the two CTAs of a cluster split the 576 columns
+// of every cache row: CTA r holds c^KV columns [256r, 256r+256) and k^R columns
+// [32r, 32r+32) (288 columns), computes the partial scores over them, and keeps the O
+// columns [256r, 256r+256). The two fp32 partial score tiles are swapped through
+// distributed shared memory; both CTAs then add the same two tiles (S0 + S1, bit for bit
+// the same sum) and run the same softmax, so P, the running max and the normaliser agree
+// without any further exchange. Each cache byte is read from HBM once, by one CTA.
+//
+// Tensor memory (512 columns per CTA): O [0,256) fp32, S [256,320) fp32, P [320,352)
+// bf16x2, Q [352,496) bf16x2 (the CTA's 288 query columns, the A operand of Q.K^T).
+// Shared memory: 5 stages x 36 KB of cache tiles (four 64x64 c^KV boxes with 128-byte
+// swizzle + one 64x32 k^R box with 64-byte swizzle), a 32 KB receive buffer for the
+// peer's partial scores, and the mbarriers.
+// Warps: 0 = TMA producer, 1 = MMA issuer (and TMEM owner), 2..5 = softmax / epilogue,
+// one thread per head (TMEM lane).
+//
+// Every wait is bounded: after about a second it sets the device error word (timeout bit)
+// and the CTA's abort flag, all roles leave their loops, wait for their own copies and
+// MMAs in flight, and the CTA frees its tensor memory and exits.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "mla_internal.cuh"
+#include "sm100.cuh"
+
+namespace mla {
+namespace {
+
+using namespace sm100;
+
+constexpr int kT = 64;                    // tokens per tile
+static_assert(kT == kTileTokens, "the plan and the kernel use the same tile");
+constexpr int kStages = 5;
+constexpr int kKSteps = 18;               // 288 columns / 16
+constexpr uint32_t kBoxC = kT * 128;      // 8 KB: 64 tokens x 64 c^KV columns
+constexpr uint32_t kBoxR = kT * 64;       // 4 KB: 64 tokens x 32 k^R columns
+constexpr uint32_t kStageBytes = 4 * kBoxC + kBoxR;   // 36 KB
+constexpr uint32_t kXinBytes = 128 * kT * 4;          // 32 KB
+constexpr uint32_t kOffXin = kStages * kStageBytes;
+constexpr uint32_t kOffBars = kOffXin + kXinBytes;
+constexpr int kNumBars = 2 * kStages + 9;
+constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;
+constexpr uint32_t kSmemUsed = kOffMisc + 64;
+constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;     // room to align the base to 1 KB
+
+constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 320, kTmemQ = 352, kTmemCols = 512;
+constexpr int kThreads = 192;
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kT, false, false);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, false, true);
+constexpr float kRescaleThreshold = 8.f;   // log2 units: rescale O only when the max grows more
+
+// barrier indices
+constexpr int kBarKvFull = 0;                 // [kStages]  TMA landed
+constexpr int kBarKvEmpty = kStages;          // [kStages]  PV of the tile done
+constexpr int kBarSFull = 2 * kStages;        // partial S in TMEM
+constexpr int kBarSEmpty = kBarSFull + 1;     // softmax copied S out
+constexpr int kBarPFull = kBarSFull + 2;      // P in TMEM (and O rescaled, V tail zeroed)
+constexpr int kBarPvDone = kBarSFull + 3;     // PV done (P free, O final)
+constexpr int kBarQReady = kBarSFull + 4;     // Q of the segment in TMEM
+constexpr int kBarXFull = kBarSFull + 5;      // the peer's partial scores arrived
+constexpr int kBarXFree = kBarSFull + 6;      // the peer read what we sent
+constexpr int kBarFinal = kBarSFull + 7;      // all MMAs of this CTA done (teardown)
+
+struct Params {
+  const __nv_bfloat16* q_abs;
+  PlanView plan;
+  int batch, n_heads;
+  int64_t seq_stride;
+  const int32_t* page_table;
+  int max_pages, num_pages;
+  float scale_log2;
+  float* part_o;
+  float* part_lse;
+  uint32_t* err;
+  long long wait_limit;
+};
+
+struct Segment {
+  int b, slot, len, j0, ntiles;
+};
+
+// Visit this cluster's segments in order; f returns false to stop.
+template <class F>
+__device__ __forceinline__ void for_each_segment(const Params& p, F&& f) {
+  const int n_units = p.plan.header[1];
+  for (int u = (int)cluster_id_x(); u < n_units; u += (int)num_clusters_x()) {
+    const int ub = p.plan.unit_begin[u], ue = p.plan.unit_begin[u + 1];
+    for (int b = p.plan.unit_seq[u]; b < p.batch && p.plan.seq_tile[b] < ue; ++b) {
+      const int tb = p.plan.seq_tile[b], te = p.plan.seq_tile[b + 1];
+      if (te <= ub) continue;
+      Segment s;
+      s.b = b;
+      s.len = p.plan.seq_len[b];
+      const int lt0 = max(ub, tb) - tb, lt1 = min(ue, te) - tb;
+      s.j0 = lt0 * kT;
+      s.ntiles = lt1 - lt0;
+      s.slot = p.plan.seq_slot[b] + (u - p.plan.seq_unit[b]);
+      if (!f(s)) return;
+    }
+  }
+}
+
+__device__ __forceinline__ bool wait_teardown(uint32_t bar, uint32_t parity, long long limit) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > limit) return false;
+  return true;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constant__ CUtensorMap tmap_r,
+                const Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bars = sbase + kOffBars;
+  auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  volatile int* tile_valid = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);  // [kStages]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t peer = rank ^ 1u;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(bar(kBarKvFull + i), 1);
+      mbar_init(bar(kBarKvEmpty + i), 1);
+      tile_valid[i] = 0;
+    }
+    mbar_init(bar(kBarSFull), 1);
+    mbar_init(bar(kBarSEmpty), 128);
+    mbar_init(bar(kBarPFull), 128);
+    mbar_init(bar(kBarPvDone), 1);
+    mbar_init(bar(kBarQReady), 128);
+    mbar_init(bar(kBarXFull), 128);
+    mbar_init(bar(kBarXFree), 128);
+    mbar_init(bar(kBarFinal), 1);
+    *abort_flag = 0;
+    fence_mbarrier_init_cluster();
+    prefetch_tmap(&tmap_c);
+    prefetch_tmap(&tmap_r);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  cluster_sync();  // the peer's barriers are initialised before anyone arrives on them
+
+  const WaitGuard guard{abort_flag, p.err, kErrTimeout, p.wait_limit};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t g = 0;
+      for_each_segment(p, [&](const Segment& s) {
+        for (int k = 0; k < s.ntiles; ++k, ++g) {
+          const uint32_t st = g % kStages;
+          if (!wait_bounded(bar(kBarKvEmpty + st), ((g / kStages) & 1u) ^ 1u, guard)) return false;
+          const int j = s.j0 + k * kT;
+          bool ok = true;
+          int64_t row;
+          if (p.page_table != nullptr) {
+            const int32_t page = p.page_table[(int64_t)s.b * p.max_pages + j / kT];
+            ok = page >= 0 && page < p.num_pages;
+            if (!ok) atomicOr(p.err, kErrBadPage);
+            row = (int64_t)page * kT;
+          } else {
+            row = (int64_t)s.b * p.seq_stride + j;
+          }
+          tile_valid[st] = ok ? 1 : 0;
+          const uint32_t dst = sbase + st * kStageBytes;
+          if (ok) {
+            mbar_arrive_expect_tx(bar(kBarKvFull + st), kStageBytes);
+            for (int i = 0; i < 4; ++i)
+              tma_load_2d(dst + i * kBoxC, &tmap_c, 256 * (int)rank + 64 * i, (int)row, bar(kBarKvFull + st));
+            tma_load_2d(dst + 4 * kBoxC, &tmap_r, 32 * (int)rank, (int)row, bar(kBarKvFull + st));
+          } else {
+            mbar_arrive(bar(kBarKvFull + st));
+          }
+        }
+        return true;
+      });
+      // copies still in flight (only after an abort) land before the CTA leaves
+      for (uint32_t i = 0; i < kStages && i < g; ++i) {
+        const uint32_t gi = g - 1 - i;
+        wait_teardown(bar(kBarKvFull + gi % kStages), (gi / kStages) & 1u, p.wait_limit);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t g = 0, seg = 0;
+      auto issue_qk = [&](uint32_t gt) -> bool {
+        const uint32_t st = gt % kStages;
+        if (!wait_bounded(bar(kBarKvFull + st), (gt / kStages) & 1u, guard)) return false;
+        if (!wait_bounded(bar(kBarSEmpty), (gt & 1u) ^ 1u, guard)) return false;
+        tc_fence_after();
+        const uint32_t a = sbase + st * kStageBytes;
+#pragma unroll
+        for (int ks = 0; ks < kKSteps; ++ks) {
+          const uint64_t bd = ks < 16
+              ? smem_desc(a + (ks >> 2) * kBoxC + (ks & 3) * 32, 16, 1024, 2)
+              : smem_desc(a + 4 * kBoxC + (ks - 16) * 32, 16, 512, 4);
+          mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * ks, bd, kIdescQK, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(kBarSFull));
+        return true;
+      };
+      for_each_segment(p, [&](const Segment& s) {
+        if (!wait_bounded(bar(kBarQReady), seg & 1u, guard)) return false;
+        tc_fence_after();
+        if (!issue_qk(g)) return false;
+        for (int k = 0; k < s.ntiles; ++k) {
+          const uint32_t gt = g + k;
+          if (k + 1 < s.ntiles && !issue_qk(gt + 1)) return false;
+          if (!wait_bounded(bar(kBarPFull), gt & 1u, guard)) return false;
+          tc_fence_after();
+          const uint32_t v = sbase + (gt % kStages) * kStageBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(tmem + kTmemO, tmem + kTmemP + 8 * kk, smem_desc(v + kk * 2048, kBoxC, 1024, 2),
+                   kIdescPV, (k > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(kBarKvEmpty + gt % kStages));
+          mma_commit(bar(kBarPvDone));
+        }
+        g += s.ntiles;
+        ++seg;
+        return true;
+      });
+      mma_commit(bar(kBarFinal));
+      wait_teardown(bar(kBarFinal), 0, p.wait_limit);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int quarter = warp & 3;                       // TMEM lanes this warp may touch
+    const int h = 32 * quarter + lane;                  // head = TMEM lane
+    const uint32_t lanes = (uint32_t)(32 * quarter) << 16;
+    const int tid = threadIdx.x - 64;                   // 0..127 among the softmax threads
+    const uint32_t xin = sbase + kOffXin;
+    const uint32_t peer_xin = map_to_rank(xin, peer);
+    const uint32_t peer_xfull = map_to_rank(bar(kBarXFull), peer);
+    const uint32_t peer_xfree = map_to_rank(bar(kBarXFree), peer);
+    const bool head_ok = h < p.n_heads;
+    uint32_t g = 0, seg = 0, nsend = 0, nrecv = 0;
+
+    auto load_s = [&](float (&dst)[kT]) {
+      uint32_t r[32];
+      tmem_ld32_sync(lanes | (tmem + kTmemS), r);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) dst[j] = __uint_as_float(r[j]);
+      tmem_ld32_sync(lanes | (tmem + kTmemS + 32), r);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) dst[32 + j] = __uint_as_float(r[j]);
+    };
+    auto send = [&](const float (&v)[kT]) -> bool {
+      if (!wait_bounded(bar(kBarXFree), (nsend & 1u) ^ 1u, guard, true)) return false;
+      const uint32_t row = peer_xin + (uint32_t)h * (kT * 4);
+#pragma unroll
+      for (int c = 0; c < kT / 4; ++c)
+        st_cluster_v4(row + (uint32_t)((c ^ (h & 7)) * 16), __float_as_uint(v[4 * c]),
+                      __float_as_uint(v[4 * c + 1]), __float_as_uint(v[4 * c + 2]),
+                      __float_as_uint(v[4 * c + 3]));
+      mbar_arrive_remote(peer_xfull);
+      ++nsend;
+      return true;
+    };
+
+    for_each_segment(p, [&](const Segment& s) {
+      // the segment's query columns -> TMEM (A operand of Q.K^T)
+      {
+        const __nv_bfloat16* qrow = p.q_abs + ((int64_t)s.b * p.n_heads + (head_ok ? h : 0)) * kRow;
+#pragma unroll 1
+        for (int grp = 0; grp < kKSteps / 2; ++grp) {
+          uint32_t r[16];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int ci = grp * 4 + i;  // 16-byte chunk 0..35 of this CTA's 288 columns
+            const int col = ci < 32 ? 256 * (int)rank + 8 * ci : kDLatent + 32 * (int)rank + 8 * (ci - 32);
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (head_ok) v = *reinterpret_cast<const uint4*>(qrow + col);
+            r[4 * i] = v.x; r[4 * i + 1] = v.y; r[4 * i + 2] = v.z; r[4 * i + 3] = v.w;
+          }
+          tmem_st16(lanes | (tmem + kTmemQ + 16 * grp), r);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(kBarQReady));
+      }
+
+      float m_used = -INFINITY, l = 0.f;
+      float cur[kT], nxt[kT];
+      if (!wait_bounded(bar(kBarSFull), g & 1u, guard)) return false;
+      tc_fence_after();
+      load_s(cur);
+      tc_fence_before();
+      mbar_arrive(bar(kBarSEmpty));
+      if (!send(cur)) return false;
+
+      for (int k = 0; k < s.ntiles; ++k) {
+        const uint32_t gt = g + k, st = gt % kStages;
+        if (!wait_bounded(bar(kBarKvFull + st), (gt / kStages) & 1u, guard)) return false;
+        const int r = tile_valid[st] ? min(kT, s.len - (s.j0 + k * kT)) : 0;
+        const bool more = k + 1 < s.ntiles;
+        if (more) {
+          if (!wait_bounded(bar(kBarSFull), (gt + 1) & 1u, guard)) return false;
+          tc_fence_after();
+          load_s(nxt);
+          tc_fence_before();
+          mbar_arrive(bar(kBarSEmpty));
+        }
+        // the peer's partial scores of this tile: S = own + peer (same sum on both CTAs)
+        if (!wait_bounded(bar(kBarXFull), nrecv & 1u, guard, true)) return false;
+        {
+          const float4* row = reinterpret_cast<const float4*>(smem + kOffXin + h * (kT * 4));
+#pragma unroll
+          for (int c = 0; c < kT / 4; ++c) {
+            const float4 v = row[c ^ (h & 7)];
+            cur[4 * c] += v.x; cur[4 * c + 1] += v.y; cur[4 * c + 2] += v.z; cur[4 * c + 3] += v.w;
+          }
+        }
+        ++nrecv;
+        mbar_arrive_remote(peer_xfree);
+        if (more && !send(nxt)) return false;
+
+        // online softmax in the log2 domain
+        float mt = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < kT; ++j) {
+          cur[j] = j < r ? cur[j] * p.scale_log2 : -INFINITY;
+          mt = fmaxf(mt, cur[j]);
+        }
+        float alpha = 1.f;
+        bool need = false;
+        if (m_used == -INFINITY) {
+          m_used = mt;
+        } else if (mt > m_used + kRescaleThreshold) {
+          need = true;
+          alpha = exp2f(m_used - mt);
+          m_used = mt;
+          l *= alpha;
+        }
+        uint32_t pk[32];
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < kT; j += 2) {
+          const float p0 = m_used == -INFINITY ? 0.f : exp2f(cur[j] - m_used);
+          const float p1 = m_used == -INFINITY ? 0.f : exp2f(cur[j + 1] - m_used);
+          sum += p0 + p1;
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+          pk[j / 2] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        l += sum;
+        const bool warp_need = __any_sync(0xffffffffu, need);
+
+        // P may be overwritten and O rescaled once the previous PV has finished
+        if (!wait_bounded(bar(kBarPvDone), (gt & 1u) ^ 1u, guard)) return false;
+        tc_fence_after();
+        if (warp_need) {
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t o[32];
+            tmem_ld32_sync(lanes | (tmem + kTmemO + 32 * c), o);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+            tmem_st32(lanes | (tmem + kTmemO + 32 * c), o);
+          }
+        }
+        tmem_st32(lanes | (tmem + kTmemP), pk);
+        tmem_wait_st();
+        if (r < kT) {
+          // rows past the sequence end (or of a skipped page) must not reach P.V as NaN/Inf
+          uint8_t* stage = smem + st * kStageBytes;
+          for (int i = tid; i < (kT - r) * 32; i += 128) {
+            const int row = r + (i >> 5), box = (i >> 3) & 3, chunk = i & 7;
+            *reinterpret_cast<uint4*>(stage + box * kBoxC + row * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        mbar_arrive(bar(kBarPFull));
+#pragma unroll
+        for (int j = 0; j < kT; ++j) cur[j] = nxt[j];
+      }
+
+      // epilogue: O / l and the log-sum-exp of this segment
+      const uint32_t glast = g + s.ntiles - 1;
+      if (!wait_bounded(bar(kBarPvDone), glast & 1u, guard)) return false;
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      float* dst = p.part_o + ((int64_t)s.slot * p.n_heads + (head_ok ? h : 0)) * kDLatent + 256 * rank;
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t o[32];
+        tmem_ld32_sync(lanes | (tmem + kTmemO + 32 * c), o);
+        if (head_ok) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(dst + 32 * c + j) =
+                make_float4(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv,
+                            __uint_as_float(o[j + 2]) * inv, __uint_as_float(o[j + 3]) * inv);
+        }
+      }
+      if (head_ok && rank == 0)
+        p.part_lse[(int64_t)s.slot * p.n_heads + h] =
+            l > 0.f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      tc_fence_before();
+      g += s.ntiles;
+      ++seg;
+      return true;
+    });
+  }
+
+  // teardown: nobody touches the peer's shared memory after this point
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+bool encode_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, int64_t row_stride,
+                 uint32_t box_cols, CUtensorMapSwizzle swz) {
+  const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)row_stride * 2};
+  const cuuint32_t box[2] = {box_cols, (cuuint32_t)kT};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfloat16* q_abs,
+                                const CacheView& cv, cudaStream_t s) {
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(decode_split_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kSmemAlloc);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+
+  const int64_t rows = cv.page_table != nullptr ? (int64_t)cv.num_pages * cv.page_size
+                                                : (int64_t)batch * cv.seq_stride;
+  if (rows <= 0 || rows >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+  CUtensorMap tc, tr;
+  if (!encode_rows(&tc, cv.c_kv, kDLatent, (uint64_t)rows, cv.row_stride, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_rows(&tr, cv.k_r, kDRope, (uint64_t)rows, cv.row_stride, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+
+  Params p{};
+  p.q_abs = q_abs;
+  p.plan = h.ws.plan;
+  p.batch = batch;
+  p.n_heads = h.cfg.n_heads;
+  p.seq_stride = cv.seq_stride;
+  p.page_table = cv.page_table;
+  p.max_pages = cv.max_pages;
+  p.num_pages = cv.num_pages;
+  p.scale_log2 = h.scale * 1.4426950408889634f;
+  p.part_o = h.ws.part_o;
+  p.part_lse = h.ws.part_lse;
+  p.err = h.ws.err;
+  p.wait_limit = 2000000000LL;  // SM cycles, about a second
+
+  const int pairs = std::max(1, std::min(h.units, h.num_sms / 2));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemAlloc;
+  cfg.stream = s;
+  cfg.attrs = nullptr;  // the 2-CTA cluster shape is compiled into the kernel
+  cfg.numAttrs = 0;
+  return cudaLaunchKernelEx(&cfg, decode_split_tc, tc, tr, p);
+}
+
+}  // namespace mla

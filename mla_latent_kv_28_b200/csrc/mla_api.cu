@@ -71,7 +71,7 @@ int mla_decode_create(const mla_config_t* cfg, int device, mla_handle_t* out) {
   h->num_sms = sms;
   h->scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale
                                       : (float)(1.0 / std::sqrt((double)(kDHead + kDRope)));
-  h->units = sms;
+  h->units = sms / 2;  // the decode kernel runs one 2-CTA cluster per unit of work
 
   const int B = cfg->max_batch;
   const int max_units = cfg->max_splits > 0 ? B * cfg->max_splits : h->units;

@@ -1,0 +1,252 @@
+// The two per-head projections of the decode step on the sm_100a tensor core:
+//
+//   absorb (query absorption + RoPE):  q_abs[b,i,0:512]  = W_UK,i^T q^C_{b,i}
+//                                      q_abs[b,i,512:]   = RoPE_{kv_len[b]-1}(q^R_{b,i})
+//   W_UV up-projection:                out[b,i,:]        = W_UV,i latent[b,i,:]
+//
+// Both are a small batch of vectors times one 128x512 bf16 weight matrix per head, so they
+// are bound by reading the weights (16 MiB each at 128 heads). One CTA per (head, batch
+// chunk) pulls its head's 128 KB of weights with TMA, runs the product as tcgen05 MMAs with
+// the weights as the M = 128 operand ("swap AB": M = output features, N = batch), and writes
+// the accumulator back from tensor memory with one thread per output feature, so every
+// store instruction of a warp covers consecutive features of one sequence.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "mla_internal.cuh"
+#include "sm100.cuh"
+
+namespace mla {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 128;
+constexpr uint32_t kWeightBox = 128 * 128;      // 128 rows x 64 columns bf16 = 16 KB
+constexpr uint32_t kWeightBytes = 8 * kWeightBox;  // one head's 128 x 512 matrix
+
+enum Mode { kAbsorb = 0, kUpProject = 1 };
+
+struct GemmParams {
+  int batch, n_heads, n_tile;     // n_tile: sequences per CTA (multiple of 16, <= 128)
+  uint32_t idesc;
+  __nv_bfloat16* out;             // q_abs [B, n_h, 576] or out [B, n_h, 128]
+  const __nv_bfloat16* q_r;       // absorb only
+  const int32_t* kv_lens;         // absorb only
+  double rope_base;
+  uint32_t* err;
+  long long wait_limit;
+};
+
+__device__ __forceinline__ bool wait_simple(uint32_t bar, uint32_t parity, const GemmParams& p) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > p.wait_limit) {
+      atomicOr(p.err, kErrTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+             const GemmParams p) {
+  // MODE kAbsorb:    D[c, b] = sum_d W_UK[h][d][c] x[b][d]   (A = W_UK, M-major; 4 M blocks, K = 128)
+  // MODE kUpProject: D[d, b] = sum_c W_UV[h][d][c] x[b][c]   (A = W_UV, K-major; 1 M block,  K = 512)
+  constexpr int kMBlocks = MODE == kAbsorb ? 4 : 1;
+  constexpr int kXBoxes = MODE == kAbsorb ? 2 : 8;   // 64-column boxes of one x row
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t xbase = sbase + kWeightBytes;
+  const uint32_t xbox = (uint32_t)p.n_tile * 128;        // bytes of one x box
+  const uint32_t bars = xbase + kXBoxes * xbox;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (bars - sbase) + 16);
+  const int h = blockIdx.x, b0 = blockIdx.y * p.n_tile;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // accumulator block mb sits at column mb * col_stride; the epilogue reads 32 columns at a
+  // time, so a block never spans fewer than 32 allocated columns
+  const uint32_t col_stride = p.n_tile < 32 ? 32u : (uint32_t)p.n_tile;
+  const uint32_t need = kMBlocks * col_stride;
+  const uint32_t tmem_cols = need <= 32 ? 32 : need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bars, 1);        // operands landed
+    mbar_init(bars + 8, 1);    // MMAs done
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  bool ok = true;
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(bars, kWeightBytes + kXBoxes * xbox);
+    for (int i = 0; i < 8; ++i) tma_load_2d(sbase + i * kWeightBox, &tmap_w, 64 * i, 128 * h, bars);
+    const int xcol = h * (MODE == kAbsorb ? kDHead : kDLatent);
+    for (int i = 0; i < kXBoxes; ++i) tma_load_2d(xbase + i * xbox, &tmap_x, xcol + 64 * i, b0, bars);
+    ok = wait_simple(bars, 0, p);
+    tc_fence_after();
+    if (ok) {
+#pragma unroll 1
+      for (int mb = 0; mb < kMBlocks; ++mb) {
+#pragma unroll 1
+        for (int kk = 0; kk < (MODE == kAbsorb ? 8 : 32); ++kk) {
+          uint64_t ad, bd;
+          if (MODE == kAbsorb) {
+            // A[c, d]: W_UK box (2mb) holds d rows x 64 c; 16 d rows per K step
+            ad = smem_desc(sbase + 2 * mb * kWeightBox + kk * 2048, kWeightBox, 1024, 2);
+            bd = smem_desc(xbase + (kk >> 2) * xbox + (kk & 3) * 32, 16, 1024, 2);
+          } else {
+            ad = smem_desc(sbase + (kk >> 2) * kWeightBox + (kk & 3) * 32, 16, 1024, 2);
+            bd = smem_desc(xbase + (kk >> 2) * xbox + (kk & 3) * 32, 16, 1024, 2);
+          }
+          mma_ss(tmem + mb * col_stride, ad, bd, p.idesc, kk > 0 ? 1u : 0u);
+        }
+      }
+      mma_commit(bars + 8);
+      ok = wait_simple(bars + 8, 0, p);
+    } else {
+      wait_simple(bars, 0, p);  // never leave with copies in flight
+    }
+    *reinterpret_cast<volatile int*>(smem + (bars - sbase) + 20) = ok ? 1 : 0;
+  }
+  __syncthreads();
+  tc_fence_after();
+  ok = *reinterpret_cast<volatile int*>(smem + (bars - sbase) + 20) != 0;
+
+  // epilogue: TMEM lane = output feature, column = sequence
+  const uint32_t lanes = (uint32_t)(32 * warp) << 16;
+  if (ok) {
+    for (int mb = 0; mb < kMBlocks; ++mb) {
+      for (int c0 = 0; c0 < p.n_tile; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32_sync(lanes | (tmem + mb * col_stride + c0), r);
+        const int feat = 128 * mb + 32 * warp + lane;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int b = b0 + c0 + j;
+          if (c0 + j < p.n_tile && b < p.batch) {
+            const float v = __uint_as_float(r[j]);
+            if (MODE == kAbsorb)
+              p.out[((int64_t)b * p.n_heads + h) * kRow + feat] = __float2bfloat16_rn(v);
+            else
+              p.out[((int64_t)b * p.n_heads + h) * kDHead + feat] = __float2bfloat16_rn(v);
+          }
+        }
+      }
+    }
+  }
+  if (MODE == kAbsorb) {
+    // RoPE of the decoupled query (angles in double: positions reach 2^17)
+    for (int i = threadIdx.x; i < p.n_tile * (kDRope / 2); i += kThreads) {
+      const int b = b0 + i / (kDRope / 2), m = i % (kDRope / 2);
+      if (b >= p.batch) continue;
+      const __nv_bfloat16* src = p.q_r + ((int64_t)b * p.n_heads + h) * kDRope + 2 * m;
+      const double x0 = __bfloat162float(src[0]), x1 = __bfloat162float(src[1]);
+      double y0 = x0, y1 = x1;
+      if (p.rope_base != 0.0) {
+        const int pos = max(p.kv_lens[b] - 1, 0);
+        const double theta = pow(p.rope_base, -2.0 * m / kDRope);
+        double sn, cs;
+        sincos((double)pos * theta, &sn, &cs);
+        y0 = x0 * cs - x1 * sn;
+        y1 = x0 * sn + x1 * cs;
+      }
+      __nv_bfloat16* dst = p.out + ((int64_t)b * p.n_heads + h) * kRow + kDLatent + 2 * m;
+      dst[0] = __double2bfloat16(y0);
+      dst[1] = __double2bfloat16(y1);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, tmem_cols);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// A row-major bf16 matrix [rows, cols] as a TMA source with 64-column, 128-byte-swizzled boxes.
+bool encode(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  const PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t launch(const mla_decode_s& h, int batch, const __nv_bfloat16* w, const __nv_bfloat16* x,
+                   __nv_bfloat16* out, const __nv_bfloat16* q_r, const int32_t* kv_lens,
+                   cudaStream_t s) {
+  constexpr int kXBoxes = MODE == kAbsorb ? 2 : 8;
+  constexpr int kCap = MODE == kAbsorb ? 128 : 64;  // weights + x boxes fit in shared memory
+  const int n_tile = std::min(kCap, (batch + 15) / 16 * 16);
+  const int kx = MODE == kAbsorb ? kDHead : kDLatent;
+  CUtensorMap tw, tx;
+  if (!encode(&tw, w, (uint64_t)h.cfg.n_heads * kDHead, kDLatent, 128) ||
+      !encode(&tx, x, (uint64_t)batch, (uint64_t)h.cfg.n_heads * kx, (uint32_t)n_tile))
+    return cudaErrorInvalidValue;
+  constexpr uint32_t kSmemMax = kWeightBytes + kXBoxes * kCap * 128 + 64 + 1024;
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [] {
+    attr = cudaFuncSetAttribute(head_gemm_tc<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kSmemMax);
+  });
+  if (attr != cudaSuccess) return attr;
+  GemmParams p{};
+  p.batch = batch;
+  p.n_heads = h.cfg.n_heads;
+  p.n_tile = n_tile;
+  p.idesc = idesc_bf16_f32(128, n_tile, MODE == kAbsorb, false);
+  p.out = out;
+  p.q_r = q_r;
+  p.kv_lens = kv_lens;
+  p.rope_base = (double)h.cfg.rope_base;
+  p.err = h.ws.err;
+  p.wait_limit = 2000000000LL;
+  const uint32_t smem = kWeightBytes + kXBoxes * n_tile * 128 + 64 + 1024;
+  dim3 grid(h.cfg.n_heads, (batch + n_tile - 1) / n_tile);
+  head_gemm_tc<MODE><<<grid, kThreads, smem, s>>>(tw, tx, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_absorb_q(const mla_decode_s& h, int batch, const __nv_bfloat16* q_c,
+                            const __nv_bfloat16* q_r, const __nv_bfloat16* w_uk,
+                            const int32_t* kv_lens, __nv_bfloat16* q_abs, cudaStream_t s) {
+  return launch<kAbsorb>(h, batch, w_uk, q_c, q_abs, q_r, kv_lens, s);
+}
+
+cudaError_t launch_apply_wuv(const mla_decode_s& h, int batch, const __nv_bfloat16* latent,
+                             const __nv_bfloat16* w_uv, __nv_bfloat16* out, cudaStream_t s) {
+  return launch<kUpProject>(h, batch, w_uv, latent, out, nullptr, nullptr, s);
+}
+
+}  // namespace mla

@@ -1,9 +1,9 @@
 // Split-KV decode attention over the latent cache on the sm_100a tensor core.
 //
 // Per (sequence, split) segment, for all 128 heads at once (heads are the MMA's M = 128):
-//   S = Q_abs [128 x 576] . [c ; k^R]^T [576 x 64 tokens]     (tcgen05, fp32 in TMEM)
+//   S = Q_abs [128 x 576] . [c ; k^R]^T [576 x 32 tokens]     (tcgen05, fp32 in TMEM)
 //   online softmax over the tokens (exp2, running max with lazy rescale)
-//   O += P [128 x 64] . c [64 x 512]                            (tcgen05, fp32 in TMEM)
+//   O += P [128 x 32] . c [32 x 512]                            (tcgen05, fp32 in TMEM)
 // and the segment's partial O / l and log-sum-exp go to the split slots.
 //
 // Why a 2-CTA cluster: O alone (128 heads x 512 fp32) is the whole 256 KB of one SM's
@@ -11,17 +11,28 @@
 // of every cache row: CTA r holds c^KV columns [256r, 256r+256) and k^R columns
 // [32r, 32r+32) (288 columns), computes the partial scores over them, and keeps the O
 // columns [256r, 256r+256). The two fp32 partial score tiles are swapped through
-// distributed shared memory; both CTAs then add the same two tiles (S0 + S1, bit for bit
-// the same sum) and run the same softmax, so P, the running max and the normaliser agree
-// without any further exchange. Each cache byte is read from HBM once, by one CTA.
+// distributed shared memory (st.async, counted by the receiver's mbarrier); both CTAs then
+// add the same two tiles (S0 + S1, bit for bit the same sum) and run the same softmax, so
+// P, the running max and the normaliser agree without any further exchange. Each cache
+// byte is read from HBM once, by one CTA.
 //
-// Tensor memory (512 columns per CTA): O [0,256) fp32, S [256,320) fp32, P [320,352)
-// bf16x2, Q [352,496) bf16x2 (the CTA's 288 query columns, the A operand of Q.K^T).
-// Shared memory: 5 stages x 36 KB of cache tiles (four 64x64 c^KV boxes with 128-byte
-// swizzle + one 64x32 k^R box with 64-byte swizzle), a 32 KB receive buffer for the
-// peer's partial scores, and the mbarriers.
-// Warps: 0 = TMA producer, 1 = MMA issuer (and TMEM owner), 2..5 = softmax / epilogue,
-// one thread per head (TMEM lane).
+// Pipeline (32-token tiles, g = tile index within this cluster's work):
+//   TMA ring of 10 stages -> QK(g) into S[g%2] -> softmax threads copy S(g+1) out of TMEM
+//   and send it to the peer while they finish tile g with the peer's S(g) -> P(g) into
+//   P[g%2] -> PV(g). The MMA thread issues whichever of QK / PV is ready, so QK runs two
+//   tiles ahead and the tensor core never waits for the exchange round trip.
+// Segment boundaries (a unit may hold the tail of one sequence and the head of the next)
+// are handled by a separate warpgroup: it loads the next segment's query columns into
+// TMEM as soon as the last QK of the previous segment is done, and writes the finished
+// segment's O / l while the next segment is already running.
+//
+// Tensor memory (512 columns per CTA): O [0,256) fp32, S [256,320) 2 x 32 fp32,
+// P [320,352) 2 x 16 bf16x2, Q [352,496) bf16x2 (the CTA's 288 query columns, the A
+// operand of Q.K^T). Shared memory: 10 stages x 18 KB of cache tiles (four 32x64 c^KV
+// boxes with 128-byte swizzle + one 32x32 k^R box with 64-byte swizzle), 2 x 16 KB
+// receive buffers for the peer's partial scores, per-segment (max, sum), mbarriers.
+// Warps: 0 TMA producer, 1 MMA issuer (and TMEM owner), 2..5 softmax (one thread per head
+// = TMEM lane), 6..9 segment transitions (query load, epilogue).
 //
 // Every wait is bounded: after about a second it sets the device error word (timeout bit)
 // and the CTA's abort flag, all roles leave their loops, wait for their own copies and
@@ -39,38 +50,42 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kT = 64;                    // tokens per tile
-static_assert(kT == kTileTokens, "the plan and the kernel use the same tile");
-constexpr int kStages = 5;
+constexpr int kT = 32;                    // tokens per kernel tile (the plan uses 64)
+constexpr int kStages = 10;
 constexpr int kKSteps = 18;               // 288 columns / 16
-constexpr uint32_t kBoxC = kT * 128;      // 8 KB: 64 tokens x 64 c^KV columns
-constexpr uint32_t kBoxR = kT * 64;       // 4 KB: 64 tokens x 32 k^R columns
-constexpr uint32_t kStageBytes = 4 * kBoxC + kBoxR;   // 36 KB
-constexpr uint32_t kXinBytes = 128 * kT * 4;          // 32 KB
+constexpr uint32_t kBoxC = kT * 128;      // 4 KB: 32 tokens x 64 c^KV columns
+constexpr uint32_t kBoxR = kT * 64;       // 2 KB: 32 tokens x 32 k^R columns
+constexpr uint32_t kStageBytes = 4 * kBoxC + kBoxR;   // 18 KB
+constexpr uint32_t kXinBytes = 128 * kT * 4;          // 16 KB: 128 heads x 32 fp32
 constexpr uint32_t kOffXin = kStages * kStageBytes;
-constexpr uint32_t kOffBars = kOffXin + kXinBytes;
-constexpr int kNumBars = 2 * kStages + 9;
+constexpr uint32_t kOffMl = kOffXin + 2 * kXinBytes;  // [2][128] float2 (max, sum)
+constexpr uint32_t kOffBars = kOffMl + 2 * 128 * 8;
+
+// barrier indices
+constexpr int kBarKvFull = 0;                    // [kStages] TMA landed
+constexpr int kBarKvEmpty = kStages;             // [kStages] PV of the tile done
+constexpr int kBarSFull = 2 * kStages;           // [2] partial S in TMEM
+constexpr int kBarSEmpty = kBarSFull + 2;        // [2] softmax copied S out
+constexpr int kBarPFull = kBarSFull + 4;         // [2] P in TMEM (O rescaled, V tail zeroed)
+constexpr int kBarXFull = kBarSFull + 6;         // [2] the peer's partial scores arrived
+constexpr int kBarXFree = kBarSFull + 8;         // [2] the peer has read what we sent
+constexpr int kBarPvDone = kBarSFull + 10;       // a PV finished
+constexpr int kBarQReady = kBarSFull + 11;       // query columns of the next segment in TMEM
+constexpr int kBarQFree = kBarSFull + 12;        // the last QK of a segment finished
+constexpr int kBarOFull = kBarSFull + 13;        // the last PV of a segment finished
+constexpr int kBarOFree = kBarSFull + 14;        // the epilogue has read O
+constexpr int kBarMlFull = kBarSFull + 15;       // (max, sum) of a finished segment in smem
+constexpr int kBarFinal = kBarSFull + 16;        // all MMAs of this CTA done (teardown)
+constexpr int kNumBars = kBarFinal + 1;
 constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;
-constexpr uint32_t kSmemUsed = kOffMisc + 64;
+constexpr uint32_t kSmemUsed = kOffMisc + 128;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;     // room to align the base to 1 KB
 
 constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 320, kTmemQ = 352, kTmemCols = 512;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kT, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, false, true);
 constexpr float kRescaleThreshold = 8.f;   // log2 units: rescale O only when the max grows more
-
-// barrier indices
-constexpr int kBarKvFull = 0;                 // [kStages]  TMA landed
-constexpr int kBarKvEmpty = kStages;          // [kStages]  PV of the tile done
-constexpr int kBarSFull = 2 * kStages;        // partial S in TMEM
-constexpr int kBarSEmpty = kBarSFull + 1;     // softmax copied S out
-constexpr int kBarPFull = kBarSFull + 2;      // P in TMEM (and O rescaled, V tail zeroed)
-constexpr int kBarPvDone = kBarSFull + 3;     // PV done (P free, O final)
-constexpr int kBarQReady = kBarSFull + 4;     // Q of the segment in TMEM
-constexpr int kBarXFull = kBarSFull + 5;      // the peer's partial scores arrived
-constexpr int kBarXFree = kBarSFull + 6;      // the peer read what we sent
-constexpr int kBarFinal = kBarSFull + 7;      // all MMAs of this CTA done (teardown)
 
 struct Params {
   const __nv_bfloat16* q_abs;
@@ -86,30 +101,62 @@ struct Params {
   long long wait_limit;
 };
 
-struct Segment {
-  int b, slot, len, j0, ntiles;
-};
+// Walks this cluster's work tile by tile: units in turn, the segments (one sequence's
+// tokens inside a unit) of each unit, and the 32-token tiles of each segment.
+struct TileCursor {
+  int u, b, ub, ue;        // unit, sequence, the unit's plan-tile range
+  int slot, len, j0, j1;   // the segment: partial slot, kv_len, token range [j0, j1)
+  int k, nk;               // tile within the segment, tiles in the segment
+  uint32_t g, seg;         // tile and segment counters of this cluster
+  bool valid;
 
-// Visit this cluster's segments in order; f returns false to stop.
-template <class F>
-__device__ __forceinline__ void for_each_segment(const Params& p, F&& f) {
-  const int n_units = p.plan.header[1];
-  for (int u = (int)cluster_id_x(); u < n_units; u += (int)num_clusters_x()) {
-    const int ub = p.plan.unit_begin[u], ue = p.plan.unit_begin[u + 1];
-    for (int b = p.plan.unit_seq[u]; b < p.batch && p.plan.seq_tile[b] < ue; ++b) {
+  __device__ __forceinline__ bool enter_sequence(const Params& p) {
+    // find the next sequence of the current unit that overlaps it; false if none
+    for (; b < p.batch && p.plan.seq_tile[b] < ue; ++b) {
       const int tb = p.plan.seq_tile[b], te = p.plan.seq_tile[b + 1];
       if (te <= ub) continue;
-      Segment s;
-      s.b = b;
-      s.len = p.plan.seq_len[b];
-      const int lt0 = max(ub, tb) - tb, lt1 = min(ue, te) - tb;
-      s.j0 = lt0 * kT;
-      s.ntiles = lt1 - lt0;
-      s.slot = p.plan.seq_slot[b] + (u - p.plan.seq_unit[b]);
-      if (!f(s)) return;
+      len = p.plan.seq_len[b];
+      j0 = (max(ub, tb) - tb) * kTileTokens;
+      j1 = min((min(ue, te) - tb) * kTileTokens, len);
+      nk = (j1 - j0 + kT - 1) / kT;
+      slot = p.plan.seq_slot[b] + (u - p.plan.seq_unit[b]);
+      k = 0;
+      return true;
     }
+    return false;
   }
-}
+  __device__ __forceinline__ void find(const Params& p) {
+    const int n_units = p.plan.header[1];
+    for (; u < n_units; u += (int)num_clusters_x()) {
+      ub = p.plan.unit_begin[u];
+      ue = p.plan.unit_begin[u + 1];
+      if (enter_sequence(p)) { valid = true; return; }
+      b = u + (int)num_clusters_x() < n_units ? p.plan.unit_seq[u + (int)num_clusters_x()] : 0;
+    }
+    valid = false;
+  }
+  __device__ __forceinline__ void init(const Params& p) {
+    u = (int)cluster_id_x();
+    g = 0;
+    seg = 0;
+    b = u < p.plan.header[1] ? p.plan.unit_seq[u] : 0;
+    find(p);
+  }
+  __device__ __forceinline__ void next(const Params& p) {
+    ++g;
+    if (++k < nk) return;
+    ++seg;
+    ++b;
+    if (enter_sequence(p)) return;
+    u += (int)num_clusters_x();
+    b = u < p.plan.header[1] ? p.plan.unit_seq[u] : 0;
+    find(p);
+  }
+  __device__ __forceinline__ int j() const { return j0 + kT * k; }
+  __device__ __forceinline__ int rows() const { return min(kT, j1 - j()); }
+  __device__ __forceinline__ bool first() const { return k == 0; }
+  __device__ __forceinline__ bool last() const { return k == nk - 1; }
+};
 
 __device__ __forceinline__ bool wait_teardown(uint32_t bar, uint32_t parity, long long limit) {
   const long long t0 = clock64();
@@ -129,6 +176,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   volatile int* tile_valid = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);  // [kStages]
+  float2* ml = reinterpret_cast<float2*>(smem + kOffMl);                             // [2][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -140,15 +188,24 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       mbar_init(bar(kBarKvEmpty + i), 1);
       tile_valid[i] = 0;
     }
-    mbar_init(bar(kBarSFull), 1);
-    mbar_init(bar(kBarSEmpty), 128);
-    mbar_init(bar(kBarPFull), 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kBarSFull + i), 1);
+      mbar_init(bar(kBarSEmpty + i), 128);
+      mbar_init(bar(kBarPFull + i), 128);
+      mbar_init(bar(kBarXFull + i), 1);
+      mbar_init(bar(kBarXFree + i), 4);
+    }
     mbar_init(bar(kBarPvDone), 1);
     mbar_init(bar(kBarQReady), 128);
-    mbar_init(bar(kBarXFull), 128);
-    mbar_init(bar(kBarXFree), 128);
+    mbar_init(bar(kBarQFree), 1);
+    mbar_init(bar(kBarOFull), 1);
+    mbar_init(bar(kBarOFree), 128);
+    mbar_init(bar(kBarMlFull), 128);
     mbar_init(bar(kBarFinal), 1);
     *abort_flag = 0;
+    // the receive buffers expect their first tile of partial scores
+    mbar_arrive_expect_tx(bar(kBarXFull + 0), kXinBytes);
+    mbar_arrive_expect_tx(bar(kBarXFull + 1), kXinBytes);
     fence_mbarrier_init_cluster();
     prefetch_tmap(&tmap_c);
     prefetch_tmap(&tmap_r);
@@ -161,94 +218,106 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  cluster_sync();  // the peer's barriers are initialised before anyone arrives on them
+  cluster_sync();  // the peer's barriers are initialised before anyone signals them
 
   const WaitGuard guard{abort_flag, p.err, kErrTimeout, p.wait_limit};
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t g = 0;
-      for_each_segment(p, [&](const Segment& s) {
-        for (int k = 0; k < s.ntiles; ++k, ++g) {
-          const uint32_t st = g % kStages;
-          if (!wait_bounded(bar(kBarKvEmpty + st), ((g / kStages) & 1u) ^ 1u, guard)) return false;
-          const int j = s.j0 + k * kT;
-          bool ok = true;
-          int64_t row;
-          if (p.page_table != nullptr) {
-            const int32_t page = p.page_table[(int64_t)s.b * p.max_pages + j / kT];
-            ok = page >= 0 && page < p.num_pages;
-            if (!ok) atomicOr(p.err, kErrBadPage);
-            row = (int64_t)page * kT;
-          } else {
-            row = (int64_t)s.b * p.seq_stride + j;
-          }
-          tile_valid[st] = ok ? 1 : 0;
-          const uint32_t dst = sbase + st * kStageBytes;
-          if (ok) {
-            mbar_arrive_expect_tx(bar(kBarKvFull + st), kStageBytes);
-            for (int i = 0; i < 4; ++i)
-              tma_load_2d(dst + i * kBoxC, &tmap_c, 256 * (int)rank + 64 * i, (int)row, bar(kBarKvFull + st));
-            tma_load_2d(dst + 4 * kBoxC, &tmap_r, 32 * (int)rank, (int)row, bar(kBarKvFull + st));
-          } else {
-            mbar_arrive(bar(kBarKvFull + st));
-          }
+      TileCursor c;
+      c.init(p);
+      for (; c.valid; c.next(p)) {
+        const uint32_t g = c.g, st = g % kStages;
+        if (!wait_bounded(bar(kBarKvEmpty + st), ((g / kStages) & 1u) ^ 1u, guard)) break;
+        const int j = c.j();
+        bool ok = true;
+        int64_t row;
+        if (p.page_table != nullptr) {
+          const int32_t page = p.page_table[(int64_t)c.b * p.max_pages + j / kTileTokens];
+          ok = page >= 0 && page < p.num_pages;
+          if (!ok) atomicOr(p.err, kErrBadPage);
+          row = (int64_t)page * kTileTokens + (j % kTileTokens);
+        } else {
+          row = (int64_t)c.b * p.seq_stride + j;
         }
-        return true;
-      });
+        tile_valid[st] = ok ? 1 : 0;
+        const uint32_t dst = sbase + st * kStageBytes;
+        if (ok) {
+          mbar_arrive_expect_tx(bar(kBarKvFull + st), kStageBytes);
+          for (int i = 0; i < 4; ++i)
+            tma_load_2d(dst + i * kBoxC, &tmap_c, 256 * (int)rank + 64 * i, (int)row, bar(kBarKvFull + st));
+          tma_load_2d(dst + 4 * kBoxC, &tmap_r, 32 * (int)rank, (int)row, bar(kBarKvFull + st));
+        } else {
+          mbar_arrive(bar(kBarKvFull + st));
+        }
+      }
       // copies still in flight (only after an abort) land before the CTA leaves
-      for (uint32_t i = 0; i < kStages && i < g; ++i) {
-        const uint32_t gi = g - 1 - i;
+      for (uint32_t i = 0; i < kStages && i < c.g; ++i) {
+        const uint32_t gi = c.g - 1 - i;
         wait_teardown(bar(kBarKvFull + gi % kStages), (gi / kStages) & 1u, p.wait_limit);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t g = 0, seg = 0;
-      auto issue_qk = [&](uint32_t gt) -> bool {
-        const uint32_t st = gt % kStages;
-        if (!wait_bounded(bar(kBarKvFull + st), (gt / kStages) & 1u, guard)) return false;
-        if (!wait_bounded(bar(kBarSEmpty), (gt & 1u) ^ 1u, guard)) return false;
-        tc_fence_after();
-        const uint32_t a = sbase + st * kStageBytes;
+      TileCursor cq, cv;   // next QK, next PV
+      cq.init(p);
+      cv.init(p);
+      long long idle_since = clock64();
+      while (cv.valid && !*abort_flag) {
+        bool issued = false;
+        // PV first when it is ready: its completion gates the softmax of the next tile
+        if (cv.g < cq.g) {
+          const uint32_t g = cv.g, st = g % kStages, pb = g & 1u;
+          if (mbar_test(bar(kBarPFull + pb), (g >> 1) & 1u) &&
+              (!cv.first() || cv.seg == 0 || mbar_test(bar(kBarOFree), (cv.seg - 1) & 1u))) {
+            tc_fence_after();
+            const uint32_t v = sbase + st * kStageBytes;
 #pragma unroll
-        for (int ks = 0; ks < kKSteps; ++ks) {
-          const uint64_t bd = ks < 16
-              ? smem_desc(a + (ks >> 2) * kBoxC + (ks & 3) * 32, 16, 1024, 2)
-              : smem_desc(a + 4 * kBoxC + (ks - 16) * 32, 16, 512, 4);
-          mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * ks, bd, kIdescQK, ks > 0 ? 1u : 0u);
+            for (int kk = 0; kk < kT / 16; ++kk)
+              mma_ts(tmem + kTmemO, tmem + kTmemP + (kT / 2) * pb + 8 * kk,
+                     smem_desc(v + kk * 2048, kBoxC, 1024, 2), kIdescPV, (!cv.first() || kk > 0) ? 1u : 0u);
+            mma_commit(bar(kBarKvEmpty + st));
+            mma_commit(bar(kBarPvDone));
+            if (cv.last()) mma_commit(bar(kBarOFull));
+            cv.next(p);
+            issued = true;
+          }
         }
-        mma_commit(bar(kBarSFull));
-        return true;
-      };
-      for_each_segment(p, [&](const Segment& s) {
-        if (!wait_bounded(bar(kBarQReady), seg & 1u, guard)) return false;
-        tc_fence_after();
-        if (!issue_qk(g)) return false;
-        for (int k = 0; k < s.ntiles; ++k) {
-          const uint32_t gt = g + k;
-          if (k + 1 < s.ntiles && !issue_qk(gt + 1)) return false;
-          if (!wait_bounded(bar(kBarPFull), gt & 1u, guard)) return false;
-          tc_fence_after();
-          const uint32_t v = sbase + (gt % kStages) * kStageBytes;
+        // QK up to two tiles ahead of PV (S is double-buffered; s_empty guards the reuse)
+        if (!issued && cq.valid && cq.g < cv.g + 3) {
+          const uint32_t g = cq.g, st = g % kStages, sb = g & 1u;
+          if (mbar_test(bar(kBarKvFull + st), (g / kStages) & 1u) &&
+              mbar_test(bar(kBarSEmpty + sb), ((g >> 1) & 1u) ^ 1u) &&
+              (!cq.first() || mbar_test(bar(kBarQReady), cq.seg & 1u))) {
+            tc_fence_after();
+            const uint32_t a = sbase + st * kStageBytes;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tmem + kTmemO, tmem + kTmemP + 8 * kk, smem_desc(v + kk * 2048, kBoxC, 1024, 2),
-                   kIdescPV, (k > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(bar(kBarKvEmpty + gt % kStages));
-          mma_commit(bar(kBarPvDone));
+            for (int ks = 0; ks < kKSteps; ++ks) {
+              const uint64_t bd = ks < 16
+                  ? smem_desc(a + (ks >> 2) * kBoxC + (ks & 3) * 32, 16, 1024, 2)
+                  : smem_desc(a + 4 * kBoxC + (ks - 16) * 32, 16, 512, 4);
+              mma_ts(tmem + kTmemS + kT * sb, tmem + kTmemQ + 8 * ks, bd, kIdescQK, ks > 0 ? 1u : 0u);
+            }
+            mma_commit(bar(kBarSFull + sb));
+            if (cq.last()) mma_commit(bar(kBarQFree));
+            cq.next(p);
+            issued = true;
+          }
         }
-        g += s.ntiles;
-        ++seg;
-        return true;
-      });
+        if (issued) {
+          idle_since = clock64();
+        } else if (clock64() - idle_since > p.wait_limit) {
+          atomicOr(p.err, kErrTimeout);
+          *abort_flag = 1;
+        }
+      }
       mma_commit(bar(kBarFinal));
       wait_teardown(bar(kBarFinal), 0, p.wait_limit);
     }
-  } else {
-    // ------------------------------------------------------------ softmax / epilogue
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ softmax
     const int quarter = warp & 3;                       // TMEM lanes this warp may touch
     const int h = 32 * quarter + lane;                  // head = TMEM lane
     const uint32_t lanes = (uint32_t)(32 * quarter) << 16;
@@ -257,35 +326,166 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     const uint32_t peer_xin = map_to_rank(xin, peer);
     const uint32_t peer_xfull = map_to_rank(bar(kBarXFull), peer);
     const uint32_t peer_xfree = map_to_rank(bar(kBarXFree), peer);
-    const bool head_ok = h < p.n_heads;
-    uint32_t g = 0, seg = 0, nsend = 0, nrecv = 0;
+    const uint32_t rowoff = (uint32_t)h * (kT * 4);
 
-    auto load_s = [&](float (&dst)[kT]) {
+    // own partial S of tile g: out of TMEM, then to the peer's receive buffer g % 2
+    auto fetch_and_send = [&](uint32_t g, float (&dst)[kT]) -> bool {
+      const uint32_t sb = g & 1u;
+      if (!wait_bounded(bar(kBarSFull + sb), (g >> 1) & 1u, guard)) return false;
+      tc_fence_after();
       uint32_t r[32];
-      tmem_ld32_sync(lanes | (tmem + kTmemS), r);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) dst[j] = __uint_as_float(r[j]);
-      tmem_ld32_sync(lanes | (tmem + kTmemS + 32), r);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) dst[32 + j] = __uint_as_float(r[j]);
-    };
-    auto send = [&](const float (&v)[kT]) -> bool {
-      if (!wait_bounded(bar(kBarXFree), (nsend & 1u) ^ 1u, guard, true)) return false;
-      const uint32_t row = peer_xin + (uint32_t)h * (kT * 4);
+      tmem_ld32_sync(lanes | (tmem + kTmemS + kT * sb), r);
+      tc_fence_before();
+      mbar_arrive(bar(kBarSEmpty + sb));
+      if (!wait_bounded(bar(kBarXFree + sb), ((g >> 1) & 1u) ^ 1u, guard, true)) return false;
+      const uint32_t row = peer_xin + sb * kXinBytes + rowoff;
 #pragma unroll
       for (int c = 0; c < kT / 4; ++c)
-        st_cluster_v4(row + (uint32_t)((c ^ (h & 7)) * 16), __float_as_uint(v[4 * c]),
-                      __float_as_uint(v[4 * c + 1]), __float_as_uint(v[4 * c + 2]),
-                      __float_as_uint(v[4 * c + 3]));
-      mbar_arrive_remote(peer_xfull);
-      ++nsend;
+        st_async_v4(row + (uint32_t)((c ^ (h & 7)) * 16), r[4 * c], r[4 * c + 1], r[4 * c + 2],
+                    r[4 * c + 3], peer_xfull + 8u * sb);
+#pragma unroll
+      for (int j = 0; j < kT; ++j) dst[j] = __uint_as_float(r[j]);
       return true;
     };
 
-    for_each_segment(p, [&](const Segment& s) {
-      // the segment's query columns -> TMEM (A operand of Q.K^T)
+    TileCursor c, nx;
+    c.init(p);
+    nx = c;
+    float cur[kT], nxt[kT];
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    if (c.valid) ok = fetch_and_send(0, cur);
+    if (c.valid) nx.next(p);
+    for (; ok && c.valid; c.next(p)) {
+      const uint32_t g = c.g, st = g % kStages, xb = g & 1u;
+      if (!wait_bounded(bar(kBarKvFull + st), (g / kStages) & 1u, guard)) break;
+      const int r = tile_valid[st] ? c.rows() : 0;
+      if (nx.valid) {
+        if (!fetch_and_send(g + 1, nxt)) break;
+      }
+      // the peer's partial scores of tile g: S = own + peer (the same sum on both CTAs)
+      if (!wait_bounded(bar(kBarXFull + xb), (g >> 1) & 1u, guard)) break;
       {
-        const __nv_bfloat16* qrow = p.q_abs + ((int64_t)s.b * p.n_heads + (head_ok ? h : 0)) * kRow;
+        const float4* row = reinterpret_cast<const float4*>(smem + kOffXin + xb * kXinBytes + rowoff);
+#pragma unroll
+        for (int q = 0; q < kT / 4; ++q) {
+          const float4 v = row[q ^ (h & 7)];
+          cur[4 * q] += v.x; cur[4 * q + 1] += v.y; cur[4 * q + 2] += v.z; cur[4 * q + 3] += v.w;
+        }
+      }
+      if (tid == 0) mbar_arrive_expect_tx(bar(kBarXFull + xb), kXinBytes);  // arm the next use
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote_relaxed(peer_xfree + 8u * xb);
+
+      // online softmax in the log2 domain
+      if (c.first()) { m_used = -INFINITY; l = 0.f; }
+      float mt = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kT; ++j) {
+        cur[j] = j < r ? cur[j] * p.scale_log2 : -INFINITY;
+        mt = fmaxf(mt, cur[j]);
+      }
+      float alpha = 1.f;
+      bool need = false;
+      if (m_used == -INFINITY) {
+        m_used = mt;
+      } else if (mt > m_used + kRescaleThreshold) {
+        need = true;
+        alpha = exp2f(m_used - mt);
+        m_used = mt;
+        l *= alpha;
+      }
+      uint32_t pk[16];
+      float sum = 0.f;
+      const bool live = m_used != -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kT; j += 2) {
+        const float p0 = live ? exp2f(cur[j] - m_used) : 0.f;
+        const float p1 = live ? exp2f(cur[j + 1] - m_used) : 0.f;
+        sum += p0 + p1;
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+        pk[j / 2] = *reinterpret_cast<uint32_t*>(&b2);
+      }
+      l += sum;
+      const bool warp_need = __any_sync(0xffffffffu, need);
+
+      // the previous PV is done: O may be rescaled and P[g%2] (last read by PV(g-2)) reused
+      if (!wait_bounded(bar(kBarPvDone), (g & 1u) ^ 1u, guard)) break;
+      tc_fence_after();
+      if (warp_need) {
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t o[32];
+          tmem_ld32_sync(lanes | (tmem + kTmemO + 32 * cc), o);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tmem_st32(lanes | (tmem + kTmemO + 32 * cc), o);
+        }
+      }
+      tmem_st16(lanes | (tmem + kTmemP + (kT / 2) * xb), pk);
+      tmem_wait_st();
+      if (r < kT) {
+        // rows past the sequence end (or of a skipped page) must not reach P.V as NaN/Inf
+        uint8_t* stage = smem + st * kStageBytes;
+        for (int i = tid; i < (kT - r) * 32; i += 128) {
+          const int row = r + (i >> 5), box = (i >> 3) & 3, chunk = i & 7;
+          *reinterpret_cast<uint4*>(stage + box * kBoxC + row * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(kBarPFull + xb));
+      if (c.last()) {
+        ml[(c.seg & 1u) * 128 + h] = make_float2(m_used, l);
+        mbar_arrive(bar(kBarMlFull));
+      }
+#pragma unroll
+      for (int j = 0; j < kT; ++j) cur[j] = nxt[j];
+      if (nx.valid) nx.next(p);
+    }
+  } else {
+    // ------------------------------------------------------------ segment transitions
+    const int quarter = warp & 3;
+    const int h = 32 * quarter + lane;
+    const uint32_t lanes = (uint32_t)(32 * quarter) << 16;
+    const bool head_ok = h < p.n_heads;
+    TileCursor c;
+    c.init(p);
+    int prev_slot = -1;
+    auto epilogue = [&](uint32_t seg, int slot) -> bool {
+      if (!wait_bounded(bar(kBarOFull), seg & 1u, guard)) return false;
+      if (!wait_bounded(bar(kBarMlFull), seg & 1u, guard)) return false;
+      tc_fence_after();
+      const float2 mls = ml[(seg & 1u) * 128 + h];
+      const float inv = mls.y > 0.f ? 1.f / mls.y : 0.f;
+      float* dst = p.part_o + ((int64_t)slot * p.n_heads + (head_ok ? h : 0)) * kDLatent + 256 * rank;
+#pragma unroll 1
+      for (int cc = 0; cc < 8; ++cc) {
+        uint32_t o[32];
+        tmem_ld32_sync(lanes | (tmem + kTmemO + 32 * cc), o);
+        if (head_ok) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(dst + 32 * cc + j) =
+                make_float4(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv,
+                            __uint_as_float(o[j + 2]) * inv, __uint_as_float(o[j + 3]) * inv);
+        }
+      }
+      if (head_ok && rank == 0)
+        p.part_lse[(int64_t)slot * p.n_heads + h] =
+            mls.y > 0.f ? (mls.x + log2f(mls.y)) * 0.69314718055994531f : -INFINITY;
+      tc_fence_before();
+      mbar_arrive(bar(kBarOFree));
+      return true;
+    };
+    bool ok = true;
+    while (ok && c.valid) {
+      const uint32_t seg = c.seg;
+      // this segment's query columns -> TMEM, once the previous segment's last QK is done
+      if (seg > 0 && !wait_bounded(bar(kBarQFree), (seg - 1) & 1u, guard)) break;
+      tc_fence_after();
+      {
+        const __nv_bfloat16* qrow = p.q_abs + ((int64_t)c.b * p.n_heads + (head_ok ? h : 0)) * kRow;
 #pragma unroll 1
         for (int grp = 0; grp < kKSteps / 2; ++grp) {
           uint32_t r[16];
@@ -303,128 +503,13 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
         tc_fence_before();
         mbar_arrive(bar(kBarQReady));
       }
-
-      float m_used = -INFINITY, l = 0.f;
-      float cur[kT], nxt[kT];
-      if (!wait_bounded(bar(kBarSFull), g & 1u, guard)) return false;
-      tc_fence_after();
-      load_s(cur);
-      tc_fence_before();
-      mbar_arrive(bar(kBarSEmpty));
-      if (!send(cur)) return false;
-
-      for (int k = 0; k < s.ntiles; ++k) {
-        const uint32_t gt = g + k, st = gt % kStages;
-        if (!wait_bounded(bar(kBarKvFull + st), (gt / kStages) & 1u, guard)) return false;
-        const int r = tile_valid[st] ? min(kT, s.len - (s.j0 + k * kT)) : 0;
-        const bool more = k + 1 < s.ntiles;
-        if (more) {
-          if (!wait_bounded(bar(kBarSFull), (gt + 1) & 1u, guard)) return false;
-          tc_fence_after();
-          load_s(nxt);
-          tc_fence_before();
-          mbar_arrive(bar(kBarSEmpty));
-        }
-        // the peer's partial scores of this tile: S = own + peer (same sum on both CTAs)
-        if (!wait_bounded(bar(kBarXFull), nrecv & 1u, guard, true)) return false;
-        {
-          const float4* row = reinterpret_cast<const float4*>(smem + kOffXin + h * (kT * 4));
-#pragma unroll
-          for (int c = 0; c < kT / 4; ++c) {
-            const float4 v = row[c ^ (h & 7)];
-            cur[4 * c] += v.x; cur[4 * c + 1] += v.y; cur[4 * c + 2] += v.z; cur[4 * c + 3] += v.w;
-          }
-        }
-        ++nrecv;
-        mbar_arrive_remote(peer_xfree);
-        if (more && !send(nxt)) return false;
-
-        // online softmax in the log2 domain
-        float mt = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < kT; ++j) {
-          cur[j] = j < r ? cur[j] * p.scale_log2 : -INFINITY;
-          mt = fmaxf(mt, cur[j]);
-        }
-        float alpha = 1.f;
-        bool need = false;
-        if (m_used == -INFINITY) {
-          m_used = mt;
-        } else if (mt > m_used + kRescaleThreshold) {
-          need = true;
-          alpha = exp2f(m_used - mt);
-          m_used = mt;
-          l *= alpha;
-        }
-        uint32_t pk[32];
-        float sum = 0.f;
-#pragma unroll
-        for (int j = 0; j < kT; j += 2) {
-          const float p0 = m_used == -INFINITY ? 0.f : exp2f(cur[j] - m_used);
-          const float p1 = m_used == -INFINITY ? 0.f : exp2f(cur[j + 1] - m_used);
-          sum += p0 + p1;
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-          pk[j / 2] = *reinterpret_cast<uint32_t*>(&b2);
-        }
-        l += sum;
-        const bool warp_need = __any_sync(0xffffffffu, need);
-
-        // P may be overwritten and O rescaled once the previous PV has finished
-        if (!wait_bounded(bar(kBarPvDone), (gt & 1u) ^ 1u, guard)) return false;
-        tc_fence_after();
-        if (warp_need) {
-#pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            uint32_t o[32];
-            tmem_ld32_sync(lanes | (tmem + kTmemO + 32 * c), o);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-            tmem_st32(lanes | (tmem + kTmemO + 32 * c), o);
-          }
-        }
-        tmem_st32(lanes | (tmem + kTmemP), pk);
-        tmem_wait_st();
-        if (r < kT) {
-          // rows past the sequence end (or of a skipped page) must not reach P.V as NaN/Inf
-          uint8_t* stage = smem + st * kStageBytes;
-          for (int i = tid; i < (kT - r) * 32; i += 128) {
-            const int row = r + (i >> 5), box = (i >> 3) & 3, chunk = i & 7;
-            *reinterpret_cast<uint4*>(stage + box * kBoxC + row * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
-          }
-          fence_proxy_async_smem();
-        }
-        tc_fence_before();
-        mbar_arrive(bar(kBarPFull));
-#pragma unroll
-        for (int j = 0; j < kT; ++j) cur[j] = nxt[j];
-      }
-
-      // epilogue: O / l and the log-sum-exp of this segment
-      const uint32_t glast = g + s.ntiles - 1;
-      if (!wait_bounded(bar(kBarPvDone), glast & 1u, guard)) return false;
-      tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      float* dst = p.part_o + ((int64_t)s.slot * p.n_heads + (head_ok ? h : 0)) * kDLatent + 256 * rank;
-#pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        uint32_t o[32];
-        tmem_ld32_sync(lanes | (tmem + kTmemO + 32 * c), o);
-        if (head_ok) {
-#pragma unroll
-          for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4*>(dst + 32 * c + j) =
-                make_float4(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv,
-                            __uint_as_float(o[j + 2]) * inv, __uint_as_float(o[j + 3]) * inv);
-        }
-      }
-      if (head_ok && rank == 0)
-        p.part_lse[(int64_t)s.slot * p.n_heads + h] =
-            l > 0.f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
-      tc_fence_before();
-      g += s.ntiles;
-      ++seg;
-      return true;
-    });
+      // the previous segment's output, while this one runs
+      if (seg > 0) ok = epilogue(seg - 1, prev_slot);
+      prev_slot = c.slot;
+      // skip to the next segment
+      while (c.valid && c.seg == seg) c.next(p);
+      if (!c.valid && ok) ok = epilogue(seg, prev_slot);
+    }
   }
 
   // teardown: nobody touches the peer's shared memory after this point

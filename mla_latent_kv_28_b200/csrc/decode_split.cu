@@ -1,9 +1,9 @@
 // Split-KV decode attention over the latent cache on the sm_100a tensor core.
 //
 // Per (sequence, split) segment, for all 128 heads at once (heads are the MMA's M = 128):
-//   S = Q_abs [128 x 576] . [c ; k^R]^T [576 x 32 tokens]     (tcgen05, fp32 in TMEM)
+//   S = Q_abs [128 x 576] . [c ; k^R]^T [576 x 64 tokens]     (tcgen05, fp32 in TMEM)
 //   online softmax over the tokens (exp2, running max with lazy rescale)
-//   O += P [128 x 32] . c [32 x 512]                            (tcgen05, fp32 in TMEM)
+//   O += P [128 x 64] . c [64 x 512]                            (tcgen05, fp32 in TMEM)
 // and the segment's partial O / l and log-sum-exp go to the split slots.
 //
 // Why a 2-CTA cluster: O alone (128 heads x 512 fp32) is the whole 256 KB of one SM's
@@ -16,23 +16,26 @@
 // P, the running max and the normaliser agree without any further exchange. Each cache
 // byte is read from HBM once, by one CTA.
 //
-// Pipeline (32-token tiles, g = tile index within this cluster's work):
-//   TMA ring of 10 stages -> QK(g) into S[g%2] -> softmax threads copy S(g+1) out of TMEM
-//   and send it to the peer while they finish tile g with the peer's S(g) -> P(g) into
-//   P[g%2] -> PV(g). The MMA thread issues whichever of QK / PV is ready, so QK runs two
-//   tiles ahead and the tensor core never waits for the exchange round trip.
+// Pipeline (64-token tiles, g = tile index within this cluster's work):
+//   TMA ring of 4 stages -> QK(g) into S -> softmax threads copy S(g+1) out of TMEM and
+//   send it to the peer while they finish tile g with the peer's S(g) -> P(g) -> PV(g).
+// A single thread can issue a tcgen05.mma only every ~50 cycles, far slower than the
+// tensor core retires small-N MMAs, so QK and PV have issuer warps of their own, and the
+// tile is 64 tokens wide (QK N = 64: 18 MMAs per 64 tokens, PV 4 MMAs of N = 256).
 // Segment boundaries (a unit may hold the tail of one sequence and the head of the next)
 // are handled by a separate warpgroup: it loads the next segment's query columns into
 // TMEM as soon as the last QK of the previous segment is done, and writes the finished
 // segment's O / l while the next segment is already running.
 //
-// Tensor memory (512 columns per CTA): O [0,256) fp32, S [256,320) 2 x 32 fp32,
-// P [320,352) 2 x 16 bf16x2, Q [352,496) bf16x2 (the CTA's 288 query columns, the A
-// operand of Q.K^T). Shared memory: 10 stages x 18 KB of cache tiles (four 32x64 c^KV
-// boxes with 128-byte swizzle + one 32x32 k^R box with 64-byte swizzle), 2 x 16 KB
-// receive buffers for the peer's partial scores, per-segment (max, sum), mbarriers.
-// Warps: 0 TMA producer, 1 MMA issuer (and TMEM owner), 2..5 softmax (one thread per head
-// = TMEM lane), 6..9 segment transitions (query load, epilogue).
+// Tensor memory (512 columns per CTA): O [0,256) fp32, S [256,320) fp32, P [320,352)
+// bf16x2, Q [352,496) bf16x2 (the CTA's 288 query columns, the A operand of Q.K^T).
+// Shared memory: 4 stages x 36 KB of cache tiles (four 64x64 c^KV boxes with 128-byte
+// swizzle + one 64x32 k^R box with 64-byte swizzle), 2 x 32 KB receive buffers for the
+// peer's partial scores, per-segment (max, sum), mbarriers.
+// Warps: 0 TMA producer, 1 QK issuer (and TMEM owner), 2 PV issuer and relay (tells the
+// peer its scores were read, so no softmax warp waits on a cross-SM round trip), 3 idle,
+// 4..7 softmax (one thread per head = TMEM lane), 8..11 segment transitions (query load,
+// epilogue).
 //
 // Every wait is bounded: after about a second it sets the device error word (timeout bit)
 // and the CTA's abort flag, all roles leave their loops, wait for their own copies and
@@ -50,13 +53,13 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kT = 32;                    // tokens per kernel tile (the plan uses 64)
-constexpr int kStages = 10;
+constexpr int kT = 64;                    // tokens per tile (the plan's tile)
+constexpr int kStages = 4;
 constexpr int kKSteps = 18;               // 288 columns / 16
-constexpr uint32_t kBoxC = kT * 128;      // 4 KB: 32 tokens x 64 c^KV columns
-constexpr uint32_t kBoxR = kT * 64;       // 2 KB: 32 tokens x 32 k^R columns
-constexpr uint32_t kStageBytes = 4 * kBoxC + kBoxR;   // 18 KB
-constexpr uint32_t kXinBytes = 128 * kT * 4;          // 16 KB: 128 heads x 32 fp32
+constexpr uint32_t kBoxC = kT * 128;      // 8 KB: 64 tokens x 64 c^KV columns
+constexpr uint32_t kBoxR = kT * 64;       // 4 KB: 64 tokens x 32 k^R columns
+constexpr uint32_t kStageBytes = 4 * kBoxC + kBoxR;   // 36 KB
+constexpr uint32_t kXinBytes = 128 * kT * 4;          // 32 KB: 128 heads x 64 fp32
 constexpr uint32_t kOffXin = kStages * kStageBytes;
 constexpr uint32_t kOffMl = kOffXin + 2 * kXinBytes;  // [2][128] float2 (max, sum)
 constexpr uint32_t kOffBars = kOffMl + 2 * 128 * 8;
@@ -64,9 +67,9 @@ constexpr uint32_t kOffBars = kOffMl + 2 * 128 * 8;
 // barrier indices
 constexpr int kBarKvFull = 0;                    // [kStages] TMA landed
 constexpr int kBarKvEmpty = kStages;             // [kStages] PV of the tile done
-constexpr int kBarSFull = 2 * kStages;           // [2] partial S in TMEM
-constexpr int kBarSEmpty = kBarSFull + 2;        // [2] softmax copied S out
-constexpr int kBarPFull = kBarSFull + 4;         // [2] P in TMEM (O rescaled, V tail zeroed)
+constexpr int kBarSFull = 2 * kStages;           // partial S in TMEM (+1 unused)
+constexpr int kBarSEmpty = kBarSFull + 2;        // softmax copied S out (+1 unused)
+constexpr int kBarPFull = kBarSFull + 4;         // P in TMEM, O rescaled, V tail zeroed (+1 unused)
 constexpr int kBarXFull = kBarSFull + 6;         // [2] the peer's partial scores arrived
 constexpr int kBarXFree = kBarSFull + 8;         // [2] the peer has read what we sent
 constexpr int kBarPvDone = kBarSFull + 10;       // a PV finished
@@ -76,13 +79,20 @@ constexpr int kBarOFull = kBarSFull + 13;        // the last PV of a segment fin
 constexpr int kBarOFree = kBarSFull + 14;        // the epilogue has read O
 constexpr int kBarMlFull = kBarSFull + 15;       // (max, sum) of a finished segment in smem
 constexpr int kBarFinal = kBarSFull + 16;        // all MMAs of this CTA done (teardown)
-constexpr int kNumBars = kBarFinal + 1;
+constexpr int kBarXRead = kBarSFull + 17;        // [2] our softmax warps read the peer's scores
+constexpr int kBarFinal2 = kBarXRead + 2;        // all PV MMAs done (teardown)
+constexpr int kNumBars = kBarFinal2 + 1;
 constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;
 constexpr uint32_t kSmemUsed = kOffMisc + 128;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;     // room to align the base to 1 KB
 
 constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 320, kTmemQ = 352, kTmemCols = 512;
-constexpr int kThreads = 320;
+static_assert(kTmemS + kT <= kTmemP && kTmemP + kT / 2 <= kTmemQ && kTmemQ + 144 <= kTmemCols, "TMEM map");
+constexpr int kThreads = 384;   // 12 warps = 3 warpgroups (roles below)
+// Register split between the warpgroups (setmaxnreg): the softmax warpgroup holds two
+// 64-wide score rows per thread. 128 x (104 + 224 + 80) = 52,224 <= 384 x 168 at launch.
+constexpr int kRegsLaunch = 168, kRegsCtrl = 104, kRegsSoftmax = 224, kRegsTrans = 80;
+static_assert(128 * (kRegsCtrl + kRegsSoftmax + kRegsTrans) <= kThreads * kRegsLaunch, "register split");
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kT, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, false, true);
 constexpr float kRescaleThreshold = 8.f;   // log2 units: rescale O only when the max grows more
@@ -188,12 +198,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       mbar_init(bar(kBarKvEmpty + i), 1);
       tile_valid[i] = 0;
     }
+    mbar_init(bar(kBarSFull), 1);
+    mbar_init(bar(kBarSEmpty), 128);
+    mbar_init(bar(kBarPFull), 128);
+    mbar_init(bar(kBarFinal2), 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(kBarSFull + i), 1);
-      mbar_init(bar(kBarSEmpty + i), 128);
-      mbar_init(bar(kBarPFull + i), 128);
       mbar_init(bar(kBarXFull + i), 1);
-      mbar_init(bar(kBarXFree + i), 4);
+      mbar_init(bar(kBarXFree + i), 1);
+      mbar_init(bar(kBarXRead + i), 4);
     }
     mbar_init(bar(kBarPvDone), 1);
     mbar_init(bar(kBarQReady), 128);
@@ -222,6 +234,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
 
   const WaitGuard guard{abort_flag, p.err, kErrTimeout, p.wait_limit};
 
+  if (warp < 4) regs_dec<kRegsCtrl>();
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -259,112 +272,127 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ QK issuer
+    // S(g) = Q . K(g)^T once the tile landed, the softmax has copied S(g-1) out of TMEM
+    // and (first tile of a segment) the segment's query columns are in TMEM.
     if (lane == 0) {
-      TileCursor cq, cv;   // next QK, next PV
-      cq.init(p);
-      cv.init(p);
-      long long idle_since = clock64();
-      while (cv.valid && !*abort_flag) {
-        bool issued = false;
-        // PV first when it is ready: its completion gates the softmax of the next tile
-        if (cv.g < cq.g) {
-          const uint32_t g = cv.g, st = g % kStages, pb = g & 1u;
-          if (mbar_test(bar(kBarPFull + pb), (g >> 1) & 1u) &&
-              (!cv.first() || cv.seg == 0 || mbar_test(bar(kBarOFree), (cv.seg - 1) & 1u))) {
-            tc_fence_after();
-            const uint32_t v = sbase + st * kStageBytes;
+      TileCursor c;
+      c.init(p);
+      for (; c.valid; c.next(p)) {
+        const uint32_t g = c.g, st = g % kStages;
+        if (!wait_bounded(bar(kBarKvFull + st), (g / kStages) & 1u, guard)) break;
+        if (!wait_bounded(bar(kBarSEmpty), (g & 1u) ^ 1u, guard)) break;
+        if (c.first() && !wait_bounded(bar(kBarQReady), c.seg & 1u, guard)) break;
+        tc_fence_after();
+        const uint32_t a = sbase + st * kStageBytes;
 #pragma unroll
-            for (int kk = 0; kk < kT / 16; ++kk)
-              mma_ts(tmem + kTmemO, tmem + kTmemP + (kT / 2) * pb + 8 * kk,
-                     smem_desc(v + kk * 2048, kBoxC, 1024, 2), kIdescPV, (!cv.first() || kk > 0) ? 1u : 0u);
-            mma_commit(bar(kBarKvEmpty + st));
-            mma_commit(bar(kBarPvDone));
-            if (cv.last()) mma_commit(bar(kBarOFull));
-            cv.next(p);
-            issued = true;
-          }
+        for (int ks = 0; ks < kKSteps; ++ks) {
+          const uint64_t bd = ks < 16
+              ? smem_desc(a + (ks >> 2) * kBoxC + (ks & 3) * 32, 16, 1024, 2)
+              : smem_desc(a + 4 * kBoxC + (ks - 16) * 32, 16, 512, 4);
+          mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * ks, bd, kIdescQK, ks > 0 ? 1u : 0u);
         }
-        // QK up to two tiles ahead of PV (S is double-buffered; s_empty guards the reuse)
-        if (!issued && cq.valid && cq.g < cv.g + 3) {
-          const uint32_t g = cq.g, st = g % kStages, sb = g & 1u;
-          if (mbar_test(bar(kBarKvFull + st), (g / kStages) & 1u) &&
-              mbar_test(bar(kBarSEmpty + sb), ((g >> 1) & 1u) ^ 1u) &&
-              (!cq.first() || mbar_test(bar(kBarQReady), cq.seg & 1u))) {
-            tc_fence_after();
-            const uint32_t a = sbase + st * kStageBytes;
-#pragma unroll
-            for (int ks = 0; ks < kKSteps; ++ks) {
-              const uint64_t bd = ks < 16
-                  ? smem_desc(a + (ks >> 2) * kBoxC + (ks & 3) * 32, 16, 1024, 2)
-                  : smem_desc(a + 4 * kBoxC + (ks - 16) * 32, 16, 512, 4);
-              mma_ts(tmem + kTmemS + kT * sb, tmem + kTmemQ + 8 * ks, bd, kIdescQK, ks > 0 ? 1u : 0u);
-            }
-            mma_commit(bar(kBarSFull + sb));
-            if (cq.last()) mma_commit(bar(kBarQFree));
-            cq.next(p);
-            issued = true;
-          }
-        }
-        if (issued) {
-          idle_since = clock64();
-        } else if (clock64() - idle_since > p.wait_limit) {
-          atomicOr(p.err, kErrTimeout);
-          *abort_flag = 1;
-        }
+        mma_commit(bar(kBarSFull));
+        if (c.last()) mma_commit(bar(kBarQFree));
       }
       mma_commit(bar(kBarFinal));
       wait_teardown(bar(kBarFinal), 0, p.wait_limit);
     }
-  } else if (warp < 6) {
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ PV issuer and relay
+    // Relay: when our softmax warps have read the peer's scores of tile g, re-arm the receive
+    // barrier for tile g + 2 and tell the peer that buffer g % 2 is free again (so no
+    // softmax warp waits on a cross-SM round trip). That always happens before P(g) is ready.
+    // PV: O += P(g) . V(g) once P(g) is in TMEM and (first tile of a segment) the previous
+    // segment's O has been read out. Its completion frees the stage, P, and O.
+    if (lane == 0) {
+      const uint32_t peer_xfree = map_to_rank(bar(kBarXFree), peer);
+      TileCursor c;
+      c.init(p);
+      for (; c.valid; c.next(p)) {
+        const uint32_t g = c.g, st = g % kStages, xb = g & 1u;
+        if (!wait_bounded(bar(kBarXRead + xb), (g >> 1) & 1u, guard)) break;
+        mbar_arrive_expect_tx(bar(kBarXFull + xb), kXinBytes);
+        mbar_arrive_remote_relaxed(peer_xfree + 8u * xb);
+        if (!wait_bounded(bar(kBarPFull), g & 1u, guard)) break;
+        if (c.first() && c.seg > 0 && !wait_bounded(bar(kBarOFree), (c.seg - 1) & 1u, guard)) break;
+        tc_fence_after();
+        const uint32_t v = sbase + st * kStageBytes;
+#pragma unroll
+        for (int kk = 0; kk < kT / 16; ++kk)
+          mma_ts(tmem + kTmemO, tmem + kTmemP + 8 * kk, smem_desc(v + kk * 2048, kBoxC, 1024, 2),
+                 kIdescPV, (!c.first() || kk > 0) ? 1u : 0u);
+        mma_commit(bar(kBarKvEmpty + st));
+        mma_commit(bar(kBarPvDone));
+        if (c.last()) mma_commit(bar(kBarOFull));
+      }
+      mma_commit(bar(kBarFinal2));
+      wait_teardown(bar(kBarFinal2), 0, p.wait_limit);
+    }
+  } else if (warp == 3) {
+    // idle
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax
+    regs_inc<kRegsSoftmax>();
     const int quarter = warp & 3;                       // TMEM lanes this warp may touch
     const int h = 32 * quarter + lane;                  // head = TMEM lane
     const uint32_t lanes = (uint32_t)(32 * quarter) << 16;
-    const int tid = threadIdx.x - 64;                   // 0..127 among the softmax threads
+    const int tid = threadIdx.x - 128;                  // 0..127 among the softmax threads
     const uint32_t xin = sbase + kOffXin;
     const uint32_t peer_xin = map_to_rank(xin, peer);
     const uint32_t peer_xfull = map_to_rank(bar(kBarXFull), peer);
-    const uint32_t peer_xfree = map_to_rank(bar(kBarXFree), peer);
     const uint32_t rowoff = (uint32_t)h * (kT * 4);
 
-    // own partial S of tile g: out of TMEM, then to the peer's receive buffer g % 2
-    auto fetch_and_send = [&](uint32_t g, float (&dst)[kT]) -> bool {
-      const uint32_t sb = g & 1u;
-      if (!wait_bounded(bar(kBarSFull + sb), (g >> 1) & 1u, guard)) return false;
+    // own partial S of tile g: out of TMEM (freeing S for the next QK), then to the peer's
+    // receive buffer g % 2 (16-byte chunks, XOR-swizzled by head to spread the banks)
+    auto fetch_and_send = [&](uint32_t g, uint32_t (&dst)[kT]) -> bool {
+      const uint32_t xb = g & 1u;
+      if (!wait_spin(bar(kBarSFull), g & 1u, guard)) return false;
       tc_fence_after();
-      uint32_t r[32];
-      tmem_ld32_sync(lanes | (tmem + kTmemS + kT * sb), r);
+      uint32_t (&r0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dst[0]);
+      uint32_t (&r1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dst[32]);
+      tmem_ld32_sync(lanes | (tmem + kTmemS), r0);
+      tmem_ld32_sync(lanes | (tmem + kTmemS + 32), r1);
       tc_fence_before();
-      mbar_arrive(bar(kBarSEmpty + sb));
-      if (!wait_bounded(bar(kBarXFree + sb), ((g >> 1) & 1u) ^ 1u, guard, true)) return false;
-      const uint32_t row = peer_xin + sb * kXinBytes + rowoff;
+      mbar_arrive(bar(kBarSEmpty));
+      if (!wait_spin(bar(kBarXFree + xb), ((g >> 1) & 1u) ^ 1u, guard)) return false;
+      const uint32_t row = peer_xin + xb * kXinBytes + rowoff;
 #pragma unroll
-      for (int c = 0; c < kT / 4; ++c)
-        st_async_v4(row + (uint32_t)((c ^ (h & 7)) * 16), r[4 * c], r[4 * c + 1], r[4 * c + 2],
-                    r[4 * c + 3], peer_xfull + 8u * sb);
+      for (int c = 0; c < 8; ++c)
+        st_async_v4(row + (uint32_t)((c ^ (h & 7)) * 16), r0[4 * c], r0[4 * c + 1], r0[4 * c + 2],
+                    r0[4 * c + 3], peer_xfull + 8u * xb);
 #pragma unroll
-      for (int j = 0; j < kT; ++j) dst[j] = __uint_as_float(r[j]);
+      for (int c = 0; c < 8; ++c)
+        st_async_v4(row + (uint32_t)(((c + 8) ^ (h & 7)) * 16), r1[4 * c], r1[4 * c + 1], r1[4 * c + 2],
+                    r1[4 * c + 3], peer_xfull + 8u * xb);
       return true;
     };
 
-    TileCursor c, nx;
+    uint32_t total = 0;   // tiles of this cluster's work
+    {
+      TileCursor t;
+      for (t.init(p); t.valid; t.next(p)) ++total;
+    }
+    TileCursor c;
     c.init(p);
-    nx = c;
-    float cur[kT], nxt[kT];
+    float cur[kT];
+    uint32_t nxt[kT];
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    if (c.valid) ok = fetch_and_send(0, cur);
-    if (c.valid) nx.next(p);
+    if (c.valid) {
+      ok = fetch_and_send(0, nxt);
+#pragma unroll
+      for (int j = 0; j < kT; ++j) cur[j] = __uint_as_float(nxt[j]);
+    }
     for (; ok && c.valid; c.next(p)) {
       const uint32_t g = c.g, st = g % kStages, xb = g & 1u;
-      if (!wait_bounded(bar(kBarKvFull + st), (g / kStages) & 1u, guard)) break;
+      if (!wait_spin(bar(kBarKvFull + st), (g / kStages) & 1u, guard)) break;
       const int r = tile_valid[st] ? c.rows() : 0;
-      if (nx.valid) {
+      if (g + 1 < total) {
         if (!fetch_and_send(g + 1, nxt)) break;
       }
       // the peer's partial scores of tile g: S = own + peer (the same sum on both CTAs)
-      if (!wait_bounded(bar(kBarXFull + xb), (g >> 1) & 1u, guard)) break;
+      if (!wait_spin(bar(kBarXFull + xb), (g >> 1) & 1u, guard)) break;
       {
         const float4* row = reinterpret_cast<const float4*>(smem + kOffXin + xb * kXinBytes + rowoff);
 #pragma unroll
@@ -373,44 +401,47 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
           cur[4 * q] += v.x; cur[4 * q + 1] += v.y; cur[4 * q + 2] += v.z; cur[4 * q + 3] += v.w;
         }
       }
-      if (tid == 0) mbar_arrive_expect_tx(bar(kBarXFull + xb), kXinBytes);  // arm the next use
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote_relaxed(peer_xfree + 8u * xb);
+      if (lane == 0) mbar_arrive(bar(kBarXRead + xb));   // the relay frees the buffer
 
-      // online softmax in the log2 domain
+      // online softmax in the log2 domain: p = 2^(s * scale * log2(e) - m)
       if (c.first()) { m_used = -INFINITY; l = 0.f; }
-      float mt = -INFINITY;
+      if (r < kT) {  // the last tile of a sequence (or a skipped page): mask what is not there
 #pragma unroll
-      for (int j = 0; j < kT; ++j) {
-        cur[j] = j < r ? cur[j] * p.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, cur[j]);
+        for (int j = 0; j < kT; ++j) cur[j] = j < r ? cur[j] : -INFINITY;
       }
+      float mx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = cur[i];
+#pragma unroll
+      for (int j = 8; j < kT; ++j) mx[j & 7] = fmaxf(mx[j & 7], cur[j]);
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * p.scale_log2;
       float alpha = 1.f;
       bool need = false;
       if (m_used == -INFINITY) {
         m_used = mt;
       } else if (mt > m_used + kRescaleThreshold) {
         need = true;
-        alpha = exp2f(m_used - mt);
+        alpha = ex2_approx(m_used - mt);
         m_used = mt;
         l *= alpha;
       }
-      uint32_t pk[16];
-      float sum = 0.f;
       const bool live = m_used != -INFINITY;
+      const float neg_m = live ? -m_used : 0.f;
+      float sm[8];
 #pragma unroll
-      for (int j = 0; j < kT; j += 2) {
-        const float p0 = live ? exp2f(cur[j] - m_used) : 0.f;
-        const float p1 = live ? exp2f(cur[j + 1] - m_used) : 0.f;
-        sum += p0 + p1;
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-        pk[j / 2] = *reinterpret_cast<uint32_t*>(&b2);
+      for (int i = 0; i < 8; ++i) sm[i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < kT; ++j) {   // P in place
+        cur[j] = live ? ex2_approx(fmaf(cur[j], p.scale_log2, neg_m)) : 0.f;
+        sm[j & 7] += cur[j];
       }
-      l += sum;
+      l += ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
       const bool warp_need = __any_sync(0xffffffffu, need);
 
-      // the previous PV is done: O may be rescaled and P[g%2] (last read by PV(g-2)) reused
-      if (!wait_bounded(bar(kBarPvDone), (g & 1u) ^ 1u, guard)) break;
+      // the previous PV is done: O may be rescaled and P (read by PV(g-1)) overwritten
+      if (!wait_spin(bar(kBarPvDone), (g & 1u) ^ 1u, guard)) break;
       tc_fence_after();
       if (warp_need) {
 #pragma unroll 1
@@ -422,7 +453,16 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
           tmem_st32(lanes | (tmem + kTmemO + 32 * cc), o);
         }
       }
-      tmem_st16(lanes | (tmem + kTmemP + (kT / 2) * xb), pk);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {   // P as bf16 pairs, 16 columns at a time
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(cur[32 * half + 2 * j], cur[32 * half + 2 * j + 1]);
+          pk[j] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        tmem_st16(lanes | (tmem + kTmemP + 16 * half), pk);
+      }
       tmem_wait_st();
       if (r < kT) {
         // rows past the sequence end (or of a skipped page) must not reach P.V as NaN/Inf
@@ -434,17 +474,17 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
         fence_proxy_async_smem();
       }
       tc_fence_before();
-      mbar_arrive(bar(kBarPFull + xb));
+      mbar_arrive(bar(kBarPFull));
       if (c.last()) {
         ml[(c.seg & 1u) * 128 + h] = make_float2(m_used, l);
         mbar_arrive(bar(kBarMlFull));
       }
 #pragma unroll
-      for (int j = 0; j < kT; ++j) cur[j] = nxt[j];
-      if (nx.valid) nx.next(p);
+      for (int j = 0; j < kT; ++j) cur[j] = __uint_as_float(nxt[j]);
     }
   } else {
     // ------------------------------------------------------------ segment transitions
+    regs_dec<kRegsTrans>();
     const int quarter = warp & 3;
     const int h = 32 * quarter + lane;
     const uint32_t lanes = (uint32_t)(32 * quarter) << 16;

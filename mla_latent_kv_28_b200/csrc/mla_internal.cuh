@@ -5,7 +5,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-#include "../../include/mla_decode.h"
+#include "mla_decode.h"
 
 namespace mla {
 

@@ -132,17 +132,42 @@ struct WaitGuard {
 
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const WaitGuard& g,
                                              bool cluster_scope = false) {
-  if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+  // Threads whose waits gate nothing urgent suspend in try_wait (freeing issue slots for the
+  // warps that do the arithmetic); a phase that is already complete costs one probe.
+  if (!cluster_scope && mbar_test(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (*g.abort) return false;
     if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    if (*g.abort) return false;
     if (clock64() - t0 > g.limit) {
       atomicOr(g.err, g.flag);
       *g.abort = 1;
       return false;
     }
   }
+}
+
+// The same bound, spinning on the non-blocking probe: for the latency-critical softmax
+// warps, which resume the moment the phase completes.
+__device__ __forceinline__ bool wait_spin(uint32_t bar, uint32_t parity, const WaitGuard& g) {
+  if (mbar_test(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_test(bar, parity)) return true;
+    if (*g.abort) return false;
+    if (clock64() - t0 > g.limit) {
+      atomicOr(g.err, g.flag);
+      *g.abort = 1;
+      return false;
+    }
+  }
+}
+
+// 2^x on the MUFU unit (ex2.approx.ftz: about 2 ulp, flushes denormal results to zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // ------------------------------------------------------------------ proxies and TMA
@@ -161,6 +186,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, 
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];"
       :: "r"(dst), "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+
+// ------------------------------------------------------------------ register budget
+// Move registers between warpgroups. The increase waits until the decreases of the other
+// warpgroups have returned enough registers to the block's pool, so the shares must add up
+// to no more than the block was launched with (threads x registers per thread).
+template <int N> __device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(N));
+}
+template <int N> __device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(N));
 }
 
 // ------------------------------------------------------------------ tcgen05

@@ -33,9 +33,11 @@
 // swizzle + one 64x32 k^R box with 64-byte swizzle), 2 x 32 KB receive buffers for the
 // peer's partial scores, per-segment (max, sum), mbarriers.
 // Warps: 0 TMA producer, 1 QK issuer (and TMEM owner), 2 PV issuer and relay (tells the
-// peer its scores were read, so no softmax warp waits on a cross-SM round trip), 3 idle,
-// 4..7 softmax (one thread per head = TMEM lane), 8..11 segment transitions (query load,
-// epilogue).
+// peer its scores were read, so no softmax warp waits on a cross-SM round trip), 3 idle;
+// 4..7 and 8..11 softmax, one thread per (head = TMEM lane, half of the tile's 64 tokens):
+// two warps per SM sub-partition hide each other's latencies, and the pair of threads of
+// a head agree on the tile maximum through shared memory; 12..15 segment transitions
+// (query load, epilogue).
 //
 // Every wait is bounded: after about a second it sets the device error word (timeout bit)
 // and the CTA's abort flag, all roles leave their loops, wait for their own copies and
@@ -61,8 +63,9 @@ constexpr uint32_t kBoxR = kT * 64;       // 4 KB: 64 tokens x 32 k^R columns
 constexpr uint32_t kStageBytes = 4 * kBoxC + kBoxR;   // 36 KB
 constexpr uint32_t kXinBytes = 128 * kT * 4;          // 32 KB: 128 heads x 64 fp32
 constexpr uint32_t kOffXin = kStages * kStageBytes;
-constexpr uint32_t kOffMl = kOffXin + 2 * kXinBytes;  // [2][128] float2 (max, sum)
-constexpr uint32_t kOffBars = kOffMl + 2 * 128 * 8;
+constexpr uint32_t kOffMl = kOffXin + 2 * kXinBytes;  // [2 segs][2 halves][128] float2 (max, sum)
+constexpr uint32_t kOffHmax = kOffMl + 2 * 2 * 128 * 8;  // [2 tiles][2 halves][128] float
+constexpr uint32_t kOffBars = kOffHmax + 2 * 2 * 128 * 4;
 
 // barrier indices
 constexpr int kBarKvFull = 0;                    // [kStages] TMA landed
@@ -88,11 +91,12 @@ constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;     // room to align the base 
 
 constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 320, kTmemQ = 352, kTmemCols = 512;
 static_assert(kTmemS + kT <= kTmemP && kTmemP + kT / 2 <= kTmemQ && kTmemQ + 144 <= kTmemCols, "TMEM map");
-constexpr int kThreads = 384;   // 12 warps = 3 warpgroups (roles below)
-// Register split between the warpgroups (setmaxnreg): the softmax warpgroup holds two
-// 64-wide score rows per thread. 128 x (104 + 224 + 80) = 52,224 <= 384 x 168 at launch.
-constexpr int kRegsLaunch = 168, kRegsCtrl = 104, kRegsSoftmax = 224, kRegsTrans = 80;
-static_assert(128 * (kRegsCtrl + kRegsSoftmax + kRegsTrans) <= kThreads * kRegsLaunch, "register split");
+constexpr int kThreads = 512;   // 16 warps = 4 warpgroups (roles below)
+// Register split between the warpgroups (setmaxnreg), against 512 x 128 at launch:
+// 128 x (64 + 160 + 160 + 96) = 61,440 <= 65,536.
+constexpr int kRegsLaunch = 128, kRegsCtrl = 64, kRegsSoftmax = 160, kRegsTrans = 96;
+static_assert(128 * (kRegsCtrl + 2 * kRegsSoftmax + kRegsTrans) <= kThreads * kRegsLaunch, "register split");
+constexpr int kHalf = kT / 2;   // tokens per softmax thread
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kT, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, false, true);
 constexpr float kRescaleThreshold = 8.f;   // log2 units: rescale O only when the max grows more
@@ -186,7 +190,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   volatile int* tile_valid = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);  // [kStages]
-  float2* ml = reinterpret_cast<float2*>(smem + kOffMl);                             // [2][128]
+  float2* ml = reinterpret_cast<float2*>(smem + kOffMl);                             // [2][2][128]
+  float* hmax = reinterpret_cast<float*>(smem + kOffHmax);                           // [2][2][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -199,20 +204,20 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       tile_valid[i] = 0;
     }
     mbar_init(bar(kBarSFull), 1);
-    mbar_init(bar(kBarSEmpty), 128);
-    mbar_init(bar(kBarPFull), 128);
+    mbar_init(bar(kBarSEmpty), 256);
+    mbar_init(bar(kBarPFull), 256);
     mbar_init(bar(kBarFinal2), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarXFull + i), 1);
       mbar_init(bar(kBarXFree + i), 1);
-      mbar_init(bar(kBarXRead + i), 4);
+      mbar_init(bar(kBarXRead + i), 8);
     }
     mbar_init(bar(kBarPvDone), 1);
     mbar_init(bar(kBarQReady), 128);
     mbar_init(bar(kBarQFree), 1);
     mbar_init(bar(kBarOFull), 1);
     mbar_init(bar(kBarOFree), 128);
-    mbar_init(bar(kBarMlFull), 128);
+    mbar_init(bar(kBarMlFull), 256);
     mbar_init(bar(kBarFinal), 1);
     *abort_flag = 0;
     // the receive buffers expect their first tile of partial scores
@@ -238,28 +243,30 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      // first row of a tile in the cache, or -1 for a page-table entry out of range
+      auto tile_row = [&](const TileCursor& t) -> int64_t {
+        const int j = t.j();
+        if (p.page_table == nullptr) return (int64_t)t.b * p.seq_stride + j;
+        const int32_t page = p.page_table[(int64_t)t.b * p.max_pages + j / kTileTokens];
+        if (page < 0 || page >= p.num_pages) return -1;
+        return (int64_t)page * kTileTokens + (j % kTileTokens);
+      };
       TileCursor c;
       c.init(p);
       for (; c.valid; c.next(p)) {
         const uint32_t g = c.g, st = g % kStages;
         if (!wait_bounded(bar(kBarKvEmpty + st), ((g / kStages) & 1u) ^ 1u, guard)) break;
-        const int j = c.j();
-        bool ok = true;
-        int64_t row;
-        if (p.page_table != nullptr) {
-          const int32_t page = p.page_table[(int64_t)c.b * p.max_pages + j / kTileTokens];
-          ok = page >= 0 && page < p.num_pages;
-          if (!ok) atomicOr(p.err, kErrBadPage);
-          row = (int64_t)page * kTileTokens + (j % kTileTokens);
-        } else {
-          row = (int64_t)c.b * p.seq_stride + j;
-        }
+        const int64_t row = tile_row(c);
+        const bool ok = row >= 0;
+        if (!ok) atomicOr(p.err, kErrBadPage);
         tile_valid[st] = ok ? 1 : 0;
         const uint32_t dst = sbase + st * kStageBytes;
         if (ok) {
           mbar_arrive_expect_tx(bar(kBarKvFull + st), kStageBytes);
-          for (int i = 0; i < 4; ++i)
-            tma_load_2d(dst + i * kBoxC, &tmap_c, 256 * (int)rank + 64 * i, (int)row, bar(kBarKvFull + st));
+          // the CTA's four 64-column c^KV boxes in one copy (3-D map: column, row, column group),
+          // then its 32 k^R columns: two TMA instructions per tile keep the producer's warp
+          // from crowding the softmax warps that share its SM sub-partition
+          tma_load_3d(dst, &tmap_c, 0, (int)row, 4 * (int)rank, bar(kBarKvFull + st));
           tma_load_2d(dst + 4 * kBoxC, &tmap_r, 32 * (int)rank, (int)row, bar(kBarKvFull + st));
         } else {
           mbar_arrive(bar(kBarKvFull + st));
@@ -331,40 +338,37 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     }
   } else if (warp == 3) {
     // idle
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ------------------------------------------------------------ softmax
     regs_inc<kRegsSoftmax>();
     const int quarter = warp & 3;                       // TMEM lanes this warp may touch
+    const int half = (warp >> 2) - 1;                   // which 32 of the tile's 64 tokens
     const int h = 32 * quarter + lane;                  // head = TMEM lane
     const uint32_t lanes = (uint32_t)(32 * quarter) << 16;
-    const int tid = threadIdx.x - 128;                  // 0..127 among the softmax threads
+    const int tid = threadIdx.x - 128;                  // 0..255 among the softmax threads
+    const uint32_t pair_bar = 1u + (uint32_t)quarter;   // named barrier of the two warps of a head
     const uint32_t xin = sbase + kOffXin;
     const uint32_t peer_xin = map_to_rank(xin, peer);
     const uint32_t peer_xfull = map_to_rank(bar(kBarXFull), peer);
     const uint32_t rowoff = (uint32_t)h * (kT * 4);
+    const uint32_t col0 = (uint32_t)(kHalf * half);
 
-    // own partial S of tile g: out of TMEM (freeing S for the next QK), then to the peer's
-    // receive buffer g % 2 (16-byte chunks, XOR-swizzled by head to spread the banks)
-    auto fetch_and_send = [&](uint32_t g, uint32_t (&dst)[kT]) -> bool {
+    // own partial S of this half of tile g: out of TMEM (freeing S for the next QK once both
+    // halves are out), then to the peer's receive buffer g % 2 (16-byte chunks,
+    // XOR-swizzled by head to spread the banks)
+    auto fetch_and_send = [&](uint32_t g, uint32_t (&dst)[kHalf]) -> bool {
       const uint32_t xb = g & 1u;
       if (!wait_spin(bar(kBarSFull), g & 1u, guard)) return false;
       tc_fence_after();
-      uint32_t (&r0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dst[0]);
-      uint32_t (&r1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dst[32]);
-      tmem_ld32_sync(lanes | (tmem + kTmemS), r0);
-      tmem_ld32_sync(lanes | (tmem + kTmemS + 32), r1);
+      tmem_ld32_sync(lanes | (tmem + kTmemS + col0), dst);
       tc_fence_before();
       mbar_arrive(bar(kBarSEmpty));
       if (!wait_spin(bar(kBarXFree + xb), ((g >> 1) & 1u) ^ 1u, guard)) return false;
       const uint32_t row = peer_xin + xb * kXinBytes + rowoff;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
-        st_async_v4(row + (uint32_t)((c ^ (h & 7)) * 16), r0[4 * c], r0[4 * c + 1], r0[4 * c + 2],
-                    r0[4 * c + 3], peer_xfull + 8u * xb);
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        st_async_v4(row + (uint32_t)(((c + 8) ^ (h & 7)) * 16), r1[4 * c], r1[4 * c + 1], r1[4 * c + 2],
-                    r1[4 * c + 3], peer_xfull + 8u * xb);
+        st_async_v4(row + (uint32_t)(((c + 8 * half) ^ (h & 7)) * 16), dst[4 * c], dst[4 * c + 1],
+                    dst[4 * c + 2], dst[4 * c + 3], peer_xfull + 8u * xb);
       return true;
     };
 
@@ -375,14 +379,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     }
     TileCursor c;
     c.init(p);
-    float cur[kT];
-    uint32_t nxt[kT];
-    float m_used = -INFINITY, l = 0.f;
+    float cur[kHalf];
+    uint32_t nxt[kHalf];
+    float m_used = -INFINITY, l = 0.f;   // l: this half's share of the normaliser
     bool ok = true;
     if (c.valid) {
       ok = fetch_and_send(0, nxt);
 #pragma unroll
-      for (int j = 0; j < kT; ++j) cur[j] = __uint_as_float(nxt[j]);
+      for (int j = 0; j < kHalf; ++j) cur[j] = __uint_as_float(nxt[j]);
     }
     for (; ok && c.valid; c.next(p)) {
       const uint32_t g = c.g, st = g % kStages, xb = g & 1u;
@@ -396,8 +400,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       {
         const float4* row = reinterpret_cast<const float4*>(smem + kOffXin + xb * kXinBytes + rowoff);
 #pragma unroll
-        for (int q = 0; q < kT / 4; ++q) {
-          const float4 v = row[q ^ (h & 7)];
+        for (int q = 0; q < kHalf / 4; ++q) {
+          const float4 v = row[(q + 8 * half) ^ (h & 7)];
           cur[4 * q] += v.x; cur[4 * q + 1] += v.y; cur[4 * q + 2] += v.z; cur[4 * q + 3] += v.w;
         }
       }
@@ -406,17 +410,22 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
 
       // online softmax in the log2 domain: p = 2^(s * scale * log2(e) - m)
       if (c.first()) { m_used = -INFINITY; l = 0.f; }
-      if (r < kT) {  // the last tile of a sequence (or a skipped page): mask what is not there
+      const int rh = min(max(r - kHalf * half, 0), kHalf);   // valid tokens in this half
+      if (rh < kHalf) {  // the last tile of a sequence (or a skipped page): mask what is not there
 #pragma unroll
-        for (int j = 0; j < kT; ++j) cur[j] = j < r ? cur[j] : -INFINITY;
+        for (int j = 0; j < kHalf; ++j) cur[j] = j < rh ? cur[j] : -INFINITY;
       }
       float mx[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx[i] = cur[i];
 #pragma unroll
-      for (int j = 8; j < kT; ++j) mx[j & 7] = fmaxf(mx[j & 7], cur[j]);
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * p.scale_log2;
+      for (int j = 8; j < kHalf; ++j) mx[j & 7] = fmaxf(mx[j & 7], cur[j]);
+      float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      // the maximum over the whole tile: swap the half maxima with the partner warp
+      hmax[((g & 1u) * 2 + half) * 128 + h] = mt;
+      asm volatile("bar.sync %0, 64;" :: "r"(pair_bar) : "memory");
+      mt = fmaxf(mt, hmax[((g & 1u) * 2 + (half ^ 1)) * 128 + h]) * p.scale_log2;
       float alpha = 1.f;
       bool need = false;
       if (m_used == -INFINITY) {
@@ -433,7 +442,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
 #pragma unroll
       for (int i = 0; i < 8; ++i) sm[i] = 0.f;
 #pragma unroll
-      for (int j = 0; j < kT; ++j) {   // P in place
+      for (int j = 0; j < kHalf; ++j) {   // P in place
         cur[j] = live ? ex2_approx(fmaf(cur[j], p.scale_log2, neg_m)) : 0.f;
         sm[j & 7] += cur[j];
       }
@@ -443,22 +452,22 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       // the previous PV is done: O may be rescaled and P (read by PV(g-1)) overwritten
       if (!wait_spin(bar(kBarPvDone), (g & 1u) ^ 1u, guard)) break;
       tc_fence_after();
-      if (warp_need) {
+      if (warp_need) {   // this half rescales O columns [128 half, 128 half + 128)
 #pragma unroll 1
-        for (int cc = 0; cc < 8; ++cc) {
+        for (int cc = 0; cc < 4; ++cc) {
           uint32_t o[32];
-          tmem_ld32_sync(lanes | (tmem + kTmemO + 32 * cc), o);
+          const uint32_t col = kTmemO + 128 * half + 32 * cc;
+          tmem_ld32_sync(lanes | (tmem + col), o);
 #pragma unroll
           for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          tmem_st32(lanes | (tmem + kTmemO + 32 * cc), o);
+          tmem_st32(lanes | (tmem + col), o);
         }
       }
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {   // P as bf16 pairs, 16 columns at a time
+      {   // P as bf16 pairs: this half's 16 columns
         uint32_t pk[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(cur[32 * half + 2 * j], cur[32 * half + 2 * j + 1]);
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(cur[2 * j], cur[2 * j + 1]);
           pk[j] = *reinterpret_cast<uint32_t*>(&b2);
         }
         tmem_st16(lanes | (tmem + kTmemP + 16 * half), pk);
@@ -467,7 +476,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       if (r < kT) {
         // rows past the sequence end (or of a skipped page) must not reach P.V as NaN/Inf
         uint8_t* stage = smem + st * kStageBytes;
-        for (int i = tid; i < (kT - r) * 32; i += 128) {
+        for (int i = tid; i < (kT - r) * 32; i += 256) {
           const int row = r + (i >> 5), box = (i >> 3) & 3, chunk = i & 7;
           *reinterpret_cast<uint4*>(stage + box * kBoxC + row * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
         }
@@ -476,11 +485,11 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       tc_fence_before();
       mbar_arrive(bar(kBarPFull));
       if (c.last()) {
-        ml[(c.seg & 1u) * 128 + h] = make_float2(m_used, l);
+        ml[((c.seg & 1u) * 2 + half) * 128 + h] = make_float2(m_used, l);
         mbar_arrive(bar(kBarMlFull));
       }
 #pragma unroll
-      for (int j = 0; j < kT; ++j) cur[j] = __uint_as_float(nxt[j]);
+      for (int j = 0; j < kHalf; ++j) cur[j] = __uint_as_float(nxt[j]);
     }
   } else {
     // ------------------------------------------------------------ segment transitions
@@ -496,7 +505,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       if (!wait_bounded(bar(kBarOFull), seg & 1u, guard)) return false;
       if (!wait_bounded(bar(kBarMlFull), seg & 1u, guard)) return false;
       tc_fence_after();
-      const float2 mls = ml[(seg & 1u) * 128 + h];
+      const float2 m0 = ml[((seg & 1u) * 2 + 0) * 128 + h];
+      const float2 m1 = ml[((seg & 1u) * 2 + 1) * 128 + h];
+      const float2 mls = make_float2(m0.x, m0.y + m1.y);   // same max in both halves
       const float inv = mls.y > 0.f ? 1.f / mls.y : 0.f;
       float* dst = p.part_o + ((int64_t)slot * p.n_heads + (head_ok ? h : 0)) * kDLatent + 256 * rank;
 #pragma unroll 1
@@ -526,18 +537,26 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       tc_fence_after();
       {
         const __nv_bfloat16* qrow = p.q_abs + ((int64_t)c.b * p.n_heads + (head_ok ? h : 0)) * kRow;
+        // 36 chunks of 16 bytes, loaded 12 at a time so the loads overlap
 #pragma unroll 1
-        for (int grp = 0; grp < kKSteps / 2; ++grp) {
-          uint32_t r[16];
+        for (int batch = 0; batch < 3; ++batch) {
+          uint4 v[12];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int ci = grp * 4 + i;  // 16-byte chunk 0..35 of this CTA's 288 columns
+          for (int i = 0; i < 12; ++i) {
+            const int ci = batch * 12 + i;  // 16-byte chunk 0..35 of this CTA's 288 columns
             const int col = ci < 32 ? 256 * (int)rank + 8 * ci : kDLatent + 32 * (int)rank + 8 * (ci - 32);
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (head_ok) v = *reinterpret_cast<const uint4*>(qrow + col);
-            r[4 * i] = v.x; r[4 * i + 1] = v.y; r[4 * i + 2] = v.z; r[4 * i + 3] = v.w;
+            v[i] = head_ok ? *reinterpret_cast<const uint4*>(qrow + col) : make_uint4(0, 0, 0, 0);
           }
-          tmem_st16(lanes | (tmem + kTmemQ + 16 * grp), r);
+#pragma unroll
+          for (int grp = 0; grp < 3; ++grp) {
+            uint32_t r[16];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              r[4 * i] = v[4 * grp + i].x; r[4 * i + 1] = v[4 * grp + i].y;
+              r[4 * i + 2] = v[4 * grp + i].z; r[4 * i + 3] = v[4 * grp + i].w;
+            }
+            tmem_st16(lanes | (tmem + kTmemQ + 16 * (3 * batch + grp)), r);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
@@ -573,6 +592,20 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
+// c^KV as a 3-D tensor (64 columns, rows, 8 column groups of 64): one box {64, 64, 4} is four
+// consecutive 64x64 boxes in shared memory, each row 128 bytes under the 128-byte swizzle.
+bool encode_latent_groups(CUtensorMap* m, const void* base, uint64_t rows, int64_t row_stride) {
+  const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[3] = {64, rows, kDLatent / 64};
+  const cuuint64_t strides[2] = {(cuuint64_t)row_stride * 2, 128};
+  const cuuint32_t box[3] = {64, (cuuint32_t)kT, 4};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, int64_t row_stride,
                  uint32_t box_cols, CUtensorMapSwizzle swz) {
   const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
@@ -602,7 +635,7 @@ cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfl
                                                 : (int64_t)batch * cv.seq_stride;
   if (rows <= 0 || rows >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
   CUtensorMap tc, tr;
-  if (!encode_rows(&tc, cv.c_kv, kDLatent, (uint64_t)rows, cv.row_stride, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  if (!encode_latent_groups(&tc, cv.c_kv, (uint64_t)rows, cv.row_stride) ||
       !encode_rows(&tr, cv.k_r, kDRope, (uint64_t)rows, cv.row_stride, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
 

@@ -62,6 +62,7 @@ constexpr uint32_t kBoxC = kT * 128;      // 8 KB: 64 tokens x 64 c^KV columns
 constexpr uint32_t kBoxR = kT * 64;       // 4 KB: 64 tokens x 32 k^R columns
 constexpr uint32_t kStageBytes = 4 * kBoxC + kBoxR;   // 36 KB
 constexpr uint32_t kXinBytes = 128 * kT * 4;          // 32 KB: 128 heads x 64 fp32
+constexpr uint32_t kXBlockBytes = kXinBytes / 8;       // one softmax warp's 32 heads x 32 tokens
 constexpr uint32_t kOffXin = kStages * kStageBytes;
 constexpr uint32_t kOffMl = kOffXin + 2 * kXinBytes;  // [2 segs][2 halves][128] float2 (max, sum)
 constexpr uint32_t kOffHmax = kOffMl + 2 * 2 * 128 * 8;  // [2 tiles][2 halves][128] float
@@ -73,8 +74,6 @@ constexpr int kBarKvEmpty = kStages;             // [kStages] PV of the tile don
 constexpr int kBarSFull = 2 * kStages;           // partial S in TMEM (+1 unused)
 constexpr int kBarSEmpty = kBarSFull + 2;        // softmax copied S out (+1 unused)
 constexpr int kBarPFull = kBarSFull + 4;         // P in TMEM, O rescaled, V tail zeroed (+1 unused)
-constexpr int kBarXFull = kBarSFull + 6;         // [2] the peer's partial scores arrived
-constexpr int kBarXFree = kBarSFull + 8;         // [2] the peer has read what we sent
 constexpr int kBarPvDone = kBarSFull + 10;       // a PV finished
 constexpr int kBarQReady = kBarSFull + 11;       // query columns of the next segment in TMEM
 constexpr int kBarQFree = kBarSFull + 12;        // the last QK of a segment finished
@@ -82,9 +81,9 @@ constexpr int kBarOFull = kBarSFull + 13;        // the last PV of a segment fin
 constexpr int kBarOFree = kBarSFull + 14;        // the epilogue has read O
 constexpr int kBarMlFull = kBarSFull + 15;       // (max, sum) of a finished segment in smem
 constexpr int kBarFinal = kBarSFull + 16;        // all MMAs of this CTA done (teardown)
-constexpr int kBarXRead = kBarSFull + 17;        // [2] our softmax warps read the peer's scores
-constexpr int kBarFinal2 = kBarXRead + 2;        // all PV MMAs done (teardown)
-constexpr int kNumBars = kBarFinal2 + 1;
+constexpr int kBarFinal2 = kBarSFull + 17;       // all PV MMAs done (teardown)
+constexpr int kBarXFull = kBarSFull + 18;        // [2 buffers][8 softmax warps] peer's block landed
+constexpr int kNumBars = kBarXFull + 16;
 constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;
 constexpr uint32_t kSmemUsed = kOffMisc + 128;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;     // room to align the base to 1 KB
@@ -207,11 +206,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     mbar_init(bar(kBarSEmpty), 256);
     mbar_init(bar(kBarPFull), 256);
     mbar_init(bar(kBarFinal2), 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(kBarXFull + i), 1);
-      mbar_init(bar(kBarXFree + i), 1);
-      mbar_init(bar(kBarXRead + i), 8);
-    }
+    for (int i = 0; i < 16; ++i) mbar_init(bar(kBarXFull + i), 1);
     mbar_init(bar(kBarPvDone), 1);
     mbar_init(bar(kBarQReady), 128);
     mbar_init(bar(kBarQFree), 1);
@@ -220,9 +215,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     mbar_init(bar(kBarMlFull), 256);
     mbar_init(bar(kBarFinal), 1);
     *abort_flag = 0;
-    // the receive buffers expect their first tile of partial scores
-    mbar_arrive_expect_tx(bar(kBarXFull + 0), kXinBytes);
-    mbar_arrive_expect_tx(bar(kBarXFull + 1), kXinBytes);
+    // every softmax warp's block of both buffers expects its first tile of partial scores
+    for (int i = 0; i < 16; ++i) mbar_arrive_expect_tx(bar(kBarXFull + i), kXBlockBytes);
     fence_mbarrier_init_cluster();
     prefetch_tmap(&tmap_c);
     prefetch_tmap(&tmap_r);
@@ -306,21 +300,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       wait_teardown(bar(kBarFinal), 0, p.wait_limit);
     }
   } else if (warp == 2) {
-    // ------------------------------------------------------------ PV issuer and relay
-    // Relay: when our softmax warps have read the peer's scores of tile g, re-arm the receive
-    // barrier for tile g + 2 and tell the peer that buffer g % 2 is free again (so no
-    // softmax warp waits on a cross-SM round trip). That always happens before P(g) is ready.
-    // PV: O += P(g) . V(g) once P(g) is in TMEM and (first tile of a segment) the previous
+    // ------------------------------------------------------------ PV issuer
+    // O += P(g) . V(g) once P(g) is in TMEM and (first tile of a segment) the previous
     // segment's O has been read out. Its completion frees the stage, P, and O.
     if (lane == 0) {
-      const uint32_t peer_xfree = map_to_rank(bar(kBarXFree), peer);
       TileCursor c;
       c.init(p);
       for (; c.valid; c.next(p)) {
-        const uint32_t g = c.g, st = g % kStages, xb = g & 1u;
-        if (!wait_bounded(bar(kBarXRead + xb), (g >> 1) & 1u, guard)) break;
-        mbar_arrive_expect_tx(bar(kBarXFull + xb), kXinBytes);
-        mbar_arrive_remote_relaxed(peer_xfree + 8u * xb);
+        const uint32_t g = c.g, st = g % kStages;
         if (!wait_bounded(bar(kBarPFull), g & 1u, guard)) break;
         if (c.first() && c.seg > 0 && !wait_bounded(bar(kBarOFree), (c.seg - 1) & 1u, guard)) break;
         tc_fence_after();
@@ -347,29 +334,40 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     const uint32_t lanes = (uint32_t)(32 * quarter) << 16;
     const int tid = threadIdx.x - 128;                  // 0..255 among the softmax threads
     const uint32_t pair_bar = 1u + (uint32_t)quarter;   // named barrier of the two warps of a head
+    const int w = warp - 4;                             // softmax warp 0..7: its block of a buffer
     const uint32_t xin = sbase + kOffXin;
     const uint32_t peer_xin = map_to_rank(xin, peer);
-    const uint32_t peer_xfull = map_to_rank(bar(kBarXFull), peer);
-    const uint32_t rowoff = (uint32_t)h * (kT * 4);
+    const uint32_t peer_xfull = map_to_rank(bar(kBarXFull + w), peer);   // + 64 bytes per buffer
+    const uint32_t blk = (uint32_t)w * kXBlockBytes;
+    const uint32_t rowoff = blk + (uint32_t)lane * (kHalf * 4);   // this thread's 32 scores
     const uint32_t col0 = (uint32_t)(kHalf * half);
 
-    // own partial S of this half of tile g: out of TMEM (freeing S for the next QK once both
-    // halves are out), then to the peer's receive buffer g % 2 (16-byte chunks,
-    // XOR-swizzled by head to spread the banks)
-    auto fetch_and_send = [&](uint32_t g, uint32_t (&dst)[kHalf]) -> bool {
-      const uint32_t xb = g & 1u;
+    // own partial S of this half of tile g out of TMEM (freeing S for the next QK once both
+    // halves are out)
+    auto fetch = [&](uint32_t g, uint32_t (&dst)[kHalf]) -> bool {
       if (!wait_spin(bar(kBarSFull), g & 1u, guard)) return false;
       tc_fence_after();
       tmem_ld32_sync(lanes | (tmem + kTmemS + col0), dst);
       tc_fence_before();
       mbar_arrive(bar(kBarSEmpty));
-      if (!wait_spin(bar(kBarXFree + xb), ((g >> 1) & 1u) ^ 1u, guard)) return false;
-      const uint32_t row = peer_xin + xb * kXinBytes + rowoff;
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        st_async_v4(row + (uint32_t)(((c + 8 * half) ^ (h & 7)) * 16), dst[4 * c], dst[4 * c + 1],
-                    dst[4 * c + 2], dst[4 * c + 3], peer_xfull + 8u * xb);
       return true;
+    };
+    // ... and to the peer. The block is staged in our buffer (g + 1) % 2, whose scores of
+    // tile g - 1 this warp has already read, and copied in one bulk transfer into the peer's
+    // buffer g % 2. That buffer is free: the peer read tile g - 2 there, then staged its own
+    // tile g - 1 there, and that copy has landed (we waited for it before calling this).
+    // Rows are 128 bytes (one head, 32 tokens) in 16-byte chunks XOR-swizzled by lane.
+    auto send = [&](uint32_t g, const uint32_t (&v)[kHalf]) {
+      const uint32_t sb = (g + 1) & 1u, db = g & 1u;
+      const uint32_t row = xin + sb * kXinBytes + rowoff;
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        st_shared_v4(row + (uint32_t)((q ^ (lane & 7)) * 16), v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0)
+        bulk_copy_to_peer(peer_xin + db * kXinBytes + blk, xin + sb * kXinBytes + blk, kXBlockBytes,
+                          peer_xfull + 64u * db);
     };
 
     uint32_t total = 0;   // tiles of this cluster's work
@@ -383,8 +381,10 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     uint32_t nxt[kHalf];
     float m_used = -INFINITY, l = 0.f;   // l: this half's share of the normaliser
     bool ok = true;
+    uint32_t consumed = 0;               // tiles whose peer scores this warp has read
     if (c.valid) {
-      ok = fetch_and_send(0, nxt);
+      ok = fetch(0, nxt);
+      if (ok) send(0, nxt);
 #pragma unroll
       for (int j = 0; j < kHalf; ++j) cur[j] = __uint_as_float(nxt[j]);
     }
@@ -392,21 +392,23 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       const uint32_t g = c.g, st = g % kStages, xb = g & 1u;
       if (!wait_spin(bar(kBarKvFull + st), (g / kStages) & 1u, guard)) break;
       const int r = tile_valid[st] ? c.rows() : 0;
-      if (g + 1 < total) {
-        if (!fetch_and_send(g + 1, nxt)) break;
-      }
+      const bool more = g + 1 < total;
+      if (more && !fetch(g + 1, nxt)) break;
       // the peer's partial scores of tile g: S = own + peer (the same sum on both CTAs)
-      if (!wait_spin(bar(kBarXFull + xb), (g >> 1) & 1u, guard)) break;
+      const uint32_t xfull = bar(kBarXFull + 8 * (int)xb + w);
+      if (!wait_spin(xfull, (g >> 1) & 1u, guard)) break;
+      if (lane == 0) mbar_arrive_expect_tx(xfull, kXBlockBytes);   // the block of tile g + 2
       {
         const float4* row = reinterpret_cast<const float4*>(smem + kOffXin + xb * kXinBytes + rowoff);
 #pragma unroll
         for (int q = 0; q < kHalf / 4; ++q) {
-          const float4 v = row[(q + 8 * half) ^ (h & 7)];
+          const float4 v = row[q ^ (lane & 7)];
           cur[4 * q] += v.x; cur[4 * q + 1] += v.y; cur[4 * q + 2] += v.z; cur[4 * q + 3] += v.w;
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBarXRead + xb));   // the relay frees the buffer
+      consumed = g + 1;
+      __syncwarp();   // the block is read by all lanes before tile g + 1 is staged over it
+      if (more) send(g + 1, nxt);
 
       // online softmax in the log2 domain: p = 2^(s * scale * log2(e) - m)
       if (c.first()) { m_used = -INFINITY; l = 0.f; }
@@ -491,6 +493,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
 #pragma unroll
       for (int j = 0; j < kHalf; ++j) cur[j] = __uint_as_float(nxt[j]);
     }
+    // after an abort: blocks the peer may still have in flight to us land before we leave
+    for (uint32_t t = consumed; t < consumed + 2 && t < total; ++t)
+      wait_teardown(bar(kBarXFull + 8 * (int)(t & 1u) + w), (t >> 1) & 1u, p.wait_limit >> 10);
   } else {
     // ------------------------------------------------------------ segment transitions
     regs_dec<kRegsTrans>();

@@ -230,6 +230,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   cluster_sync();  // the peer's barriers are initialised before anyone signals them
+  grid_dependency_wait();   // the plan, the query and the cache come from earlier kernels
+  allow_dependent_launch();
 
   const WaitGuard guard{abort_flag, p.err, kErrTimeout, p.wait_limit};
 
@@ -514,17 +516,21 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       const float2 m1 = ml[((seg & 1u) * 2 + 1) * 128 + h];
       const float2 mls = make_float2(m0.x, m0.y + m1.y);   // same max in both halves
       const float inv = mls.y > 0.f ? 1.f / mls.y : 0.f;
-      float* dst = p.part_o + ((int64_t)slot * p.n_heads + (head_ok ? h : 0)) * kDLatent + 256 * rank;
+      // partial O as [slot][column quad][head][4 floats]: the 32 heads of a warp write 512
+      // contiguous bytes per store
+      const int64_t quad_stride = (int64_t)p.n_heads * 4;
+      float* dst = p.part_o + ((int64_t)slot * (kDLatent / 4) + 64 * rank) * quad_stride +
+                   (head_ok ? h : 0) * 4;
 #pragma unroll 1
       for (int cc = 0; cc < 8; ++cc) {
         uint32_t o[32];
         tmem_ld32_sync(lanes | (tmem + kTmemO + 32 * cc), o);
         if (head_ok) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4*>(dst + 32 * cc + j) =
-                make_float4(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv,
-                            __uint_as_float(o[j + 2]) * inv, __uint_as_float(o[j + 3]) * inv);
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4*>(dst + (8 * cc + q) * quad_stride) =
+                make_float4(__uint_as_float(o[4 * q]) * inv, __uint_as_float(o[4 * q + 1]) * inv,
+                            __uint_as_float(o[4 * q + 2]) * inv, __uint_as_float(o[4 * q + 3]) * inv);
         }
       }
       if (head_ok && rank == 0)
@@ -660,14 +666,8 @@ cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfl
   p.wait_limit = 2000000000LL;  // SM cycles, about a second
 
   const int pairs = std::max(1, std::min(h.units, h.num_sms / 2));
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemAlloc;
-  cfg.stream = s;
-  cfg.attrs = nullptr;  // the 2-CTA cluster shape is compiled into the kernel
-  cfg.numAttrs = 0;
-  return cudaLaunchKernelEx(&cfg, decode_split_tc, tc, tr, p);
+  // the 2-CTA cluster shape is compiled into the kernel
+  return launch_pdl(decode_split_tc, dim3(2 * pairs), dim3(kThreads), kSmemAlloc, s, tc, tr, p);
 }
 
 }  // namespace mla

@@ -13,6 +13,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 
 #include "mla_internal.cuh"
@@ -35,7 +36,7 @@ struct GemmParams {
   __nv_bfloat16* out;             // q_abs [B, n_h, 576] or out [B, n_h, 128]
   const __nv_bfloat16* q_r;       // absorb only
   const int32_t* kv_lens;         // absorb only
-  double rope_base;
+  double theta[kDRope / 2];       // absorb only: RoPE frequencies base^(-2m/d_R), 0 when off
   uint32_t* err;
   long long wait_limit;
 };
@@ -51,10 +52,41 @@ __device__ __forceinline__ bool wait_simple(uint32_t bar, uint32_t parity, const
   return true;
 }
 
+// RoPE of the decoupled query of this head for the CTA's sequences, rotated to position
+// kv_len - 1. The angle pos * theta_m reaches ~1.3e5 rad at 128K tokens, so it is formed in
+// double and brought into [-pi, pi] by Cody-Waite reduction with a two-term 2*pi before the
+// sine and cosine are taken; the result is exact to far below bf16 resolution.
+__device__ __forceinline__ void rope_rows(const GemmParams& p, int h, int b0) {
+  constexpr double kTwoPiHi = 6.283185307179586;            // nearest double to 2*pi
+  constexpr double kTwoPiLo = 2.4492935982947064e-16;       // 2*pi - kTwoPiHi
+  constexpr double kInvTwoPi = 0.15915494309189535;
+  for (int i = threadIdx.x; i < p.n_tile * (kDRope / 2); i += kThreads) {
+    const int b = b0 + i / (kDRope / 2), m = i % (kDRope / 2);
+    if (b >= p.batch) continue;
+    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(
+        p.q_r + ((int64_t)b * p.n_heads + h) * kDRope + 2 * m);
+    const float x0 = __low2float(x), x1 = __high2float(x);
+    double y0 = x0, y1 = x1;
+    if (p.theta[m] != 0.0) {
+      const double a = (double)max(p.kv_lens[b] - 1, 0) * p.theta[m];
+      const double k = rint(a * kInvTwoPi);
+      const double r = fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, a));
+      double sn, cs;
+      sincos(r, &sn, &cs);
+      y0 = (double)x0 * cs - (double)x1 * sn;
+      y1 = (double)x0 * sn + (double)x1 * cs;
+    }
+    __nv_bfloat162 y;
+    y.x = __double2bfloat16(y0);   // one rounding, from double
+    y.y = __double2bfloat16(y1);
+    *reinterpret_cast<__nv_bfloat162*>(p.out + ((int64_t)b * p.n_heads + h) * kRow + kDLatent + 2 * m) = y;
+  }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
-             const GemmParams p) {
+             const __grid_constant__ CUtensorMap tmap_o, const GemmParams p) {
   // MODE kAbsorb:    D[c, b] = sum_d W_UK[h][d][c] x[b][d]   (A = W_UK, M-major; 4 M blocks, K = 128)
   // MODE kUpProject: D[d, b] = sum_c W_UV[h][d][c] x[b][c]   (A = W_UV, K-major; 1 M block,  K = 512)
   constexpr int kMBlocks = MODE == kAbsorb ? 4 : 1;
@@ -78,6 +110,12 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
     mbar_init(bars, 1);        // operands landed
     mbar_init(bars + 8, 1);    // MMAs done
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefetch_tmap(&tmap_w);
+    prefetch_tmap(&tmap_x);
+    prefetch_tmap(&tmap_o);
+    // the head's weights into L2 while the previous kernel finishes (a hint only: L2 is
+    // where writes land, so it cannot return stale data)
+    for (int i = 0; i < 8; ++i) tma_prefetch_2d(&tmap_w, 64 * i, 128 * h);
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), tmem_cols);
@@ -87,6 +125,8 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dependency_wait();   // inputs may come from the kernel before; outputs may be read by it
+  allow_dependent_launch();
 
   bool ok = true;
   if (threadIdx.x == 0) {
@@ -94,6 +134,9 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
     for (int i = 0; i < 8; ++i) tma_load_2d(sbase + i * kWeightBox, &tmap_w, 64 * i, 128 * h, bars);
     const int xcol = h * (MODE == kAbsorb ? kDHead : kDLatent);
     for (int i = 0; i < kXBoxes; ++i) tma_load_2d(xbase + i * xbox, &tmap_x, xcol + 64 * i, b0, bars);
+  }
+  if (MODE == kAbsorb) rope_rows(p, h, b0);   // needs no weights: runs while they load
+  if (threadIdx.x == 0) {
     ok = wait_simple(bars, 0, p);
     tc_fence_after();
     if (ok) {
@@ -124,48 +167,33 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
   tc_fence_after();
   ok = *reinterpret_cast<volatile int*>(smem + (bars - sbase) + 20) != 0;
 
-  // epilogue: TMEM lane = output feature, column = sequence
+  // epilogue: TMEM lane = output feature, column = sequence. The tile goes out through
+  // shared memory (the weights' buffer, free once the MMAs are done) as boxes of 64 features
+  // x n_tile sequences, written by TMA: a warp's direct stores would each cover only the
+  // 64 bytes of one output row.
   const uint32_t lanes = (uint32_t)(32 * warp) << 16;
+  const uint32_t obox = (uint32_t)p.n_tile * 128;   // bytes of one 64-feature output box
   if (ok) {
     for (int mb = 0; mb < kMBlocks; ++mb) {
+      const int feat = 128 * mb + 32 * warp + lane;
+      uint8_t* col = smem + (feat >> 6) * obox + (feat & 63) * 2;
       for (int c0 = 0; c0 < p.n_tile; c0 += 32) {
         uint32_t r[32];
         tmem_ld32_sync(lanes | (tmem + mb * col_stride + c0), r);
-        const int feat = 128 * mb + 32 * warp + lane;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int b = b0 + c0 + j;
-          if (c0 + j < p.n_tile && b < p.batch) {
-            const float v = __uint_as_float(r[j]);
-            if (MODE == kAbsorb)
-              p.out[((int64_t)b * p.n_heads + h) * kRow + feat] = __float2bfloat16_rn(v);
-            else
-              p.out[((int64_t)b * p.n_heads + h) * kDHead + feat] = __float2bfloat16_rn(v);
-          }
-        }
+        for (int j = 0; j < 32; ++j)
+          if (c0 + j < p.n_tile)
+            *reinterpret_cast<__nv_bfloat16*>(col + (c0 + j) * 128) = __float2bfloat16_rn(__uint_as_float(r[j]));
       }
     }
+    fence_proxy_async_smem();
   }
-  if (MODE == kAbsorb) {
-    // RoPE of the decoupled query (angles in double: positions reach 2^17)
-    for (int i = threadIdx.x; i < p.n_tile * (kDRope / 2); i += kThreads) {
-      const int b = b0 + i / (kDRope / 2), m = i % (kDRope / 2);
-      if (b >= p.batch) continue;
-      const __nv_bfloat16* src = p.q_r + ((int64_t)b * p.n_heads + h) * kDRope + 2 * m;
-      const double x0 = __bfloat162float(src[0]), x1 = __bfloat162float(src[1]);
-      double y0 = x0, y1 = x1;
-      if (p.rope_base != 0.0) {
-        const int pos = max(p.kv_lens[b] - 1, 0);
-        const double theta = pow(p.rope_base, -2.0 * m / kDRope);
-        double sn, cs;
-        sincos((double)pos * theta, &sn, &cs);
-        y0 = x0 * cs - x1 * sn;
-        y1 = x0 * sn + x1 * cs;
-      }
-      __nv_bfloat16* dst = p.out + ((int64_t)b * p.n_heads + h) * kRow + kDLatent + 2 * m;
-      dst[0] = __double2bfloat16(y0);
-      dst[1] = __double2bfloat16(y1);
-    }
+  __syncthreads();
+  if (ok && threadIdx.x == 0) {
+    const int x0 = h * (MODE == kAbsorb ? kRow : kDHead);
+    for (int k = 0; k < kMBlocks * 2; ++k) tma_store_2d(&tmap_o, sbase + k * obox, x0 + 64 * k, b0);
+    bulk_commit_group();
+    bulk_wait_group0();
   }
   tc_fence_before();
   __syncthreads();
@@ -186,8 +214,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   return fn;
 }
 
-// A row-major bf16 matrix [rows, cols] as a TMA source with 64-column, 128-byte-swizzled boxes.
-bool encode(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// A row-major bf16 matrix [rows, cols] as a TMA source or destination with 64-column boxes.
+bool encode(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+            CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   const PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
   if (enc == nullptr) return false;
   const cuuint64_t dims[2] = {cols, rows};
@@ -195,7 +224,7 @@ bool encode(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint
   const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -207,9 +236,12 @@ cudaError_t launch(const mla_decode_s& h, int batch, const __nv_bfloat16* w, con
   constexpr int kCap = MODE == kAbsorb ? 128 : 64;  // weights + x boxes fit in shared memory
   const int n_tile = std::min(kCap, (batch + 15) / 16 * 16);
   const int kx = MODE == kAbsorb ? kDHead : kDLatent;
-  CUtensorMap tw, tx;
+  const int ko = MODE == kAbsorb ? kRow : kDHead;   // output row of one head
+  CUtensorMap tw, tx, to;
   if (!encode(&tw, w, (uint64_t)h.cfg.n_heads * kDHead, kDLatent, 128) ||
-      !encode(&tx, x, (uint64_t)batch, (uint64_t)h.cfg.n_heads * kx, (uint32_t)n_tile))
+      !encode(&tx, x, (uint64_t)batch, (uint64_t)h.cfg.n_heads * kx, (uint32_t)n_tile) ||
+      !encode(&to, out, (uint64_t)batch, (uint64_t)h.cfg.n_heads * ko, (uint32_t)n_tile,
+              CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   constexpr uint32_t kSmemMax = kWeightBytes + kXBoxes * kCap * 128 + 64 + 1024;
   static std::once_flag once;
@@ -227,13 +259,13 @@ cudaError_t launch(const mla_decode_s& h, int batch, const __nv_bfloat16* w, con
   p.out = out;
   p.q_r = q_r;
   p.kv_lens = kv_lens;
-  p.rope_base = (double)h.cfg.rope_base;
+  for (int m = 0; m < kDRope / 2; ++m)
+    p.theta[m] = h.cfg.rope_base > 0.f ? std::pow((double)h.cfg.rope_base, -2.0 * m / kDRope) : 0.0;
   p.err = h.ws.err;
   p.wait_limit = 2000000000LL;
   const uint32_t smem = kWeightBytes + kXBoxes * n_tile * 128 + 64 + 1024;
   dim3 grid(h.cfg.n_heads, (batch + n_tile - 1) / n_tile);
-  head_gemm_tc<MODE><<<grid, kThreads, smem, s>>>(tw, tx, p);
-  return cudaGetLastError();
+  return launch_pdl(head_gemm_tc<MODE>, grid, dim3(kThreads), smem, s, tw, tx, to, p);
 }
 
 }  // namespace

@@ -5,6 +5,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "mla_decode.h"
 
 namespace mla {
@@ -44,7 +46,7 @@ struct Workspace {
   size_t bytes = 0;
   uint32_t* err = nullptr;   // device error word
   PlanView plan{};
-  float* part_o = nullptr;   // [max_slots, n_h, 512] partial latent outputs (normalised)
+  float* part_o = nullptr;   // [max_slots, 128 quads, n_h, 4] partial latent outputs (normalised)
   float* part_lse = nullptr; // [max_slots, n_h]     their log-sum-exp
   int max_units = 0;
   int max_slots = 0;
@@ -62,6 +64,35 @@ struct mla_decode_s {
 };
 
 namespace mla {
+
+// Programmatic dependent launch. Every kernel of the library is launched with it, so its
+// launch and set-up (barriers, tensor memory, descriptor prefetch) overlap the tail of the
+// kernel before it on the stream. A kernel calls grid_dependency_wait() before it reads or
+// writes any global memory that earlier work on the stream may touch; that wait returns once
+// every earlier grid has completed and its writes are visible. allow_dependent_launch() lets
+// the next kernel start launching; it changes nothing about what that kernel may read.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Launchers (each returns the cudaGetLastError() of its launch).
 cudaError_t launch_absorb_q(const mla_decode_s& h, int batch, const __nv_bfloat16* q_c,

@@ -31,6 +31,8 @@ split_plan_kernel(const int32_t* __restrict__ kv_lens, int batch, int64_t max_kv
   __shared__ int32_t s_tstart[kMaxBatch + 1];
   __shared__ int32_t s_units;
   const int tid = threadIdx.x;
+  grid_dependency_wait();   // kv_lens, and the plan arrays the previous call's kernels read
+  allow_dependent_launch();
 
   for (int b = tid; b < batch; b += blockDim.x) {
     int64_t L = kv_lens[b];
@@ -99,9 +101,8 @@ split_plan_kernel(const int32_t* __restrict__ kv_lens, int batch, int64_t max_kv
 
 cudaError_t launch_split_plan(const mla_decode_s& h, int batch, const int32_t* kv_lens,
                               cudaStream_t s) {
-  split_plan_kernel<<<1, 256, 0, s>>>(kv_lens, batch, h.cfg.max_kv_len, h.units,
-                                      h.cfg.max_splits, h.ws.plan, h.ws.err);
-  return cudaGetLastError();
+  return launch_pdl(split_plan_kernel, dim3(1), dim3(256), 0, s, kv_lens, batch,
+                    (int64_t)h.cfg.max_kv_len, h.units, h.cfg.max_splits, h.ws.plan, h.ws.err);
 }
 
 }  // namespace mla

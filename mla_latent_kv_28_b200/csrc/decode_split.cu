@@ -287,12 +287,17 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
         if (!wait_bounded(bar(kBarSEmpty), (g & 1u) ^ 1u, guard)) break;
         if (c.first() && !wait_bounded(bar(kBarQReady), c.seg & 1u, guard)) break;
         tc_fence_after();
+        // One descriptor per operand region, stepped by adding the byte offset / 16 to its
+        // start-address field (bits 0-13): shared addresses stay below 2^18, so the field never
+        // carries into the next one. The issuing thread then spends one add per MMA instead of
+        // rebuilding a 64-bit descriptor, which is what bounds how fast one thread can issue.
         const uint32_t a = sbase + st * kStageBytes;
+        const uint64_t dc = smem_desc(a, 16, 1024, 2);             // the four c^KV boxes
+        const uint64_t dr = smem_desc(a + 4 * kBoxC, 16, 512, 4);  // the k^R box
 #pragma unroll
         for (int ks = 0; ks < kKSteps; ++ks) {
-          const uint64_t bd = ks < 16
-              ? smem_desc(a + (ks >> 2) * kBoxC + (ks & 3) * 32, 16, 1024, 2)
-              : smem_desc(a + 4 * kBoxC + (ks - 16) * 32, 16, 512, 4);
+          const uint64_t bd = ks < 16 ? dc + (uint64_t)(((ks >> 2) * kBoxC + (ks & 3) * 32) >> 4)
+                                      : dr + (uint64_t)(((ks - 16) * 32) >> 4);
           mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * ks, bd, kIdescQK, ks > 0 ? 1u : 0u);
         }
         mma_commit(bar(kBarSFull));
@@ -313,11 +318,11 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
         if (!wait_bounded(bar(kBarPFull), g & 1u, guard)) break;
         if (c.first() && c.seg > 0 && !wait_bounded(bar(kBarOFree), (c.seg - 1) & 1u, guard)) break;
         tc_fence_after();
-        const uint32_t v = sbase + st * kStageBytes;
+        const uint64_t dv = smem_desc(sbase + st * kStageBytes, kBoxC, 1024, 2);
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk)
-          mma_ts(tmem + kTmemO, tmem + kTmemP + 8 * kk, smem_desc(v + kk * 2048, kBoxC, 1024, 2),
-                 kIdescPV, (!c.first() || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + kTmemO, tmem + kTmemP + 8 * kk, dv + (uint64_t)((kk * 2048) >> 4), kIdescPV,
+                 (!c.first() || kk > 0) ? 1u : 0u);
         mma_commit(bar(kBarKvEmpty + st));
         mma_commit(bar(kBarPvDone));
         if (c.last()) mma_commit(bar(kBarOFull));

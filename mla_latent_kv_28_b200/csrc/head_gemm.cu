@@ -6,10 +6,12 @@
 //
 // Both are a small batch of vectors times one 128x512 bf16 weight matrix per head, so they
 // are bound by reading the weights (16 MiB each at 128 heads). One CTA per (head, batch
-// chunk) pulls its head's 128 KB of weights with TMA, runs the product as tcgen05 MMAs with
-// the weights as the M = 128 operand ("swap AB": M = output features, N = batch), and writes
-// the accumulator back from tensor memory with one thread per output feature, so every
-// store instruction of a warp covers consecutive features of one sequence.
+// chunk) pulls its head's 128 KB of weights with TMA and runs the product as tcgen05 MMAs
+// with the weights as the M = 128 operand ("swap AB": M = output features, N = batch). A
+// single thread issues a small-N MMA only every ~80 cycles, so four warps issue in parallel
+// into separate accumulators: one 128-feature block each for the absorption, one quarter of
+// the 512-long reduction each for W_UV (the epilogue adds the four). The tile leaves tensor
+// memory through shared memory and TMA stores.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -24,7 +26,8 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;   // 8 warps: 4 MMA issuers, all 8 in the epilogue
+constexpr int kIssuers = 4;
 constexpr uint32_t kWeightBox = 128 * 128;      // 128 rows x 64 columns bf16 = 16 KB
 constexpr uint32_t kWeightBytes = 8 * kWeightBox;  // one head's 128 x 512 matrix
 
@@ -97,18 +100,19 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
   const uint32_t xbase = sbase + kWeightBytes;
   const uint32_t xbox = (uint32_t)p.n_tile * 128;        // bytes of one x box
   const uint32_t bars = xbase + kXBoxes * xbox;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (bars - sbase) + 16);
+  // barriers: [0] operands landed, [1..4] the MMAs of issuer q done; then the TMEM slot
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (bars - sbase) + 8 * (1 + kIssuers));
   const int h = blockIdx.x, b0 = blockIdx.y * p.n_tile;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // accumulator block mb sits at column mb * col_stride; the epilogue reads 32 columns at a
   // time, so a block never spans fewer than 32 allocated columns
   const uint32_t col_stride = p.n_tile < 32 ? 32u : (uint32_t)p.n_tile;
-  const uint32_t need = kMBlocks * col_stride;
+  const uint32_t need = kIssuers * col_stride;   // one accumulator per issuer
   const uint32_t tmem_cols = need <= 32 ? 32 : need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
 
   if (threadIdx.x == 0) {
-    mbar_init(bars, 1);        // operands landed
-    mbar_init(bars + 8, 1);    // MMAs done
+    mbar_init(bars, 1);                                             // operands landed
+    for (int q = 0; q < kIssuers; ++q) mbar_init(bars + 8 * (1 + q), 1);  // issuer q's MMAs done
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&tmap_w);
     prefetch_tmap(&tmap_x);
@@ -136,54 +140,71 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
     for (int i = 0; i < kXBoxes; ++i) tma_load_2d(xbase + i * xbox, &tmap_x, xcol + 64 * i, b0, bars);
   }
   if (MODE == kAbsorb) rope_rows(p, h, b0);   // needs no weights: runs while they load
-  if (threadIdx.x == 0) {
+  volatile int* ok_flags = reinterpret_cast<volatile int*>(smem + (bars - sbase) + 8 * (1 + kIssuers) + 4);
+  if (warp < kIssuers && lane == 0) {
+    const int q = warp;
     ok = wait_simple(bars, 0, p);
     tc_fence_after();
     if (ok) {
-#pragma unroll 1
-      for (int mb = 0; mb < kMBlocks; ++mb) {
-#pragma unroll 1
-        for (int kk = 0; kk < (MODE == kAbsorb ? 8 : 32); ++kk) {
-          uint64_t ad, bd;
-          if (MODE == kAbsorb) {
-            // A[c, d]: W_UK box (2mb) holds d rows x 64 c; 16 d rows per K step
-            ad = smem_desc(sbase + 2 * mb * kWeightBox + kk * 2048, kWeightBox, 1024, 2);
-            bd = smem_desc(xbase + (kk >> 2) * xbox + (kk & 3) * 32, 16, 1024, 2);
-          } else {
-            ad = smem_desc(sbase + (kk >> 2) * kWeightBox + (kk & 3) * 32, 16, 1024, 2);
-            bd = smem_desc(xbase + (kk >> 2) * xbox + (kk & 3) * 32, 16, 1024, 2);
-          }
-          mma_ss(tmem + mb * col_stride, ad, bd, p.idesc, kk > 0 ? 1u : 0u);
+      // absorb: accumulator q = output features [128q, 128q+128), K = 128 (8 steps);
+      // W_UV: accumulator q = the partial sum over latent columns [128q, 128q+128)
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        uint64_t ad, bd;
+        if (MODE == kAbsorb) {
+          // A[c, d]: W_UK box (2q) holds d rows x 64 c; 16 d rows per K step
+          ad = smem_desc(sbase + 2 * q * kWeightBox + kk * 2048, kWeightBox, 1024, 2);
+          bd = smem_desc(xbase + (kk >> 2) * xbox + (kk & 3) * 32, 16, 1024, 2);
+        } else {
+          const int k = 8 * q + kk;   // K step over the 512 latent columns
+          ad = smem_desc(sbase + (k >> 2) * kWeightBox + (k & 3) * 32, 16, 1024, 2);
+          bd = smem_desc(xbase + (k >> 2) * xbox + (k & 3) * 32, 16, 1024, 2);
         }
+        mma_ss(tmem + q * col_stride, ad, bd, p.idesc, kk > 0 ? 1u : 0u);
       }
-      mma_commit(bars + 8);
-      ok = wait_simple(bars + 8, 0, p);
+      mma_commit(bars + 8 * (1 + q));
+      ok = wait_simple(bars + 8 * (1 + q), 0, p);
     } else {
       wait_simple(bars, 0, p);  // never leave with copies in flight
     }
-    *reinterpret_cast<volatile int*>(smem + (bars - sbase) + 20) = ok ? 1 : 0;
+    ok_flags[q] = ok ? 1 : 0;
   }
   __syncthreads();
   tc_fence_after();
-  ok = *reinterpret_cast<volatile int*>(smem + (bars - sbase) + 20) != 0;
+  ok = ok_flags[0] && ok_flags[1] && ok_flags[2] && ok_flags[3];
 
   // epilogue: TMEM lane = output feature, column = sequence. The tile goes out through
   // shared memory (the weights' buffer, free once the MMAs are done) as boxes of 64 features
   // x n_tile sequences, written by TMA: a warp's direct stores would each cover only the
   // 64 bytes of one output row.
-  const uint32_t lanes = (uint32_t)(32 * warp) << 16;
+  // Warp w reads TMEM lanes [32(w%4), +32) and, of every 32 columns, the 16 of half w/4.
+  const uint32_t lanes = (uint32_t)(32 * (warp & 3)) << 16;
+  const int chalf = 16 * (warp >> 2);
   const uint32_t obox = (uint32_t)p.n_tile * 128;   // bytes of one 64-feature output box
   if (ok) {
     for (int mb = 0; mb < kMBlocks; ++mb) {
-      const int feat = 128 * mb + 32 * warp + lane;
+      const int feat = 128 * mb + 32 * (warp & 3) + lane;
       uint8_t* col = smem + (feat >> 6) * obox + (feat & 63) * 2;
-      for (int c0 = 0; c0 < p.n_tile; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32_sync(lanes | (tmem + mb * col_stride + c0), r);
+      for (int c0 = chalf; c0 < p.n_tile; c0 += 32) {
+        float v[16];
+        uint32_t r[16];
+        if (MODE == kAbsorb) {
+          tmem_ld16_sync(lanes | (tmem + mb * col_stride + c0), r);
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
+          for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = 0.f;
+          for (int q = 0; q < kIssuers; ++q) {   // the four partial sums over the latent columns
+            tmem_ld16_sync(lanes | (tmem + q * col_stride + c0), r);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] += __uint_as_float(r[j]);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
           if (c0 + j < p.n_tile)
-            *reinterpret_cast<__nv_bfloat16*>(col + (c0 + j) * 128) = __float2bfloat16_rn(__uint_as_float(r[j]));
+            *reinterpret_cast<__nv_bfloat16*>(col + (c0 + j) * 128) = __float2bfloat16_rn(v[j]);
       }
     }
     fence_proxy_async_smem();

@@ -24,84 +24,128 @@ __device__ int upper_index(const int32_t* v, int n, int t) {
   return lo;
 }
 
-__global__ void __launch_bounds__(256)
+constexpr int kPlanThreads = 256;
+constexpr int kPerThread = kMaxBatch / kPlanThreads;   // sequences per thread (4)
+
+// Exclusive prefix sum over the block of x[0..n) (n <= kMaxBatch) into out[0..n], out[n] = total.
+// Each thread scans its kPerThread consecutive entries, the warps scan their threads with
+// shuffles, and one warp scans the warp totals.
+__device__ void block_exclusive_scan(const int32_t* x, int n, int32_t* out, int32_t* warp_tot) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int v[kPerThread];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
+    const int idx = tid * kPerThread + i;
+    v[i] = idx < n ? x[idx] : 0;
+    sum += v[i];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < kPlanThreads / 32 ? warp_tot[lane] : 0;
+    int ti = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, ti, o);
+      if (lane >= o) ti += y;
+    }
+    if (lane < kPlanThreads / 32) warp_tot[lane] = ti - t;   // exclusive warp offsets
+    if (lane == kPlanThreads / 32 - 1) warp_tot[kPlanThreads / 32] = ti;   // total
+  }
+  __syncthreads();
+  int run = warp_tot[warp] + incl - sum;
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
+    const int idx = tid * kPerThread + i;
+    if (idx < n) out[idx] = run;
+    run += v[i];
+  }
+  if (tid == 0) out[n] = warp_tot[kPlanThreads / 32];
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kPlanThreads)
 split_plan_kernel(const int32_t* __restrict__ kv_lens, int batch, int64_t max_kv_len,
                   int units_target, int max_splits, PlanView plan, uint32_t* err) {
-  __shared__ int32_t s_tiles[kMaxBatch];
+  __shared__ int32_t s_a[kMaxBatch + 1];      // per-sequence counts
   __shared__ int32_t s_tstart[kMaxBatch + 1];
-  __shared__ int32_t s_units;
+  __shared__ int32_t s_aux[kMaxBatch + 1];
+  __shared__ int32_t s_warp[kPlanThreads / 32 + 1];
   const int tid = threadIdx.x;
   grid_dependency_wait();   // kv_lens, and the plan arrays the previous call's kernels read
   allow_dependent_launch();
 
-  for (int b = tid; b < batch; b += blockDim.x) {
+  for (int b = tid; b < batch; b += kPlanThreads) {
     int64_t L = kv_lens[b];
     if (L < 0 || L > max_kv_len) {
       atomicOr(err, kErrBadKvLen);
       L = L < 0 ? 0 : max_kv_len;
     }
     plan.seq_len[b] = (int32_t)L;
-    s_tiles[b] = (int32_t)((L + kTileTokens - 1) / kTileTokens);
+    s_a[b] = (int32_t)((L + kTileTokens - 1) / kTileTokens);   // tiles of sequence b
   }
   __syncthreads();
+  block_exclusive_scan(s_a, batch, s_tstart, s_warp);
+  const int total = s_tstart[batch];
+  for (int b = tid; b <= batch; b += kPlanThreads) plan.seq_tile[b] = s_tstart[b];
 
-  if (tid == 0) {
-    int acc = 0;
-    for (int b = 0; b < batch; ++b) { s_tstart[b] = acc; acc += s_tiles[b]; }
-    s_tstart[batch] = acc;
-    const int total = acc;
-    int n_units = 0;
-    if (total > 0) {
-      if (max_splits == 0) {
-        const int per = (total + units_target - 1) / units_target;
-        n_units = (total + per - 1) / per;
-        for (int u = 0; u < n_units; ++u) plan.unit_begin[u] = u * per;
-      } else {
-        for (int b = 0; b < batch; ++b) {
-          const int t = s_tiles[b];
-          const int n = t < max_splits ? t : max_splits;
-          for (int k = 0; k < n; ++k) plan.unit_begin[n_units++] = s_tstart[b] + (k * t) / n;
-        }
+  int n_units = 0;
+  if (total > 0) {
+    if (max_splits == 0) {
+      const int per = (total + units_target - 1) / units_target;
+      n_units = (total + per - 1) / per;
+      for (int u = tid; u < n_units; u += kPlanThreads) plan.unit_begin[u] = u * per;
+    } else {
+      // sequence b is cut into min(max_splits, tiles) near-equal ranges
+      for (int b = tid; b < batch; b += kPlanThreads) s_aux[b] = min(s_a[b], max_splits);
+      __syncthreads();
+      block_exclusive_scan(s_aux, batch, s_aux, s_warp);
+      n_units = s_aux[batch];
+      for (int b = tid; b < batch; b += kPlanThreads) {
+        const int t = s_a[b], n = min(t, max_splits);
+        for (int k = 0; k < n; ++k) plan.unit_begin[s_aux[b] + k] = s_tstart[b] + (k * t) / n;
       }
     }
+  }
+  if (tid == 0) {
     plan.unit_begin[n_units] = total;
     plan.header[0] = total;
     plan.header[1] = n_units;
-    s_units = n_units;
-    for (int b = 0; b <= batch; ++b) plan.seq_tile[b] = s_tstart[b];
   }
-  __syncthreads();
-  const int n_units = s_units;
-  const int total = s_tstart[batch];
+  __threadfence_block();
+  __syncthreads();   // unit_begin is read back below
 
   // first sequence of each unit: the one whose tile range holds the unit's first tile
-  for (int u = tid; u < n_units; u += blockDim.x)
+  for (int u = tid; u < n_units; u += kPlanThreads)
     plan.unit_seq[u] = upper_index(s_tstart, batch, plan.unit_begin[u]);
   // first unit of each sequence, and how many units (slots) it spans
-  for (int b = tid; b < batch; b += blockDim.x) {
+  for (int b = tid; b < batch; b += kPlanThreads) {
     int n = 0, first = 0;
-    if (s_tiles[b] > 0) {
+    if (s_a[b] > 0) {
       first = upper_index(plan.unit_begin, n_units, s_tstart[b]);
-      const int last = upper_index(plan.unit_begin, n_units, s_tstart[b] + s_tiles[b] - 1);
+      const int last = upper_index(plan.unit_begin, n_units, s_tstart[b] + s_a[b] - 1);
       n = last - first + 1;
     }
     plan.seq_unit[b] = first;
-    s_tiles[b] = n;  // reuse: slots of sequence b
+    s_aux[b] = n;   // slots of sequence b
   }
   __syncthreads();
-  if (tid == 0) {
-    int acc = 0;
-    for (int b = 0; b < batch; ++b) { plan.seq_slot[b] = acc; acc += s_tiles[b]; }
-    plan.seq_slot[batch] = acc;
-  }
-  (void)total;
+  block_exclusive_scan(s_aux, batch, s_aux, s_warp);
+  for (int b = tid; b <= batch; b += kPlanThreads) plan.seq_slot[b] = s_aux[b];
 }
 
 }  // namespace
 
 cudaError_t launch_split_plan(const mla_decode_s& h, int batch, const int32_t* kv_lens,
                               cudaStream_t s) {
-  return launch_pdl(split_plan_kernel, dim3(1), dim3(256), 0, s, kv_lens, batch,
+  return launch_pdl(split_plan_kernel, dim3(1), dim3(kPlanThreads), 0, s, kv_lens, batch,
                     (int64_t)h.cfg.max_kv_len, h.units, h.cfg.max_splits, h.ws.plan, h.ws.err);
 }
 

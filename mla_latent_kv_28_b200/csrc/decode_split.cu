@@ -83,7 +83,15 @@ constexpr int kBarMlFull = kBarSFull + 15;       // (max, sum) of a finished seg
 constexpr int kBarFinal = kBarSFull + 16;        // all MMAs of this CTA done (teardown)
 constexpr int kBarFinal2 = kBarSFull + 17;       // all PV MMAs done (teardown)
 constexpr int kBarXFull = kBarSFull + 18;        // [2 buffers][8 softmax warps] peer's block landed
-constexpr int kNumBars = kBarXFull + 16;
+constexpr int kBarQReady0 = kBarXFull + 16;      // the first segment's query columns in TMEM
+constexpr int kBarQLanded = kBarQReady0 + 1;     // ... and in shared memory (stages 1-2)
+constexpr int kNumBars = kBarQLanded + 1;
+// The first segment's query columns arrive by TMA in stages 1-2 (exactly 72 KB: four 64-column
+// boxes of 128 heads with 128-byte swizzle, then one 32-column k^R box with 64-byte swizzle);
+// the producer fills those stages with cache tiles only after the query has moved to TMEM.
+constexpr uint32_t kQBoxC = 128 * 128;   // 16 KB
+constexpr uint32_t kQBytes = 4 * kQBoxC + 128 * 64;
+static_assert(kQBytes == 2 * kStageBytes, "query staging fills stages 1-2 exactly");
 constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;
 constexpr uint32_t kSmemUsed = kOffMisc + 128;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;     // room to align the base to 1 KB
@@ -178,8 +186,60 @@ __device__ __forceinline__ bool wait_teardown(uint32_t bar, uint32_t parity, lon
   return true;
 }
 
+// One third (12 of the 36 16-byte chunks) of this CTA's 288 query columns of head h of
+// sequence b, into TMEM columns [kTmemQ + 48 part, +48) of the calling warp's lanes.
+__device__ __forceinline__ void load_q_part(const Params& p, uint32_t tmem, uint32_t lanes, int h,
+                                            int b, int part, uint32_t rank) {
+  const bool head_ok = h < p.n_heads;
+  const __nv_bfloat16* qrow = p.q_abs + ((int64_t)b * p.n_heads + (head_ok ? h : 0)) * kRow;
+  uint4 v[12];
+#pragma unroll
+  for (int i = 0; i < 12; ++i) {
+    const int ci = part * 12 + i;  // 16-byte chunk 0..35 of this CTA's 288 columns
+    const int col = ci < 32 ? 256 * (int)rank + 8 * ci : kDLatent + 32 * (int)rank + 8 * (ci - 32);
+    v[i] = head_ok ? *reinterpret_cast<const uint4*>(qrow + col) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int grp = 0; grp < 3; ++grp) {
+    uint32_t r[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      r[4 * i] = v[4 * grp + i].x; r[4 * i + 1] = v[4 * grp + i].y;
+      r[4 * i + 2] = v[4 * grp + i].z; r[4 * i + 3] = v[4 * grp + i].w;
+    }
+    tmem_st16(lanes | (tmem + kTmemQ + 16 * (3 * part + grp)), r);
+  }
+}
+
+// The same third of the first segment's query columns, from the TMA copy in stages 1-2
+// (row h of each box, 16-byte chunks under the boxes' 128- and 64-byte swizzles).
+__device__ __forceinline__ void q_part_from_smem(const uint8_t* smem, uint32_t tmem, uint32_t lanes,
+                                                 int h, bool head_ok, int part) {
+  const uint8_t* q = smem + kStageBytes;
+  uint4 v[12];
+#pragma unroll
+  for (int i = 0; i < 12; ++i) {
+    const int ci = part * 12 + i;
+    const uint32_t off = ci < 32
+        ? (uint32_t)(ci >> 3) * kQBoxC + (uint32_t)h * 128 + (uint32_t)(((ci & 7) ^ (h & 7)) << 4)
+        : 4 * kQBoxC + (uint32_t)h * 64 + (uint32_t)((((ci - 32) & 3) ^ ((h >> 1) & 3)) << 4);
+    v[i] = head_ok ? *reinterpret_cast<const uint4*>(q + off) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int grp = 0; grp < 3; ++grp) {
+    uint32_t r[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      r[4 * i] = v[4 * grp + i].x; r[4 * i + 1] = v[4 * grp + i].y;
+      r[4 * i + 2] = v[4 * grp + i].z; r[4 * i + 3] = v[4 * grp + i].w;
+    }
+    tmem_st16(lanes | (tmem + kTmemQ + 16 * (3 * part + grp)), r);
+  }
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constant__ CUtensorMap tmap_r,
+                const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_qr,
                 const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -209,6 +269,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     for (int i = 0; i < 16; ++i) mbar_init(bar(kBarXFull + i), 1);
     mbar_init(bar(kBarPvDone), 1);
     mbar_init(bar(kBarQReady), 128);
+    mbar_init(bar(kBarQReady0), 384);
+    mbar_init(bar(kBarQLanded), 1);
     mbar_init(bar(kBarQFree), 1);
     mbar_init(bar(kBarOFull), 1);
     mbar_init(bar(kBarOFree), 128);
@@ -220,6 +282,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     fence_mbarrier_init_cluster();
     prefetch_tmap(&tmap_c);
     prefetch_tmap(&tmap_r);
+    prefetch_tmap(&tmap_q);
+    prefetch_tmap(&tmap_qr);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -249,9 +313,19 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       };
       TileCursor c;
       c.init(p);
+      if (c.valid) {   // the first segment's query columns: one request, ahead of the tiles
+        const int qrow = c.b * p.n_heads;
+        const uint32_t qdst = sbase + kStageBytes;
+        mbar_arrive_expect_tx(bar(kBarQLanded), kQBytes);
+        for (int i = 0; i < 4; ++i)
+          tma_load_2d(qdst + i * kQBoxC, &tmap_q, 256 * (int)rank + 64 * i, qrow, bar(kBarQLanded));
+        tma_load_2d(qdst + 4 * kQBoxC, &tmap_qr, kDLatent + 32 * (int)rank, qrow, bar(kBarQLanded));
+      }
       for (; c.valid; c.next(p)) {
         const uint32_t g = c.g, st = g % kStages;
         if (!wait_bounded(bar(kBarKvEmpty + st), ((g / kStages) & 1u) ^ 1u, guard)) break;
+        // stages 1-2 hold the first segment's query until it is in TMEM
+        if (g == 1 && !wait_bounded(bar(kBarQReady0), 0, guard)) break;
         const int64_t row = tile_row(c);
         const bool ok = row >= 0;
         if (!ok) atomicOr(p.err, kErrBadPage);
@@ -285,7 +359,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
         const uint32_t g = c.g, st = g % kStages;
         if (!wait_bounded(bar(kBarKvFull + st), (g / kStages) & 1u, guard)) break;
         if (!wait_bounded(bar(kBarSEmpty), (g & 1u) ^ 1u, guard)) break;
-        if (c.first() && !wait_bounded(bar(kBarQReady), c.seg & 1u, guard)) break;
+        if (c.first() && !wait_bounded(c.seg == 0 ? bar(kBarQReady0) : bar(kBarQReady),
+                                       c.seg == 0 ? 0u : (c.seg - 1) & 1u, guard))
+          break;
         tc_fence_after();
         // One descriptor per operand region, stepped by adding the byte offset / 16 to its
         // start-address field (bits 0-13): shared addresses stay below 2^18, so the field never
@@ -380,7 +456,16 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     uint32_t total = 0;   // tiles of this cluster's work
     {
       TileCursor t;
-      for (t.init(p); t.valid; t.next(p)) ++total;
+      t.init(p);
+      if (t.valid) {   // two thirds of the first segment's query columns (the rest: transitions)
+        if (wait_bounded(bar(kBarQLanded), 0, guard)) {
+          q_part_from_smem(smem, tmem, lanes, h, h < p.n_heads, half);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        mbar_arrive(bar(kBarQReady0));
+      }
+      for (; t.valid; t.next(p)) ++total;
     }
     TileCursor c;
     c.init(p);
@@ -552,37 +637,36 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       if (seg > 0 && !wait_bounded(bar(kBarQFree), (seg - 1) & 1u, guard)) break;
       tc_fence_after();
       {
-        const __nv_bfloat16* qrow = p.q_abs + ((int64_t)c.b * p.n_heads + (head_ok ? h : 0)) * kRow;
-        // 36 chunks of 16 bytes, loaded 12 at a time so the loads overlap
+        if (seg == 0) {
+          // the first segment's query: the softmax warps load the other two thirds, so the
+          // three batches of loads overlap instead of queueing behind the first cache tiles
+          if (wait_bounded(bar(kBarQLanded), 0, guard)) {
+            q_part_from_smem(smem, tmem, lanes, h, head_ok, 2);
+            tmem_wait_st();
+          }
+          tc_fence_before();
+          mbar_arrive(bar(kBarQReady0));
+        } else {
 #pragma unroll 1
-        for (int batch = 0; batch < 3; ++batch) {
-          uint4 v[12];
-#pragma unroll
-          for (int i = 0; i < 12; ++i) {
-            const int ci = batch * 12 + i;  // 16-byte chunk 0..35 of this CTA's 288 columns
-            const int col = ci < 32 ? 256 * (int)rank + 8 * ci : kDLatent + 32 * (int)rank + 8 * (ci - 32);
-            v[i] = head_ok ? *reinterpret_cast<const uint4*>(qrow + col) : make_uint4(0, 0, 0, 0);
-          }
-#pragma unroll
-          for (int grp = 0; grp < 3; ++grp) {
-            uint32_t r[16];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              r[4 * i] = v[4 * grp + i].x; r[4 * i + 1] = v[4 * grp + i].y;
-              r[4 * i + 2] = v[4 * grp + i].z; r[4 * i + 3] = v[4 * grp + i].w;
-            }
-            tmem_st16(lanes | (tmem + kTmemQ + 16 * (3 * batch + grp)), r);
-          }
+          for (int part = 0; part < 3; ++part) load_q_part(p, tmem, lanes, h, c.b, part, rank);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(kBarQReady));
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(kBarQReady));
       }
       // the previous segment's output, while this one runs
       if (seg > 0) ok = epilogue(seg - 1, prev_slot);
       prev_slot = c.slot;
-      // skip to the next segment
+      // skip to the next segment, and pull its query rows into L2 while this one runs
       while (c.valid && c.seg == seg) c.next(p);
+      if (c.valid && head_ok) {
+        const __nv_bfloat16* qrow = p.q_abs + ((int64_t)c.b * p.n_heads + h) * kRow;
+        asm volatile("prefetch.global.L2 [%0];" :: "l"(qrow + 256 * (int)rank) : "memory");
+        asm volatile("prefetch.global.L2 [%0];" :: "l"(qrow + 256 * (int)rank + 64) : "memory");
+        asm volatile("prefetch.global.L2 [%0];" :: "l"(qrow + 256 * (int)rank + 128) : "memory");
+        asm volatile("prefetch.global.L2 [%0];" :: "l"(qrow + 256 * (int)rank + 192) : "memory");
+        asm volatile("prefetch.global.L2 [%0];" :: "l"(qrow + kDLatent + 32 * (int)rank) : "memory");
+      }
       if (!c.valid && ok) ok = epilogue(seg, prev_slot);
     }
   }
@@ -623,12 +707,12 @@ bool encode_latent_groups(CUtensorMap* m, const void* base, uint64_t rows, int64
 }
 
 bool encode_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, int64_t row_stride,
-                 uint32_t box_cols, CUtensorMapSwizzle swz) {
+                 uint32_t box_cols, CUtensorMapSwizzle swz, uint32_t box_rows = kT) {
   const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {(cuuint64_t)row_stride * 2};
-  const cuuint32_t box[2] = {box_cols, (cuuint32_t)kT};
+  const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -650,9 +734,12 @@ cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfl
   const int64_t rows = cv.page_table != nullptr ? (int64_t)cv.num_pages * cv.page_size
                                                 : (int64_t)batch * cv.seq_stride;
   if (rows <= 0 || rows >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
-  CUtensorMap tc, tr;
+  CUtensorMap tc, tr, tq, tqr;
+  const uint64_t qrows = (uint64_t)batch * h.cfg.n_heads;   // q_abs as [B * n_h, 576]
   if (!encode_latent_groups(&tc, cv.c_kv, (uint64_t)rows, cv.row_stride) ||
-      !encode_rows(&tr, cv.k_r, kDRope, (uint64_t)rows, cv.row_stride, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+      !encode_rows(&tr, cv.k_r, kDRope, (uint64_t)rows, cv.row_stride, 32, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !encode_rows(&tq, q_abs, kRow, qrows, kRow, 64, CU_TENSOR_MAP_SWIZZLE_128B, 128) ||
+      !encode_rows(&tqr, q_abs, kRow, qrows, kRow, 32, CU_TENSOR_MAP_SWIZZLE_64B, 128))
     return cudaErrorInvalidValue;
 
   Params p{};
@@ -672,7 +759,7 @@ cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfl
 
   const int pairs = std::max(1, std::min(h.units, h.num_sms / 2));
   // the 2-CTA cluster shape is compiled into the kernel
-  return launch_pdl(decode_split_tc, dim3(2 * pairs), dim3(kThreads), kSmemAlloc, s, tc, tr, p);
+  return launch_pdl(decode_split_tc, dim3(2 * pairs), dim3(kThreads), kSmemAlloc, s, tc, tr, tq, tqr, p);
 }
 
 }  // namespace mla

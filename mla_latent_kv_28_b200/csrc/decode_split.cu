@@ -61,20 +61,26 @@ constexpr int kKSteps = 18;               // 288 columns / 16
 constexpr uint32_t kBoxC = kT * 128;      // 8 KB: 64 tokens x 64 c^KV columns
 constexpr uint32_t kBoxR = kT * 64;       // 4 KB: 64 tokens x 32 k^R columns
 constexpr uint32_t kStageBytes = 4 * kBoxC + kBoxR;   // 36 KB
-constexpr uint32_t kXinBytes = 128 * kT * 4;          // 32 KB: 128 heads x 64 fp32
-constexpr uint32_t kXBlockBytes = kXinBytes / 8;       // one softmax warp's 32 heads x 32 tokens
+// Partial scores cross between the two CTAs as 16-bit block floating point: per (head, tile)
+// 64 integers and one power-of-two scale. A softmax warp's block: 32 rows (heads) of 128 bytes,
+// then the 32 scale exponents. Each softmax warpgroup has two buffers of 4 blocks.
+constexpr uint32_t kXBlockBytes = 32 * 128 + 32 * 4;   // 4224
+constexpr uint32_t kXBufBytes = 4 * kXBlockBytes;       // one tile of one warpgroup (16.5 KB)
 constexpr uint32_t kOffXin = kStages * kStageBytes;
-constexpr uint32_t kOffMl = kOffXin + 2 * kXinBytes;  // [2 segs][2 halves][128] float2 (max, sum)
-constexpr uint32_t kOffHmax = kOffMl + 2 * 2 * 128 * 8;  // [2 tiles][2 halves][128] float
-constexpr uint32_t kOffBars = kOffHmax + 2 * 2 * 128 * 4;
+constexpr uint32_t kOffMl = kOffXin + 4 * kXBufBytes;  // [2 segs][2 warpgroups][128] float2 (max, sum)
+constexpr uint32_t kOffMh = kOffMl + 2 * 2 * 128 * 8;  // [128] float: running max handed between warpgroups
+constexpr uint32_t kOffBars = kOffMh + 128 * 4;
 
 // barrier indices
 constexpr int kBarKvFull = 0;                    // [kStages] TMA landed
 constexpr int kBarKvEmpty = kStages;             // [kStages] PV of the tile done
-constexpr int kBarSFull = 2 * kStages;           // partial S in TMEM (+1 unused)
-constexpr int kBarSEmpty = kBarSFull + 2;        // softmax copied S out (+1 unused)
-constexpr int kBarPFull = kBarSFull + 4;         // P in TMEM, O rescaled, V tail zeroed (+1 unused)
-constexpr int kBarPvDone = kBarSFull + 10;       // a PV finished
+// The softmax warpgroups take alternate tiles, so the signals between them and the issuers come
+// in pairs indexed by tile parity: each waiter then steps through the consecutive phases of
+// its own barrier, and a phase parity never names two different tiles.
+constexpr int kBarSFull = 2 * kStages;           // [2] partial S of tile g in TMEM (g % 2)
+constexpr int kBarSEmpty = kBarSFull + 2;        // [2] the softmax copied S(g) out
+constexpr int kBarPFull = kBarSFull + 4;         // [2] P(g) in TMEM, O rescaled, V tail zeroed
+constexpr int kBarPvDone = kBarSFull + 6;        // [2] PV(g) finished
 constexpr int kBarQReady = kBarSFull + 11;       // query columns of the next segment in TMEM
 constexpr int kBarQFree = kBarSFull + 12;        // the last QK of a segment finished
 constexpr int kBarOFull = kBarSFull + 13;        // the last PV of a segment finished
@@ -82,10 +88,11 @@ constexpr int kBarOFree = kBarSFull + 14;        // the epilogue has read O
 constexpr int kBarMlFull = kBarSFull + 15;       // (max, sum) of a finished segment in smem
 constexpr int kBarFinal = kBarSFull + 16;        // all MMAs of this CTA done (teardown)
 constexpr int kBarFinal2 = kBarSFull + 17;       // all PV MMAs done (teardown)
-constexpr int kBarXFull = kBarSFull + 18;        // [2 buffers][8 softmax warps] peer's block landed
+constexpr int kBarXFull = kBarSFull + 18;        // [2 warpgroups][2 buffers][4 warps] peer's block landed
 constexpr int kBarQReady0 = kBarXFull + 16;      // the first segment's query columns in TMEM
 constexpr int kBarQLanded = kBarQReady0 + 1;     // ... and in shared memory (stages 1-2)
-constexpr int kNumBars = kBarQLanded + 1;
+constexpr int kBarMHand = kBarQLanded + 1;       // [4 head quarters] running max of tile g-1 published
+constexpr int kNumBars = kBarMHand + 4;
 // The first segment's query columns arrive by TMA in stages 1-2 (exactly 72 KB: four 64-column
 // boxes of 128 heads with 128-byte swizzle, then one 32-column k^R box with 64-byte swizzle);
 // the producer fills those stages with cache tiles only after the query has moved to TMEM.
@@ -103,7 +110,7 @@ constexpr int kThreads = 512;   // 16 warps = 4 warpgroups (roles below)
 // 128 x (64 + 160 + 160 + 96) = 61,440 <= 65,536.
 constexpr int kRegsLaunch = 128, kRegsCtrl = 64, kRegsSoftmax = 160, kRegsTrans = 96;
 static_assert(128 * (kRegsCtrl + 2 * kRegsSoftmax + kRegsTrans) <= kThreads * kRegsLaunch, "register split");
-constexpr int kHalf = kT / 2;   // tokens per softmax thread
+static_assert(kBarPvDone + 2 <= kBarSFull + 10, "barrier map");
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kT, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, false, true);
 constexpr float kRescaleThreshold = 8.f;   // log2 units: rescale O only when the max grows more
@@ -250,7 +257,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   volatile int* tile_valid = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);  // [kStages]
   float2* ml = reinterpret_cast<float2*>(smem + kOffMl);                             // [2][2][128]
-  float* hmax = reinterpret_cast<float*>(smem + kOffHmax);                           // [2][2][128]
+  volatile float* mh = reinterpret_cast<volatile float*>(smem + kOffMh);             // [128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -262,15 +269,18 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       mbar_init(bar(kBarKvEmpty + i), 1);
       tile_valid[i] = 0;
     }
-    mbar_init(bar(kBarSFull), 1);
-    mbar_init(bar(kBarSEmpty), 256);
-    mbar_init(bar(kBarPFull), 256);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kBarSFull + i), 1);
+      mbar_init(bar(kBarSEmpty + i), 128);
+      mbar_init(bar(kBarPFull + i), 128);
+      mbar_init(bar(kBarPvDone + i), 1);
+    }
     mbar_init(bar(kBarFinal2), 1);
     for (int i = 0; i < 16; ++i) mbar_init(bar(kBarXFull + i), 1);
-    mbar_init(bar(kBarPvDone), 1);
     mbar_init(bar(kBarQReady), 128);
     mbar_init(bar(kBarQReady0), 384);
     mbar_init(bar(kBarQLanded), 1);
+    for (int i = 0; i < 4; ++i) mbar_init(bar(kBarMHand + i), 32);
     mbar_init(bar(kBarQFree), 1);
     mbar_init(bar(kBarOFull), 1);
     mbar_init(bar(kBarOFree), 128);
@@ -358,7 +368,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       for (; c.valid; c.next(p)) {
         const uint32_t g = c.g, st = g % kStages;
         if (!wait_bounded(bar(kBarKvFull + st), (g / kStages) & 1u, guard)) break;
-        if (!wait_bounded(bar(kBarSEmpty), (g & 1u) ^ 1u, guard)) break;
+        // S is free once the softmax copied S(g-1) out (tile g-1's warpgroup)
+        if (g > 0 && !wait_bounded(bar(kBarSEmpty + ((g - 1) & 1u)), ((g - 1) >> 1) & 1u, guard)) break;
         if (c.first() && !wait_bounded(c.seg == 0 ? bar(kBarQReady0) : bar(kBarQReady),
                                        c.seg == 0 ? 0u : (c.seg - 1) & 1u, guard))
           break;
@@ -376,12 +387,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
                                       : dr + (uint64_t)(((ks - 16) * 32) >> 4);
           mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * ks, bd, kIdescQK, ks > 0 ? 1u : 0u);
         }
-        mma_commit(bar(kBarSFull));
+        mma_commit(bar(kBarSFull + (g & 1u)));
         if (c.last()) mma_commit(bar(kBarQFree));
       }
       mma_commit(bar(kBarFinal));
       wait_teardown(bar(kBarFinal), 0, p.wait_limit);
     }
+  } else if (warp == 3) {
+    // idle
   } else if (warp == 2) {
     // ------------------------------------------------------------ PV issuer
     // O += P(g) . V(g) once P(g) is in TMEM and (first tile of a segment) the previous
@@ -391,7 +404,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       c.init(p);
       for (; c.valid; c.next(p)) {
         const uint32_t g = c.g, st = g % kStages;
-        if (!wait_bounded(bar(kBarPFull), g & 1u, guard)) break;
+        if (!wait_bounded(bar(kBarPFull + (g & 1u)), (g >> 1) & 1u, guard)) break;
         if (c.first() && c.seg > 0 && !wait_bounded(bar(kBarOFree), (c.seg - 1) & 1u, guard)) break;
         tc_fence_after();
         const uint64_t dv = smem_desc(sbase + st * kStageBytes, kBoxC, 1024, 2);
@@ -400,57 +413,82 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
           mma_ts(tmem + kTmemO, tmem + kTmemP + 8 * kk, dv + (uint64_t)((kk * 2048) >> 4), kIdescPV,
                  (!c.first() || kk > 0) ? 1u : 0u);
         mma_commit(bar(kBarKvEmpty + st));
-        mma_commit(bar(kBarPvDone));
+        mma_commit(bar(kBarPvDone + (g & 1u)));
         if (c.last()) mma_commit(bar(kBarOFull));
       }
       mma_commit(bar(kBarFinal2));
       wait_teardown(bar(kBarFinal2), 0, p.wait_limit);
     }
-  } else if (warp == 3) {
-    // idle
   } else if (warp < 12) {
     // ------------------------------------------------------------ softmax
+    // Two warpgroups take alternate tiles (wg = g % 2); a thread owns one head (its TMEM lane)
+    // and all 64 tokens of its warpgroup's tiles, so each warpgroup has two tile periods for a
+    // tile's fetch, exchange, exponentials and P. The running max passes from one tile to the
+    // next through shared memory and an mbarrier per head quarter (handoff k: tile k to k+1,
+    // produced only after handoff k-1 was consumed, so its phase parity is unambiguous); each warpgroup
+    // keeps its own share of the normaliser (relative to the max it last used), and the
+    // epilogue merges the two.
     regs_inc<kRegsSoftmax>();
     const int quarter = warp & 3;                       // TMEM lanes this warp may touch
-    const int half = (warp >> 2) - 1;                   // which 32 of the tile's 64 tokens
+    const int wg = (warp >> 2) - 1;                     // the tiles of parity wg are ours
     const int h = 32 * quarter + lane;                  // head = TMEM lane
     const uint32_t lanes = (uint32_t)(32 * quarter) << 16;
-    const int tid = threadIdx.x - 128;                  // 0..255 among the softmax threads
-    const uint32_t pair_bar = 1u + (uint32_t)quarter;   // named barrier of the two warps of a head
-    const int w = warp - 4;                             // softmax warp 0..7: its block of a buffer
+    const int tid = threadIdx.x - 128 - 128 * wg;       // 0..127 within the warpgroup
+    const uint32_t mhand = bar(kBarMHand + quarter);     // running-max handoff of these heads
     const uint32_t xin = sbase + kOffXin;
     const uint32_t peer_xin = map_to_rank(xin, peer);
-    const uint32_t peer_xfull = map_to_rank(bar(kBarXFull + w), peer);   // + 64 bytes per buffer
-    const uint32_t blk = (uint32_t)w * kXBlockBytes;
-    const uint32_t rowoff = blk + (uint32_t)lane * (kHalf * 4);   // this thread's 32 scores
-    const uint32_t col0 = (uint32_t)(kHalf * half);
+    const int xbar0 = kBarXFull + 8 * wg + quarter;     // + 4 * buffer
+    const uint32_t peer_xfull = map_to_rank(bar(xbar0), peer);   // + 32 bytes per buffer
+    const uint32_t blk = (uint32_t)quarter * kXBlockBytes;
+    const uint32_t rowoff = blk + (uint32_t)lane * 128;          // this head's 64 scores
+    const uint32_t expoff = blk + 32 * 128 + (uint32_t)lane * 4; // ... and their scale
+    auto xbuf = [&](uint32_t i) { return (uint32_t)(2 * wg + (int)i) * kXBufBytes; };
 
-    // own partial S of this half of tile g out of TMEM (freeing S for the next QK once both
-    // halves are out)
-    auto fetch = [&](uint32_t g, uint32_t (&dst)[kHalf]) -> bool {
-      if (!wait_spin(bar(kBarSFull), g & 1u, guard)) return false;
-      tc_fence_after();
-      tmem_ld32_sync(lanes | (tmem + kTmemS + col0), dst);
-      tc_fence_before();
-      mbar_arrive(bar(kBarSEmpty));
-      return true;
-    };
-    // ... and to the peer. The block is staged in our buffer (g + 1) % 2, whose scores of
-    // tile g - 1 this warp has already read, and copied in one bulk transfer into the peer's
-    // buffer g % 2. That buffer is free: the peer read tile g - 2 there, then staged its own
-    // tile g - 1 there, and that copy has landed (we waited for it before calling this).
-    // Rows are 128 bytes (one head, 32 tokens) in 16-byte chunks XOR-swizzled by lane.
-    auto send = [&](uint32_t g, const uint32_t (&v)[kHalf]) {
-      const uint32_t sb = (g + 1) & 1u, db = g & 1u;
-      const uint32_t row = xin + sb * kXinBytes + rowoff;
+    // Block floating point for the exchange: with 2^(e-1) <= max|s| < 2^e each score becomes
+    // k = round(s * 2^(14-e)) (|k| <= 2^14), within 2^-15 of the row's power-of-two ceiling; a
+    // row holding a non-finite score is sent as all-NaN (kNonFinite). No int/float conversion
+    // instructions (a quarter-rate pipe): fma(s, 2^(14-e), 2^23 + 2^15) rounds to the integer
+    // 2^23 + 2^15 + k, whose low 16 bits are k + 2^15; the receiver rebuilds the float
+    // 2^23 + (k + 2^15) from them with one byte permute and takes k * 2^(e-14) with one fma.
+    constexpr int kNonFinite = 1000;
+    constexpr float kMagic = 8421376.f;   // 2^23 + 2^15
+    auto quantize = [&](const float (&v)[kT], uint32_t (&q)[kT / 2]) -> int {
+      float am[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        st_shared_v4(row + (uint32_t)((q ^ (lane & 7)) * 16), v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      for (int i = 0; i < 8; ++i) am[i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < kT; ++j)   // max.NaN: a NaN anywhere survives into amax
+        asm("max.NaN.f32 %0, %0, %1;" : "+f"(am[j & 7]) : "f"(fabsf(v[j])));
+#pragma unroll
+      for (int i = 1; i < 8; ++i) asm("max.NaN.f32 %0, %0, %1;" : "+f"(am[0]) : "f"(am[i]));
+      const float amax = am[0];
+      const int eb = (int)((__float_as_uint(amax) >> 23) & 0xffu);
+      const int e = max(eb - 126, -100);
+      const float up = __uint_as_float((uint32_t)(141 - min(e, 128)) << 23);   // 2^(14 - e)
+#pragma unroll
+      for (int j = 0; j < kT / 2; ++j) {
+        const float2 y = ffma2(make_float2(v[2 * j], v[2 * j + 1]), make_float2(up, up), make_float2(kMagic, kMagic));
+        q[j] = __byte_perm(__float_as_uint(y.x), __float_as_uint(y.y), 0x5410);
+      }
+      return eb == 255 ? kNonFinite : e;
+    };
+    // Local tile u = g / 2 of this warpgroup lands in our buffer u % 2; our own block of tile u
+    // is staged in buffer (u+1) % 2 and copied in one bulk transfer into the peer's buffer
+    // u % 2. That is safe as soon as the peer's local tile u-1 has arrived here (awaited in
+    // our previous local tile): the peer sent it only after our tile u-2 had reached it, so our
+    // staging buffer (last used for tile u-2) has been read out and the peer is done with its
+    // buffer u % 2 (it read our tile u-2 there; its own u-1 staged there has landed with us).
+    auto send = [&](uint32_t u, const uint32_t (&q)[kT / 2], int e) {
+      const uint32_t base = xin + xbuf((u + 1) & 1u);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        st_shared_v4(base + rowoff + (uint32_t)((c ^ (lane & 7)) * 16), q[4 * c], q[4 * c + 1], q[4 * c + 2], q[4 * c + 3]);
+      asm volatile("st.shared.b32 [%0], %1;" :: "r"(base + expoff), "r"(e) : "memory");
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0)
-        bulk_copy_to_peer(peer_xin + db * kXinBytes + blk, xin + sb * kXinBytes + blk, kXBlockBytes,
-                          peer_xfull + 64u * db);
+        bulk_copy_to_peer(peer_xin + xbuf(u & 1u) + blk, base + blk, kXBlockBytes,
+                          peer_xfull + 32u * (u & 1u));
     };
 
     uint32_t total = 0;   // tiles of this cluster's work
@@ -459,7 +497,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       t.init(p);
       if (t.valid) {   // two thirds of the first segment's query columns (the rest: transitions)
         if (wait_bounded(bar(kBarQLanded), 0, guard)) {
-          q_part_from_smem(smem, tmem, lanes, h, h < p.n_heads, half);
+          q_part_from_smem(smem, tmem, lanes, h, h < p.n_heads, wg);
           tmem_wait_st();
         }
         tc_fence_before();
@@ -469,125 +507,164 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     }
     TileCursor c;
     c.init(p);
-    float cur[kHalf];
-    uint32_t nxt[kHalf];
-    float m_used = -INFINITY, l = 0.f;   // l: this half's share of the normaliser
+    float m_own = -INFINITY, l_own = 0.f;   // this warpgroup's max and normaliser share
+    int my_seg = -1;                        // segment of the last tile this warpgroup took
     bool ok = true;
-    uint32_t consumed = 0;               // tiles whose peer scores this warp has read
-    if (c.valid) {
-      ok = fetch(0, nxt);
-      if (ok) send(0, nxt);
-#pragma unroll
-      for (int j = 0; j < kHalf; ++j) cur[j] = __uint_as_float(nxt[j]);
-    }
+    uint32_t consumed = 0;                  // local tiles whose peer scores have been read
     for (; ok && c.valid; c.next(p)) {
-      const uint32_t g = c.g, st = g % kStages, xb = g & 1u;
-      if (!wait_spin(bar(kBarKvFull + st), (g / kStages) & 1u, guard)) break;
-      const int r = tile_valid[st] ? c.rows() : 0;
-      const bool more = g + 1 < total;
-      if (more && !fetch(g + 1, nxt)) break;
-      // the peer's partial scores of tile g: S = own + peer (the same sum on both CTAs)
-      const uint32_t xfull = bar(kBarXFull + 8 * (int)xb + w);
-      if (!wait_spin(xfull, (g >> 1) & 1u, guard)) break;
-      if (lane == 0) mbar_arrive_expect_tx(xfull, kXBlockBytes);   // the block of tile g + 2
-      {
-        const float4* row = reinterpret_cast<const float4*>(smem + kOffXin + xb * kXinBytes + rowoff);
+      const uint32_t g = c.g;
+      if ((int)(g & 1u) == wg) {
+        const uint32_t st = g % kStages, u = g >> 1, xb = u & 1u;
+        if (!wait_spin(bar(kBarKvFull + st), (g / kStages) & 1u, guard)) break;
+        const int r = tile_valid[st] ? c.rows() : 0;   // valid tokens of the tile
+        // own partial S out of TMEM (S is free for the next QK once we have it)
+        float sv[kT];
+        {
+          if (!wait_spin(bar(kBarSFull + wg), u & 1u, guard)) break;
+          tc_fence_after();
+          uint32_t a[32], b[32];
+          tmem_ld32_sync(lanes | (tmem + kTmemS), a);
+          tmem_ld32_sync(lanes | (tmem + kTmemS + 32), b);
+          tc_fence_before();
+          mbar_arrive(bar(kBarSEmpty + wg));
 #pragma unroll
-        for (int q = 0; q < kHalf / 4; ++q) {
-          const float4 v = row[q ^ (lane & 7)];
-          cur[4 * q] += v.x; cur[4 * q + 1] += v.y; cur[4 * q + 2] += v.z; cur[4 * q + 3] += v.w;
+          for (int j = 0; j < 32; ++j) { sv[j] = __uint_as_float(a[j]); sv[32 + j] = __uint_as_float(b[j]); }
         }
-      }
-      consumed = g + 1;
-      __syncwarp();   // the block is read by all lanes before tile g + 1 is staged over it
-      if (more) send(g + 1, nxt);
+        if (r < kT) {   // the last tile of a sequence (or a skipped page): what is not there is 0 ...
+#pragma unroll
+          for (int j = 0; j < kT; ++j) sv[j] = j < r ? sv[j] : 0.f;
+        }
+        {   // ... to the peer, then the peer's partial back: S = own + peer
+          uint32_t qv[kT / 2];
+          const int e = quantize(sv, qv);
+          send(u, qv, e);
+          const uint32_t xfull = bar(xbar0 + 4 * (int)xb);
+          if (!wait_spin(xfull, (u >> 1) & 1u, guard)) break;
+          if (lane == 0) mbar_arrive_expect_tx(xfull, kXBlockBytes);   // local tile u + 2
+          const uint8_t* buf = smem + kOffXin + xbuf(xb);
+          const int ep = *reinterpret_cast<const int*>(buf + expoff);
+          const float down = ep != kNonFinite ? __uint_as_float((uint32_t)(113 + ep) << 23)
+                                              : __int_as_float(0x7fc00000);
+          const float bias = -kMagic * down;   // exact: both are powers-of-two multiples
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            const uint4 v = *reinterpret_cast<const uint4*>(buf + rowoff + (uint32_t)((cc ^ (lane & 7)) * 16));
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float lo = __uint_as_float(__byte_perm(wv[i], 0x4B000000u, 0x7610));   // 2^23 + q
+              const float hi = __uint_as_float(__byte_perm(wv[i], 0x4B000000u, 0x7632));
+              const float2 t = ffma2(make_float2(lo, hi), make_float2(down, down), make_float2(bias, bias));
+              const float2 r2 = fadd2(make_float2(sv[8 * cc + 2 * i], sv[8 * cc + 2 * i + 1]), t);
+              sv[8 * cc + 2 * i] = r2.x;
+              sv[8 * cc + 2 * i + 1] = r2.y;
+            }
+          }
+          consumed = u + 1;
+        }
+        if (r < kT) {
+#pragma unroll
+          for (int j = 0; j < kT; ++j) sv[j] = j < r ? sv[j] : -INFINITY;
+        }
+        float mx[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = sv[i];
+#pragma unroll
+        for (int j = 8; j < kT; ++j) mx[j & 7] = fmaxf(mx[j & 7], sv[j]);
+        const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * p.scale_log2;
 
-      // online softmax in the log2 domain: p = 2^(s * scale * log2(e) - m)
-      if (c.first()) { m_used = -INFINITY; l = 0.f; }
-      const int rh = min(max(r - kHalf * half, 0), kHalf);   // valid tokens in this half
-      if (rh < kHalf) {  // the last tile of a sequence (or a skipped page): mask what is not there
+        // the running max after tile g-1, from the other warpgroup
+        float m_prev = -INFINITY;
+        if (g > 0) {
+          if (!wait_spin(mhand, (g - 1) & 1u, guard)) break;
+          m_prev = mh[h];
+        }
+        if (c.first()) m_prev = -INFINITY;          // a new segment starts from nothing
+        if (my_seg != c.seg) { m_own = -INFINITY; l_own = 0.f; my_seg = c.seg; }
+        float m_new = m_prev, alpha = 1.f;
+        bool need = false;
+        if (m_prev == -INFINITY) {
+          m_new = mt;
+        } else if (mt > m_prev + kRescaleThreshold) {   // rescale O only when the max grows a lot
+          m_new = mt;
+          need = true;
+          alpha = ex2_approx(m_prev - mt);
+        }
+        mh[h] = m_new;
+        if (g + 1 < total) mbar_arrive(mhand);
+        if (m_own != m_new) {   // our share of the normaliser to the new max
+          l_own = m_own == -INFINITY ? 0.f : l_own * ex2_approx(m_own - m_new);
+          m_own = m_new;
+        }
+        // P = 2^(s * scale * log2(e) - m)
+        // (with no live token yet every score is -inf and 2^-inf = 0, so no select is needed)
+        const float neg_m = m_new != -INFINITY ? -m_new : 0.f;
+        float2 sm[4];
 #pragma unroll
-        for (int j = 0; j < kHalf; ++j) cur[j] = j < rh ? cur[j] : -INFINITY;
-      }
-      float mx[8];
+        for (int i = 0; i < 4; ++i) sm[i] = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = cur[i];
-#pragma unroll
-      for (int j = 8; j < kHalf; ++j) mx[j & 7] = fmaxf(mx[j & 7], cur[j]);
-      float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      // the maximum over the whole tile: swap the half maxima with the partner warp
-      hmax[((g & 1u) * 2 + half) * 128 + h] = mt;
-      asm volatile("bar.sync %0, 64;" :: "r"(pair_bar) : "memory");
-      mt = fmaxf(mt, hmax[((g & 1u) * 2 + (half ^ 1)) * 128 + h]) * p.scale_log2;
-      float alpha = 1.f;
-      bool need = false;
-      if (m_used == -INFINITY) {
-        m_used = mt;
-      } else if (mt > m_used + kRescaleThreshold) {
-        need = true;
-        alpha = ex2_approx(m_used - mt);
-        m_used = mt;
-        l *= alpha;
-      }
-      const bool live = m_used != -INFINITY;
-      const float neg_m = live ? -m_used : 0.f;
-      float sm[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) sm[i] = 0.f;
-#pragma unroll
-      for (int j = 0; j < kHalf; ++j) {   // P in place
-        cur[j] = live ? ex2_approx(fmaf(cur[j], p.scale_log2, neg_m)) : 0.f;
-        sm[j & 7] += cur[j];
-      }
-      l += ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
-      const bool warp_need = __any_sync(0xffffffffu, need);
+        for (int j = 0; j < kT / 2; ++j) {
+          const float2 x = ffma2(make_float2(sv[2 * j], sv[2 * j + 1]), make_float2(p.scale_log2, p.scale_log2),
+                                 make_float2(neg_m, neg_m));
+          sv[2 * j] = ex2_approx(x.x);
+          sv[2 * j + 1] = ex2_approx(x.y);
+          sm[j & 3] = fadd2(sm[j & 3], make_float2(sv[2 * j], sv[2 * j + 1]));
+        }
+        l_own += ((sm[0].x + sm[0].y) + (sm[1].x + sm[1].y)) + ((sm[2].x + sm[2].y) + (sm[3].x + sm[3].y));
+        const bool warp_need = __any_sync(0xffffffffu, need);
 
-      // the previous PV is done: O may be rescaled and P (read by PV(g-1)) overwritten
-      if (!wait_spin(bar(kBarPvDone), (g & 1u) ^ 1u, guard)) break;
-      tc_fence_after();
-      if (warp_need) {   // this half rescales O columns [128 half, 128 half + 128)
+        // PV(g-1) is done: O may be rescaled and P (read by PV(g-1)) overwritten
+        if (g > 0 && !wait_spin(bar(kBarPvDone + ((g - 1) & 1u)), ((g - 1) >> 1) & 1u, guard)) break;
+        tc_fence_after();
+        if (warp_need) {   // O (all 256 columns of this head) to the new max
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t o[32];
-          const uint32_t col = kTmemO + 128 * half + 32 * cc;
-          tmem_ld32_sync(lanes | (tmem + col), o);
+          for (int cc = 0; cc < 8; ++cc) {
+            uint32_t o[32];
+            const uint32_t col = kTmemO + 32 * cc;
+            tmem_ld32_sync(lanes | (tmem + col), o);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          tmem_st32(lanes | (tmem + col), o);
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+            tmem_st32(lanes | (tmem + col), o);
+          }
         }
-      }
-      {   // P as bf16 pairs: this half's 16 columns
-        uint32_t pk[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(cur[2 * j], cur[2 * j + 1]);
-          pk[j] = *reinterpret_cast<uint32_t*>(&b2);
+        for (int hf = 0; hf < 2; ++hf) {   // P as bf16 pairs, 32 columns
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(sv[32 * hf + 2 * j], sv[32 * hf + 2 * j + 1]);
+            pk[j] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+          tmem_st16(lanes | (tmem + kTmemP + 16 * hf), pk);
         }
-        tmem_st16(lanes | (tmem + kTmemP + 16 * half), pk);
-      }
-      tmem_wait_st();
-      if (r < kT) {
-        // rows past the sequence end (or of a skipped page) must not reach P.V as NaN/Inf
-        uint8_t* stage = smem + st * kStageBytes;
-        for (int i = tid; i < (kT - r) * 32; i += 256) {
-          const int row = r + (i >> 5), box = (i >> 3) & 3, chunk = i & 7;
-          *reinterpret_cast<uint4*>(stage + box * kBoxC + row * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+        tmem_wait_st();
+        if (r < kT) {
+          // rows past the sequence end (or of a skipped page) must not reach P.V as NaN/Inf
+          uint8_t* stage = smem + st * kStageBytes;
+          for (int i = tid; i < (kT - r) * 32; i += 128) {
+            const int row = r + (i >> 5), box = (i >> 3) & 3, chunk = i & 7;
+            *reinterpret_cast<uint4*>(stage + box * kBoxC + row * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(kBarPFull + wg));
       }
-      tc_fence_before();
-      mbar_arrive(bar(kBarPFull));
-      if (c.last()) {
-        ml[((c.seg & 1u) * 2 + half) * 128 + h] = make_float2(m_used, l);
+      if (c.last()) {   // segment done: this warpgroup's (max, share) for the epilogue
+        const bool mine = my_seg == c.seg;
+        ml[((c.seg & 1u) * 2 + wg) * 128 + h] = make_float2(mine ? m_own : -INFINITY, mine ? l_own : 0.f);
         mbar_arrive(bar(kBarMlFull));
       }
-#pragma unroll
-      for (int j = 0; j < kHalf; ++j) cur[j] = __uint_as_float(nxt[j]);
     }
-    // after an abort: blocks the peer may still have in flight to us land before we leave
-    for (uint32_t t = consumed; t < consumed + 2 && t < total; ++t)
-      wait_teardown(bar(kBarXFull + 8 * (int)(t & 1u) + w), (t >> 1) & 1u, p.wait_limit >> 10);
+    // after an abort: blocks the peer may still have in flight to us (it sends local tile u
+    // once our u-1 arrived) land before we leave
+    {
+      uint32_t nloc = 0;   // local tiles of this warpgroup
+      for (uint32_t t = (uint32_t)wg; t < total; t += 2) ++nloc;
+      for (uint32_t t = consumed; t < consumed + 2 && t < nloc; ++t)
+        wait_teardown(bar(xbar0 + 4 * (int)(t & 1u)), (t >> 1) & 1u, p.wait_limit >> 10);
+    }
   } else {
     // ------------------------------------------------------------ segment transitions
     regs_dec<kRegsTrans>();
@@ -604,7 +681,12 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       tc_fence_after();
       const float2 m0 = ml[((seg & 1u) * 2 + 0) * 128 + h];
       const float2 m1 = ml[((seg & 1u) * 2 + 1) * 128 + h];
-      const float2 mls = make_float2(m0.x, m0.y + m1.y);   // same max in both halves
+      // O is relative to the last max used (the larger: the max only grows); each warpgroup's
+      // share of the normaliser is relative to the max it used last
+      const float mlast = fmaxf(m0.x, m1.x);
+      const float l0 = m0.y > 0.f ? m0.y * exp2f(m0.x - mlast) : 0.f;
+      const float l1 = m1.y > 0.f ? m1.y * exp2f(m1.x - mlast) : 0.f;
+      const float2 mls = make_float2(mlast, l0 + l1);
       const float inv = mls.y > 0.f ? 1.f / mls.y : 0.f;
       // partial O as [slot][column quad][head][4 floats]: the 32 heads of a warp write 512
       // contiguous bytes per store

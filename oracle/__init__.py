@@ -1,6 +1,8 @@
 """fp64 CPU oracle of the MLA decode step. Test infrastructure only (see mla_oracle)."""
 
 from .mla_oracle import (  # noqa: F401
+    cache_rows,
+    rms_norm,
     D_HEAD,
     D_LATENT,
     D_ROPE,

@@ -43,6 +43,11 @@ Readings where the pages are silent (each is also listed in the design doc):
   * k^R in the cache is already rotated (it is rotated when it is written, [V3-walk]
     §2.2); the decode step reads it as it is.
   * kv_len == 0: the output is 0 and the log-sum-exp is -inf.
+  * The cache row of a new token (the step before decode): c^KV = W^DKV h ([V2-arch] eq. 9,
+    [V2-walk] §2.2), followed by an RMSNorm ([V2-notes] Architecture: an RMSNorm is added
+    after the compressed latent vectors) with a learned scale gamma and eps = 1e-6 by default
+    (the pages give no eps); k^R = RoPE(W^KR h) ([V3-walk] §2.2, §2.3), rotated at the new
+    token's position, which is L-1 once the token is counted in L.
 
 Cache layouts accepted (the row is [c^KV (d_c) ; k^R (d_R)], 576 values):
   * contiguous: array [B, Lmax, d_c + d_R];
@@ -153,6 +158,31 @@ def softmax_lse(s: np.ndarray, axis: int = 0):
     p = e / z
     lse = np.squeeze(m + np.log(z), axis=axis)
     return p, lse
+
+
+# ---------------------------------------------------------------------------
+# the cache row of a new token  ([V2-arch] eq. 9, [V2-notes] Architecture, [V3-walk] §2.2)
+# ---------------------------------------------------------------------------
+
+def rms_norm(x, gamma, eps: float = 1e-6) -> np.ndarray:
+    """x / sqrt(mean(x^2) + eps) * gamma over the last axis."""
+    x, gamma = widen(x), widen(gamma)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * gamma
+
+
+def cache_rows(hidden, w_dkv, w_kr, gamma, kv_lens, rope_base: float,
+               eps: float = 1e-6) -> np.ndarray:
+    """The row each sequence appends for its new token, [c^KV ; k^R] (576 values):
+        c^KV = RMSNorm(W^DKV h_b) * gamma,   k^R = RoPE_{kv_len[b]-1}(W^KR h_b).
+    hidden [B, d]; w_dkv [d_c, d]; w_kr [d_R, d]; gamma [d_c]. Returns [B, d_c + d_R]."""
+    hidden, w_dkv, w_kr = widen(hidden), widen(w_dkv), widen(w_kr)
+    kv_lens = np.asarray(kv_lens)
+    rows = np.zeros((hidden.shape[0], w_dkv.shape[0] + w_kr.shape[0]))
+    for b in range(hidden.shape[0]):
+        c = rms_norm(w_dkv @ hidden[b], gamma, eps)
+        kr = rope_rotate(w_kr @ hidden[b], int(kv_lens[b]) - 1, rope_base)
+        rows[b] = np.concatenate([c, kr])
+    return rows
 
 
 def default_scale(d_head: int = D_HEAD, d_rope: int = D_ROPE) -> float:

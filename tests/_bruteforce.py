@@ -63,3 +63,13 @@ def decode(q_c, q_r, w_uk, w_uv, rows_of, kv_lens, scale, rope_base):
         out.append(ob)
         lse.append(lb)
     return out, lse
+
+
+def cache_row(h, w_dkv, w_kr, gamma, kv_len, rope_base, eps=1e-6):
+    """The cache row of a new token, [RMSNorm(W^DKV h) * gamma ; RoPE_{kv_len-1}(W^KR h)]
+    (DeepSeek-V2 architecture page eq. 9 and its RMSNorm after the compressed latent;
+    DeepSeek-V3 walkthrough section 2.2 for the rotated k^R), with math.fsum for the sums."""
+    x = _matvec(w_dkv, h)
+    rms = math.sqrt(math.fsum(v * v for v in x) / len(x) + eps)
+    c = [v / rms * g for v, g in zip(x, gamma)]
+    return c + _rotate(_matvec(w_kr, h), kv_len - 1, rope_base)

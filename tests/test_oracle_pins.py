@@ -319,3 +319,70 @@ def test_planted_mistakes_are_caught(monkeypatch):
     # the two up-projections swapped (W_UK where W_UV belongs)
     got = om.mla_decode_nonabsorbed(q_c, q_r, w_uk, w_uk, cache, L, scale, 10000.0, pt, ps)
     assert not np.allclose(got, ref, atol=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# the cache row of a new token (the step before decode)
+# ---------------------------------------------------------------------------
+
+def test_rms_norm_closed_form_unit_rms_and_scale_invariance():
+    # [3, 4]: mean square 12.5, so [3, 4] / sqrt(12.5) = [0.8485..., 1.1313...]
+    y = oracle.rms_norm(np.array([3.0, 4.0]), np.ones(2), eps=0.0)
+    np.testing.assert_allclose(y, [3 / math.sqrt(12.5), 4 / math.sqrt(12.5)], rtol=1e-15)
+    rng = np.random.default_rng(40)
+    x = rng.standard_normal(512)
+    y = oracle.rms_norm(x, np.ones(512), eps=0.0)
+    assert abs(np.sqrt(np.mean(y * y)) - 1.0) < 1e-14
+    np.testing.assert_allclose(oracle.rms_norm(7.5 * x, np.ones(512), eps=0.0), y, rtol=1e-13)
+    g = rng.standard_normal(512)
+    np.testing.assert_allclose(oracle.rms_norm(x, g, eps=0.0), y * g, rtol=1e-13)
+
+
+def _tiny_append(seed=41, d=16, d_c=8, d_r=4, B=3):
+    rng = np.random.default_rng(seed)
+    h = rng.standard_normal((B, d))
+    w_dkv = rng.standard_normal((d_c, d)) / math.sqrt(d)
+    w_kr = rng.standard_normal((d_r, d)) / math.sqrt(d)
+    gamma = 1.0 + 0.1 * rng.standard_normal(d_c)
+    lens = np.array([1, 5, 77])[:B]
+    return h, w_dkv, w_kr, gamma, lens
+
+
+def test_cache_rows_match_python_loops():
+    h, w_dkv, w_kr, gamma, lens = _tiny_append()
+    got = oracle.cache_rows(h, w_dkv, w_kr, gamma, lens, 10000.0)
+    for b in range(len(lens)):
+        ref = _bruteforce.cache_row(h[b].tolist(), w_dkv.tolist(), w_kr.tolist(), gamma.tolist(),
+                                    int(lens[b]), 10000.0)
+        np.testing.assert_allclose(got[b], ref, rtol=1e-12, atol=1e-14)
+
+
+def test_appended_key_and_query_at_the_same_position_keep_their_dot_product():
+    """The new token's k^R is rotated at kv_len-1, the position the decode step rotates the
+    query to: their dot product is the unrotated one (rotations by one angle cancel)."""
+    rng = np.random.default_rng(42)
+    d, d_r = 32, 64
+    h = rng.standard_normal((1, d))
+    w_kr = rng.standard_normal((d_r, d))
+    q_r = rng.standard_normal(d_r)
+    for L in (1, 2, 4097, 131072):
+        row = oracle.cache_rows(h, np.zeros((8, d)), w_kr, np.ones(8), [L], 10000.0)[0]
+        k_rot = row[8:]
+        q_rot = oracle.rope_rotate(q_r, L - 1, 10000.0)
+        assert abs(q_rot @ k_rot - q_r @ (w_kr @ h[0])) < 1e-9 * (1 + abs(q_r @ (w_kr @ h[0])))
+
+
+def test_cache_row_planted_mistakes_are_caught():
+    h, w_dkv, w_kr, gamma, lens = _tiny_append(seed=43)
+    good = oracle.cache_rows(h, w_dkv, w_kr, gamma, lens, 10000.0)
+    x = h @ w_dkv.T
+    # gamma dropped
+    no_gamma = x / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + 1e-6)
+    assert np.max(np.abs(no_gamma - good[:, :8])) > 1e-3
+    # the norm taken over the whole 576-wide row instead of the latent only
+    full = np.concatenate([x, h @ w_kr.T], axis=1)
+    whole = full / np.sqrt(np.mean(full * full, axis=1, keepdims=True) + 1e-6)
+    assert np.max(np.abs(whole[:, :8] * gamma - good[:, :8])) > 1e-3
+    # RoPE one position late (at kv_len instead of kv_len - 1)
+    late = np.stack([oracle.rope_rotate(w_kr @ h[b], int(lens[b]), 10000.0) for b in range(len(lens))])
+    assert np.max(np.abs(late - good[:, 8:])) > 1e-3

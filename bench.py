@@ -302,6 +302,56 @@ def workload_config(w, name):
             "rope_base": w.rope_base, "d_c": 512, "d_rope": 64, "d_head": 128}
 
 
+def append_kv_measure(h, w, g, caches, copies, stream, args, world, local, dev,
+                      d_model: int = 5120):
+    """The cache write of the step's new tokens (mla_append_kv) on the same workload, timed
+    alone from a graph of K calls. It is the step before the decode step, measured beside it
+    and not counted in the step's tokens/s. Its inputs rotate over enough weight copies that
+    they do not stay in L2 from one call to the next."""
+    inp = {k: v.to(dev) for k, v in wl.draw_append_inputs(w.batch, d_model, seed=7).items()}
+    wbytes = (inp["w_dkv"].numel() + inp["w_kr"].numel()) * 2
+    n_w = max(1, math.ceil(4 * L2_BYTES / wbytes))
+    weights = [(inp["w_dkv"], inp["w_kr"])] + [(inp["w_dkv"].clone(), inp["w_kr"].clone())
+                                               for _ in range(n_w - 1)]
+
+    def call(k):
+        wd, wr = weights[k % n_w]
+        h.append_kv(inp["hidden"], wd, wr, inp["gamma"], caches[k % copies], g.kv_lens,
+                    g.page_table, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for k in range(args.warmup):
+            call(k)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for k in range(args.steps):
+            call(k)
+    with torch.cuda.stream(stream):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    h.check_device_errors(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, local, True)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, local, True)
+    h.check_device_errors(stream)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    del graph
+    # algorithmic bytes: the two weights, the hidden states, gamma, the rows written
+    algo = wbytes + w.batch * d_model * 2 + 512 * 2 + w.batch * ROW_BYTES
+    hbm_gbs, _, peak_kind = measured_peaks()
+    gbs = algo / (ms * 1e-3) / 1e9
+    return {"us": ms * 1e3, "d_model": d_model, "batch": w.batch, "algorithmic_bytes": algo,
+            "achieved_gbs": gbs, "frac_of_hbm": gbs / hbm_gbs, "peak_source": f"{peak_kind} hbm_gbs",
+            "l2": f"{n_w} rotating weight copies of {wbytes / 1e6:.1f} MB",
+            "kernels": "kv_down_tc + kv_finalize", "gpu_launches": 2 * args.steps}
+
+
 def run_ours(args):
     rank, world, local = dist_env()
     if not torch.cuda.is_available():
@@ -439,6 +489,8 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / args.steps, world, dev)
     clocks.stop()
 
+    append = append_kv_measure(h, w, g, caches, copies, stream, args, world, local, dev)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tps, toks, secs = oracle_tokens_per_s(w)
@@ -471,6 +523,7 @@ def run_ours(args):
         "gpu_launches": 5 * args.steps,
         "clocks": clocks.summary(w0, w1),
     }
+    line["append_kv"] = append
     if cpu is not None:
         line["cpu_baseline"] = cpu
     h.close()

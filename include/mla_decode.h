@@ -137,6 +137,37 @@ int mla_apply_wuv(mla_handle_t h, int32_t batch, const void* latent, const void*
                   void* out, mla_stream_t stream);
 
 /*
+ * Cache write of the step's new token ([V2-arch] eq. 9 c^KV = W^DKV h; [V2-notes]
+ * architecture: an RMSNorm follows the compressed latent; [V3-walk] §2.2 k^R = RoPE(W^KR h)
+ * and only c^KV and k^R are cached):
+ *   x          = [W_DKV ; W_KR] hidden[b,:]                         (576, fp32 accumulation)
+ *   c^KV row   = x[0:512] / sqrt(mean(x[0:512]^2) + rms_eps) * gamma      (bf16)
+ *   k^R  row   = RoPE_{kv_lens[b]-1}(x[512:576])                          (bf16; pairs
+ *                (2m,2m+1), angle (kv_len-1) * base^(-2m/64); identity if rope_base == 0)
+ * written as token kv_lens[b]-1 of sequence b, in the layout mla_decode_attn reads; no other
+ * row is touched.
+ * d_model     hidden size d: a multiple of 64, 64..8192 (5120 for DeepSeek-V2)
+ * hidden      bf16 [batch, d_model]  the token's hidden state h_t (after the block's input norm)
+ * w_dkv       bf16 [512, d_model]    W^DKV, the nn.Linear weight of the down-projection
+ * w_kr        bf16 [64, d_model]     W^KR
+ * gamma       bf16 [512]             the latent RMSNorm's weight
+ * rms_eps     >= 0 and finite (1e-6 in DeepSeek-V2)
+ * c_kv, k_r, row_stride, seq_stride, page_table, max_pages, num_pages: the cache, as for
+ *             mla_decode_attn, here written
+ * kv_lens     int32 [batch], each 1..max_kv_len: tokens of the sequence with the new one;
+ *             a value outside that range (there is no row to write) or a page-table entry
+ *             outside 0..num_pages-1 sets the device error word and the sequence is skipped
+ * Errors: MLA_ERR_INVALID_ARG for NULL pointers, batch outside 1..max_batch, d_model not a
+ * positive multiple of 64, a bad rms_eps, strides or alignment, a page table given to a
+ * contiguous handle (or missing for a paged one); MLA_ERR_UNSUPPORTED for d_model > 8192.
+ */
+int mla_append_kv(mla_handle_t h, int32_t batch, int32_t d_model, const void* hidden,
+                  const void* w_dkv, const void* w_kr, const void* gamma, float rms_eps,
+                  void* c_kv, void* k_r, int64_t row_stride, int64_t seq_stride,
+                  const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                  int32_t num_pages, mla_stream_t stream);
+
+/*
  * mla_decode_attn for callers that cannot allocate device memory. The pages have no
  * counterpart to this call: it exists for library users whose device memory is owned by
  * someone else (a serving engine that has reserved nearly all of HBM for its own KV-cache
@@ -172,7 +203,7 @@ int mla_decode_attn_noalloc(int32_t n_heads, float softmax_scale, int32_t page_s
  * Synchronise `stream`, then read and clear the handle's device error word. Returns MLA_OK
  * if it was clear, MLA_ERR_DEVICE_CHECK if a kernel set it (*detail, if not NULL, gets the
  * word: bit 0 = page-table entry out of range, bit 1 = a bounded wait ran out, bit 2 = a
- * kv_len outside 0..max_kv_len, clamped), or
+ * kv_len outside 0..max_kv_len, clamped, or outside 1..max_kv_len in mla_append_kv), or
  * MLA_ERR_CUDA if the synchronisation itself failed.
  */
 int mla_check_device_errors(mla_handle_t h, mla_stream_t stream, uint32_t* detail);

@@ -57,6 +57,8 @@ SIGNATURES = {
     "mla_absorb_q": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P, _P, _P]),
     "mla_decode_attn": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32, _P, _P, _P]),
     "mla_apply_wuv": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P]),
+    "mla_append_kv": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _P, _P, ctypes.c_float, _P, _P,
+                                     _I64, _I64, _P, _P, _I32, _I32, _P]),
     "mla_decode_attn_noalloc": (ctypes.c_int, [_I32, ctypes.c_float, _I32, _I64, _I32, _P, _P, _P,
                                                _I64, _I64, _P, _P, _I32, _I32, _P, _P, _P, _P]),
     "mla_check_device_errors": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
@@ -177,15 +179,26 @@ class MlaDecode:
                                       _ptr(q_abs), _stream(stream)), "mla_absorb_q")
         return q_abs
 
-    def decode_attn(self, q_abs: torch.Tensor, cache: torch.Tensor, kv_lens: torch.Tensor,
-                    page_table: Optional[torch.Tensor] = None,
-                    out_latent: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                    want_lse: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-        """cache: contiguous [B, Lmax, 576] or paged [num_pages, page_size, 576] bf16 rows
-        [c^KV ; k^R]. Returns (out_latent [B, n_h, 512] bf16, lse [B, n_h] fp32 or None)."""
-        B, H = q_abs.shape[0], q_abs.shape[1]
-        _need(q_abs, torch.bfloat16, "q_abs")
+    def append_kv(self, hidden: torch.Tensor, w_dkv: torch.Tensor, w_kr: torch.Tensor,
+                  gamma: torch.Tensor, cache: torch.Tensor, kv_lens: torch.Tensor,
+                  page_table: Optional[torch.Tensor] = None, eps: float = 1e-6,
+                  stream=None) -> torch.Tensor:
+        """Write the new token's cache row [RMSNorm(W_DKV h)*gamma ; RoPE(W_KR h)] as token
+        kv_lens[b]-1 of every sequence b. hidden [B, d] bf16; w_dkv [512, d]; w_kr [64, d];
+        gamma [512]; cache as for decode_attn. Returns the cache."""
+        B, d = hidden.shape
+        for t, n in ((hidden, "hidden"), (w_dkv, "w_dkv"), (w_kr, "w_kr"), (gamma, "gamma")):
+            _need(t, torch.bfloat16, n)
         _need(kv_lens, torch.int32, "kv_lens")
+        row_stride, seq_stride, c_kv, k_r, max_pages, num_pages = self._cache_view(cache, page_table)
+        _check(self._lib.mla_append_kv(
+            self._h, B, d, _ptr(hidden), _ptr(w_dkv), _ptr(w_kr), _ptr(gamma), float(eps),
+            ctypes.c_void_p(c_kv), ctypes.c_void_p(k_r), row_stride, seq_stride, _ptr(kv_lens),
+            _ptr(page_table), max_pages, num_pages, _stream(stream)), "mla_append_kv")
+        return cache
+
+    @staticmethod
+    def _cache_view(cache: torch.Tensor, page_table: Optional[torch.Tensor]):
         if not cache.is_cuda or cache.dtype != torch.bfloat16 or cache.dim() != 3 or cache.stride(-1) != 1:
             raise ValueError("cache: expected a CUDA bf16 [*, *, 576] tensor with unit inner stride")
         row_stride = cache.stride(1)
@@ -198,6 +211,18 @@ class MlaDecode:
             max_pages = page_table.shape[1]
             num_pages = cache.shape[0]
             seq_stride = 0
+        return row_stride, seq_stride, c_kv, k_r, max_pages, num_pages
+
+    def decode_attn(self, q_abs: torch.Tensor, cache: torch.Tensor, kv_lens: torch.Tensor,
+                    page_table: Optional[torch.Tensor] = None,
+                    out_latent: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                    want_lse: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+        """cache: contiguous [B, Lmax, 576] or paged [num_pages, page_size, 576] bf16 rows
+        [c^KV ; k^R]. Returns (out_latent [B, n_h, 512] bf16, lse [B, n_h] fp32 or None)."""
+        B, H = q_abs.shape[0], q_abs.shape[1]
+        _need(q_abs, torch.bfloat16, "q_abs")
+        _need(kv_lens, torch.int32, "kv_lens")
+        row_stride, seq_stride, c_kv, k_r, max_pages, num_pages = self._cache_view(cache, page_table)
         if out_latent is None:
             out_latent = torch.empty((B, H, D_LATENT), dtype=torch.bfloat16, device=q_abs.device)
         if lse is None and want_lse:

@@ -87,6 +87,7 @@ int mla_decode_create(const mla_config_t* cfg, int device, mla_handle_t* out) {
   const size_t o_useq = off;      off = round_up(off + 4 * max_units, 256);
   const size_t o_plse = off;      off = round_up(off + 4 * (size_t)max_slots * cfg->n_heads, 256);
   const size_t o_po = off;        off = round_up(off + 4 * (size_t)max_slots * cfg->n_heads * kDLatent, 256);
+  const size_t o_ap = off;        off = round_up(off + 4 * (size_t)mla::kAppendSlices * B * mla::kRow, 256);
 
   void* base = nullptr;
   if (cudaMalloc(&base, off) != cudaSuccess) {
@@ -112,6 +113,7 @@ int mla_decode_create(const mla_config_t* cfg, int device, mla_handle_t* out) {
   h->ws.plan.unit_seq = reinterpret_cast<int32_t*>(p + o_useq);
   h->ws.part_lse = reinterpret_cast<float*>(p + o_plse);
   h->ws.part_o = reinterpret_cast<float*>(p + o_po);
+  h->ws.append_part = reinterpret_cast<float*>(p + o_ap);
   h->ws.max_units = max_units;
   h->ws.max_slots = max_slots;
   *out = h;
@@ -176,6 +178,45 @@ int mla_decode_attn(mla_handle_t h, int32_t batch, const void* q_abs, const void
     e = mla::launch_decode_split(*h, batch, static_cast<const __nv_bfloat16*>(q_abs), cv, stream);
   if (e == cudaSuccess)
     e = mla::launch_combine(*h, batch, static_cast<__nv_bfloat16*>(out_latent), lse, stream);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_append_kv(mla_handle_t h, int32_t batch, int32_t d_model, const void* hidden,
+                  const void* w_dkv, const void* w_kr, const void* gamma, float rms_eps,
+                  void* c_kv, void* k_r, int64_t row_stride, int64_t seq_stride,
+                  const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                  int32_t num_pages, mla_stream_t stream) {
+  if (h == nullptr || hidden == nullptr || w_dkv == nullptr || w_kr == nullptr ||
+      gamma == nullptr || c_kv == nullptr || k_r == nullptr || kv_lens == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > h->cfg.max_batch) return MLA_ERR_INVALID_ARG;
+  if (d_model < 64 || d_model % 64 != 0) return MLA_ERR_INVALID_ARG;
+  if (d_model > 8192) return MLA_ERR_UNSUPPORTED;
+  if (!(rms_eps >= 0.f) || !std::isfinite(rms_eps)) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(hidden) || !aligned16(w_dkv) || !aligned16(w_kr) || !aligned16(gamma) ||
+      !aligned16(c_kv) || !aligned16(k_r))
+    return MLA_ERR_INVALID_ARG;
+  if (row_stride < kDLatent || row_stride % 8 != 0) return MLA_ERR_INVALID_ARG;
+  mla::CacheView cv{};
+  cv.c_kv = static_cast<const __nv_bfloat16*>(c_kv);
+  cv.k_r = static_cast<const __nv_bfloat16*>(k_r);
+  cv.row_stride = row_stride;
+  cv.page_size = h->cfg.page_size;
+  if (h->cfg.page_size == 0) {
+    if (page_table != nullptr || seq_stride < h->cfg.max_kv_len) return MLA_ERR_INVALID_ARG;
+    cv.seq_stride = seq_stride;
+  } else {
+    const int64_t need = (h->cfg.max_kv_len + h->cfg.page_size - 1) / h->cfg.page_size;
+    if (page_table == nullptr || max_pages < need || num_pages < 1) return MLA_ERR_INVALID_ARG;
+    cv.page_table = page_table;
+    cv.max_pages = max_pages;
+    cv.num_pages = num_pages;
+  }
+  const cudaError_t e = mla::launch_append_kv(
+      *h, batch, d_model, static_cast<const __nv_bfloat16*>(hidden),
+      static_cast<const __nv_bfloat16*>(w_dkv), static_cast<const __nv_bfloat16*>(w_kr),
+      static_cast<const __nv_bfloat16*>(gamma), rms_eps, cv, static_cast<__nv_bfloat16*>(c_kv),
+      static_cast<__nv_bfloat16*>(k_r), kv_lens, stream);
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

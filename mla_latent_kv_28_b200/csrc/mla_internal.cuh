@@ -18,6 +18,7 @@ constexpr int kRow = kDLatent + kDRope;  // one cache row: [c^KV ; k^R]
 constexpr int kMaxHeads = 128;
 constexpr int kMaxBatch = 1024;
 constexpr int kTileTokens = 64;  // tokens per KV tile: the unit of the work plan
+constexpr int kAppendSlices = 16;  // the cache write's projection is split over at most 16 slices of d
 
 // Device error word bits (see mla_check_device_errors).
 constexpr uint32_t kErrBadPage = 1u << 0;
@@ -48,6 +49,7 @@ struct Workspace {
   PlanView plan{};
   float* part_o = nullptr;   // [max_slots, 128 quads, n_h, 4] partial latent outputs (normalised)
   float* part_lse = nullptr; // [max_slots, n_h]     their log-sum-exp
+  float* append_part = nullptr;  // [kAppendSlices, max_batch, 576] the cache write's partial sums
   int max_units = 0;
   int max_slots = 0;
 };
@@ -118,6 +120,12 @@ cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfl
 
 cudaError_t launch_combine(const mla_decode_s& h, int batch, __nv_bfloat16* out_latent,
                            float* lse, cudaStream_t s);
+
+cudaError_t launch_append_kv(const mla_decode_s& h, int batch, int d_model,
+                             const __nv_bfloat16* hidden, const __nv_bfloat16* w_dkv,
+                             const __nv_bfloat16* w_kr, const __nv_bfloat16* gamma, float eps,
+                             const CacheView& cv, __nv_bfloat16* c_kv, __nv_bfloat16* k_r,
+                             const int32_t* kv_lens, cudaStream_t s);
 
 cudaError_t launch_apply_wuv(const mla_decode_s& h, int batch, const __nv_bfloat16* latent,
                              const __nv_bfloat16* w_uv, __nv_bfloat16* out, cudaStream_t s);

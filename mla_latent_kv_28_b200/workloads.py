@@ -16,6 +16,10 @@ weights, q^C, q^R, kv lengths, cache, page assignment):
     With latent_scale="lognormal" each token's c^KV is multiplied by s_j ~ LogNormal(0, 0.5)
     before rounding (k^R is not scaled).
   * kv lengths: an int (all equal), a list, or ("uniform", lo, hi) drawn inclusive.
+  * cache write of a new token (draw_append_inputs, its own generator): hidden h [B, d]
+    N(0, 1); W_DKV [512, d] and W_KR [64, d] N(0, std = 1/sqrt(d)) (fan-in d); the latent
+    RMSNorm weight gamma [512] = 1 + 0.1 N(0, 1); all rounded to bf16. d = 5120 is
+    DeepSeek-V2's hidden size.
   * contiguous layout: cache [B, Lmax, 576]; rows at or past kv_len[b] are NaN.
   * paged layout: ceil(L_b / page_size) pages per sequence plus `spare_pages` spares form
     the physical pool [P, page_size, 576]; a seeded random permutation places the pages;
@@ -189,3 +193,15 @@ def draw_latent(batch: int, n_heads: int, seed: int = 2) -> torch.Tensor:
     """A stand-alone latent input [B, n_h, 512] bf16 ~ N(0, 1) for testing the W_UV call."""
     gen = torch.Generator().manual_seed(seed)
     return torch.randn((batch, n_heads, D_LATENT), generator=gen).to(torch.bfloat16)
+
+
+def draw_append_inputs(batch: int, d_model: int = 5120, seed: int = 3) -> dict:
+    """Inputs of the cache write of one decode step: hidden [B, d], w_dkv [512, d],
+    w_kr [64, d], gamma [512], all bf16 (recipe above)."""
+    gen = torch.Generator().manual_seed(seed)
+    wstd = 1.0 / math.sqrt(d_model)
+    hidden = _randn_bf16((batch, d_model), gen)
+    w_dkv = (torch.randn((D_LATENT, d_model), generator=gen) * wstd).to(torch.bfloat16)
+    w_kr = (torch.randn((D_ROPE, d_model), generator=gen) * wstd).to(torch.bfloat16)
+    gamma = (1.0 + 0.1 * torch.randn((D_LATENT,), generator=gen)).to(torch.bfloat16)
+    return {"hidden": hidden, "w_dkv": w_dkv, "w_kr": w_kr, "gamma": gamma}

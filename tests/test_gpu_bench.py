@@ -24,3 +24,5 @@ def test_bench_json_line():
     assert roof["bound"] == "hbm" and 0 < roof["frac"] < 1.5
     assert line["config"]["workload"] == "v2_b32_l4096"
     assert line["gpu_launches"] == 5 * 5
+    app = line["append_kv"]
+    assert app["us"] > 0 and 0 < app["frac_of_hbm"] < 1.5 and app["gpu_launches"] == 2 * 5

@@ -196,8 +196,14 @@ kv_finalize(const FinalParams p) {
     }
     row = (int64_t)page * p.cv.page_size + pos % p.cv.page_size;
   }
-  float x = 0.f;
-  for (int s = 0; s < p.slices; ++s) x += p.part[((int64_t)s * p.part_batch + b) * kRow + f];
+  // the slices' partial sums, all loads in flight at once, added in slice order
+  float v[kAppendSlices];
+#pragma unroll
+  for (int s = 0; s < kAppendSlices; ++s)
+    v[s] = s < p.slices ? p.part[((int64_t)s * p.part_batch + b) * kRow + f] : 0.f;
+  float x = v[0];
+#pragma unroll
+  for (int s = 1; s < kAppendSlices; ++s) x += v[s];
   xs[f] = x;
   // mean square of the 512 latent features: warp sums, then the 16 warp sums in order
   float sq = f < kDLatent ? x * x : 0.f;
@@ -265,7 +271,9 @@ cudaError_t launch_append_kv(const mla_decode_s& h, int batch, int d_model,
                              const __nv_bfloat16* w_kr, const __nv_bfloat16* gamma, float eps,
                              const CacheView& cv, __nv_bfloat16* c_kv, __nv_bfloat16* k_r,
                              const int32_t* kv_lens, cudaStream_t s) {
-  // slices of d: at most kAppendSlices, each a multiple of 64 columns (d itself is)
+  // slices of d: at most kAppendSlices, each a multiple of 64 columns (d itself is). (Slicing
+  // finer, to fill every SM, measured slower: the work is latency-bound at these sizes and
+  // more slices mean more partial sums to write and add.)
   const int slice = std::max(64, (d_model / kAppendSlices + 63) / 64 * 64);
   const int slices = (d_model + slice - 1) / slice;
   const int n_tile = std::min(64, (batch + 15) / 16 * 16);

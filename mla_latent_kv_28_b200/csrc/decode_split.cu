@@ -10,34 +10,31 @@
 // tensor memory, leaving no room for S. So the two CTAs of a cluster split the 576 columns
 // of every cache row: CTA r holds c^KV columns [256r, 256r+256) and k^R columns
 // [32r, 32r+32) (288 columns), computes the partial scores over them, and keeps the O
-// columns [256r, 256r+256). The two fp32 partial score tiles are swapped through
-// distributed shared memory (st.async, counted by the receiver's mbarrier); both CTAs then
-// add the same two tiles (S0 + S1, bit for bit the same sum) and run the same softmax, so
-// P, the running max and the normaliser agree without any further exchange. Each cache
-// byte is read from HBM once, by one CTA.
+// columns [256r, 256r+256). The partial score tiles cross between the two CTAs through
+// distributed shared memory (one bulk copy per warp, 16-bit block floating point); each CTA
+// adds its own exact partial to the peer's. Each cache byte is read from HBM once, by one CTA.
 //
 // Pipeline (64-token tiles, g = tile index within this cluster's work):
-//   TMA ring of 4 stages -> QK(g) into S -> softmax threads copy S(g+1) out of TMEM and
-//   send it to the peer while they finish tile g with the peer's S(g) -> P(g) -> PV(g).
-// A single thread can issue a tcgen05.mma only every ~50 cycles, far slower than the
-// tensor core retires small-N MMAs, so QK and PV have issuer warps of their own, and the
-// tile is 64 tokens wide (QK N = 64: 18 MMAs per 64 tokens, PV 4 MMAs of N = 256).
+//   TMA ring of 4 stages -> QK(g) into S -> softmax warpgroup g % 2: S out of TMEM, partial
+//   to the peer and the peer's back, max, exponentials, P(g) -> PV(g) into O.
+// Two softmax warpgroups take alternate tiles, so each has two tile periods for one tile.
+// QK and PV have issuer warps of their own (one thread issues an MMA only every ~60-90
+// cycles).
 // Segment boundaries (a unit may hold the tail of one sequence and the head of the next)
-// are handled by a separate warpgroup: it loads the next segment's query columns into
-// TMEM as soon as the last QK of the previous segment is done, and writes the finished
-// segment's O / l while the next segment is already running.
+// are handled by a separate warpgroup: it loads the next segment's query columns as soon as
+// the last QK of the previous segment is done, and writes the finished segment's O / l
+// while the next segment is already running.
 //
-// Tensor memory (512 columns per CTA): O [0,256) fp32, S [256,320) fp32, P [320,352)
-// bf16x2, Q [352,496) bf16x2 (the CTA's 288 query columns, the A operand of Q.K^T).
+// Tensor memory (512 columns per CTA): O [0,256) fp32, S [256,320) fp32, P [320,384) bf16x2
+// (one 32-column P per softmax warpgroup), Q [384,512) bf16x2 (the CTA's 256 c^KV query
+// columns, the A operand of the QK MMAs). The CTA's 32 k^R query columns are the A operand of
+// the two k^R MMAs from shared memory.
 // Shared memory: 4 stages x 36 KB of cache tiles (four 64x64 c^KV boxes with 128-byte
-// swizzle + one 64x32 k^R box with 64-byte swizzle), 2 x 32 KB receive buffers for the
-// peer's partial scores, per-segment (max, sum), mbarriers.
-// Warps: 0 TMA producer, 1 QK issuer (and TMEM owner), 2 PV issuer and relay (tells the
-// peer its scores were read, so no softmax warp waits on a cross-SM round trip), 3 idle;
-// 4..7 and 8..11 softmax, one thread per (head = TMEM lane, half of the tile's 64 tokens):
-// two warps per SM sub-partition hide each other's latencies, and the pair of threads of
-// a head agree on the tile maximum through shared memory; 12..15 segment transitions
-// (query load, epilogue).
+// swizzle + one 64x32 k^R box with 64-byte swizzle), 4 x 16.5 KB exchange buffers, the 8 KB
+// k^R query operand, per-segment (max, sum), mbarriers.
+// Warps: 0 TMA producer, 1 QK issuer (and TMEM owner), 2 PV issuer, 3 idle; 4..7 and 8..11
+// the two softmax warpgroups, one thread per head (= TMEM lane) and all 64 tokens of a tile;
+// 12..15 segment transitions (query load, epilogue).
 //
 // Every wait is bounded: after about a second it sets the device error word (timeout bit)
 // and the CTA's abort flag, all roles leave their loops, wait for their own copies and
@@ -67,9 +64,12 @@ constexpr uint32_t kStageBytes = 4 * kBoxC + kBoxR;   // 36 KB
 constexpr uint32_t kXBlockBytes = 32 * 128 + 32 * 4;   // 4224
 constexpr uint32_t kXBufBytes = 4 * kXBlockBytes;       // one tile of one warpgroup (16.5 KB)
 constexpr uint32_t kOffXin = kStages * kStageBytes;
-constexpr uint32_t kOffMl = kOffXin + 4 * kXBufBytes;  // [2 segs][2 warpgroups][128] float2 (max, sum)
+constexpr uint32_t kOffQr = kOffXin + 4 * kXBufBytes;  // [128 heads][32 k^R query columns], 64-byte swizzle
+constexpr uint32_t kQrBytes = 128 * 64;                 // 8 KB: the A operand of the two k^R MMAs
+constexpr uint32_t kOffMl = kOffQr + kQrBytes;         // [2 segs][2 warpgroups][128] float2 (max, sum)
 constexpr uint32_t kOffMh = kOffMl + 2 * 2 * 128 * 8;  // [128] float: running max handed between warpgroups
-constexpr uint32_t kOffBars = kOffMh + 128 * 4;
+constexpr uint32_t kOffEpi = kOffMh + 128 * 4;      // [128] int: segments whose epilogue read head h's (max, sum)
+constexpr uint32_t kOffBars = kOffEpi + 128 * 4;
 
 // barrier indices
 constexpr int kBarKvFull = 0;                    // [kStages] TMA landed
@@ -80,19 +80,20 @@ constexpr int kBarKvEmpty = kStages;             // [kStages] PV of the tile don
 constexpr int kBarSFull = 2 * kStages;           // [2] partial S of tile g in TMEM (g % 2)
 constexpr int kBarSEmpty = kBarSFull + 2;        // [2] the softmax copied S(g) out
 constexpr int kBarPFull = kBarSFull + 4;         // [2] P(g) in TMEM, O rescaled, V tail zeroed
-constexpr int kBarPvDone = kBarSFull + 6;        // [2] PV(g) finished
+constexpr int kBarPvDone = kBarSFull + 6;        // [4] PV(g) finished (g % 4: see the softmax's waits)
 constexpr int kBarQReady = kBarSFull + 11;       // query columns of the next segment in TMEM
 constexpr int kBarQFree = kBarSFull + 12;        // the last QK of a segment finished
 constexpr int kBarOFull = kBarSFull + 13;        // the last PV of a segment finished
 constexpr int kBarOFree = kBarSFull + 14;        // the epilogue has read O
-constexpr int kBarMlFull = kBarSFull + 15;       // (max, sum) of a finished segment in smem
+constexpr int kBarMlFull = kBarSFull + 15;       // (max, sum) of a finished even segment in smem
 constexpr int kBarFinal = kBarSFull + 16;        // all MMAs of this CTA done (teardown)
 constexpr int kBarFinal2 = kBarSFull + 17;       // all PV MMAs done (teardown)
 constexpr int kBarXFull = kBarSFull + 18;        // [2 warpgroups][2 buffers][4 warps] peer's block landed
 constexpr int kBarQReady0 = kBarXFull + 16;      // the first segment's query columns in TMEM
 constexpr int kBarQLanded = kBarQReady0 + 1;     // ... and in shared memory (stages 1-2)
 constexpr int kBarMHand = kBarQLanded + 1;       // [4 head quarters] running max of tile g-1 published
-constexpr int kNumBars = kBarMHand + 4;
+constexpr int kBarMlFull1 = kBarMHand + 4;      // ... of a finished odd segment
+constexpr int kNumBars = kBarMlFull1 + 1;
 // The first segment's query columns arrive by TMA in stages 1-2 (exactly 72 KB: four 64-column
 // boxes of 128 heads with 128-byte swizzle, then one 32-column k^R box with 64-byte swizzle);
 // the producer fills those stages with cache tiles only after the query has moved to TMEM.
@@ -102,15 +103,18 @@ static_assert(kQBytes == 2 * kStageBytes, "query staging fills stages 1-2 exactl
 constexpr uint32_t kOffMisc = kOffBars + 8 * kNumBars;
 constexpr uint32_t kSmemUsed = kOffMisc + 128;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;     // room to align the base to 1 KB
+static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
 
-constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 320, kTmemQ = 352, kTmemCols = 512;
-static_assert(kTmemS + kT <= kTmemP && kTmemP + kT / 2 <= kTmemQ && kTmemQ + 144 <= kTmemCols, "TMEM map");
+// Tensor memory: O, S, one P per softmax warpgroup (tile parity), the c^KV query columns.
+constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 320, kTmemQ = 384, kTmemCols = 512;
+static_assert(kTmemS + kT <= kTmemP && kTmemP + 2 * (kT / 2) <= kTmemQ && kTmemQ + 128 <= kTmemCols, "TMEM map");
+static_assert(kOffQr % 1024 == 0, "swizzled operand alignment");
 constexpr int kThreads = 512;   // 16 warps = 4 warpgroups (roles below)
 // Register split between the warpgroups (setmaxnreg), against 512 x 128 at launch:
-// 128 x (64 + 160 + 160 + 96) = 61,440 <= 65,536.
-constexpr int kRegsLaunch = 128, kRegsCtrl = 64, kRegsSoftmax = 160, kRegsTrans = 96;
+// 128 x (88 + 160 + 160 + 96) = 64,512 <= 65,536.
+constexpr int kRegsLaunch = 128, kRegsCtrl = 88, kRegsSoftmax = 160, kRegsTrans = 96;
 static_assert(128 * (kRegsCtrl + 2 * kRegsSoftmax + kRegsTrans) <= kThreads * kRegsLaunch, "register split");
-static_assert(kBarPvDone + 2 <= kBarSFull + 10, "barrier map");
+static_assert(kBarPvDone + 4 <= kBarSFull + 11, "barrier map");
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kT, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, false, true);
 constexpr float kRescaleThreshold = 8.f;   // log2 units: rescale O only when the max grows more
@@ -193,10 +197,33 @@ __device__ __forceinline__ bool wait_teardown(uint32_t bar, uint32_t parity, lon
   return true;
 }
 
+// Query row h as an MMA operand: 16-byte chunks 0..31 (the CTA's 256 c^KV columns) go to
+// TMEM columns kTmemQ + 4 chunk of the calling warp's lanes, chunks 32..35 (its 32 k^R
+// columns) to row h of the shared-memory A operand of the k^R MMAs (64-byte swizzle).
+__device__ __forceinline__ void q_chunks_out(const uint4 (&v)[12], uint8_t* smem, uint32_t tmem,
+                                             uint32_t lanes, int h, int part) {
+#pragma unroll
+  for (int grp = 0; grp < 3; ++grp) {
+    if (part == 2 && grp == 2) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<uint4*>(smem + kOffQr + h * 64 + ((i ^ ((h >> 1) & 3)) << 4)) = v[8 + i];
+    } else {
+      uint32_t r[16];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        r[4 * i] = v[4 * grp + i].x; r[4 * i + 1] = v[4 * grp + i].y;
+        r[4 * i + 2] = v[4 * grp + i].z; r[4 * i + 3] = v[4 * grp + i].w;
+      }
+      tmem_st16(lanes | (tmem + kTmemQ + 16 * (3 * part + grp)), r);
+    }
+  }
+}
+
 // One third (12 of the 36 16-byte chunks) of this CTA's 288 query columns of head h of
-// sequence b, into TMEM columns [kTmemQ + 48 part, +48) of the calling warp's lanes.
-__device__ __forceinline__ void load_q_part(const Params& p, uint32_t tmem, uint32_t lanes, int h,
-                                            int b, int part, uint32_t rank) {
+// sequence b, to TMEM / shared memory as above.
+__device__ __forceinline__ void load_q_part(const Params& p, uint8_t* smem, uint32_t tmem, uint32_t lanes,
+                                            int h, int b, int part, uint32_t rank) {
   const bool head_ok = h < p.n_heads;
   const __nv_bfloat16* qrow = p.q_abs + ((int64_t)b * p.n_heads + (head_ok ? h : 0)) * kRow;
   uint4 v[12];
@@ -206,21 +233,12 @@ __device__ __forceinline__ void load_q_part(const Params& p, uint32_t tmem, uint
     const int col = ci < 32 ? 256 * (int)rank + 8 * ci : kDLatent + 32 * (int)rank + 8 * (ci - 32);
     v[i] = head_ok ? *reinterpret_cast<const uint4*>(qrow + col) : make_uint4(0, 0, 0, 0);
   }
-#pragma unroll
-  for (int grp = 0; grp < 3; ++grp) {
-    uint32_t r[16];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      r[4 * i] = v[4 * grp + i].x; r[4 * i + 1] = v[4 * grp + i].y;
-      r[4 * i + 2] = v[4 * grp + i].z; r[4 * i + 3] = v[4 * grp + i].w;
-    }
-    tmem_st16(lanes | (tmem + kTmemQ + 16 * (3 * part + grp)), r);
-  }
+  q_chunks_out(v, smem, tmem, lanes, h, part);
 }
 
 // The same third of the first segment's query columns, from the TMA copy in stages 1-2
 // (row h of each box, 16-byte chunks under the boxes' 128- and 64-byte swizzles).
-__device__ __forceinline__ void q_part_from_smem(const uint8_t* smem, uint32_t tmem, uint32_t lanes,
+__device__ __forceinline__ void q_part_from_smem(uint8_t* smem, uint32_t tmem, uint32_t lanes,
                                                  int h, bool head_ok, int part) {
   const uint8_t* q = smem + kStageBytes;
   uint4 v[12];
@@ -232,16 +250,7 @@ __device__ __forceinline__ void q_part_from_smem(const uint8_t* smem, uint32_t t
         : 4 * kQBoxC + (uint32_t)h * 64 + (uint32_t)((((ci - 32) & 3) ^ ((h >> 1) & 3)) << 4);
     v[i] = head_ok ? *reinterpret_cast<const uint4*>(q + off) : make_uint4(0, 0, 0, 0);
   }
-#pragma unroll
-  for (int grp = 0; grp < 3; ++grp) {
-    uint32_t r[16];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      r[4 * i] = v[4 * grp + i].x; r[4 * i + 1] = v[4 * grp + i].y;
-      r[4 * i + 2] = v[4 * grp + i].z; r[4 * i + 3] = v[4 * grp + i].w;
-    }
-    tmem_st16(lanes | (tmem + kTmemQ + 16 * (3 * part + grp)), r);
-  }
+  q_chunks_out(v, smem, tmem, lanes, h, part);
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -258,6 +267,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
   volatile int* tile_valid = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);  // [kStages]
   float2* ml = reinterpret_cast<float2*>(smem + kOffMl);                             // [2][2][128]
   volatile float* mh = reinterpret_cast<volatile float*>(smem + kOffMh);             // [128]
+  volatile int* epi_seg = reinterpret_cast<volatile int*>(smem + kOffEpi);           // [128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -274,6 +284,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       mbar_init(bar(kBarSEmpty + i), 128);
       mbar_init(bar(kBarPFull + i), 128);
       mbar_init(bar(kBarPvDone + i), 1);
+      mbar_init(bar(kBarPvDone + 2 + i), 1);
     }
     mbar_init(bar(kBarFinal2), 1);
     for (int i = 0; i < 16; ++i) mbar_init(bar(kBarXFull + i), 1);
@@ -285,6 +296,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     mbar_init(bar(kBarOFull), 1);
     mbar_init(bar(kBarOFree), 128);
     mbar_init(bar(kBarMlFull), 256);
+    mbar_init(bar(kBarMlFull1), 256);
+    for (int i = 0; i < 128; ++i) epi_seg[i] = 0;
     mbar_init(bar(kBarFinal), 1);
     *abort_flag = 0;
     // every softmax warp's block of both buffers expects its first tile of partial scores
@@ -381,12 +394,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
         const uint32_t a = sbase + st * kStageBytes;
         const uint64_t dc = smem_desc(a, 16, 1024, 2);             // the four c^KV boxes
         const uint64_t dr = smem_desc(a + 4 * kBoxC, 16, 512, 4);  // the k^R box
+        const uint64_t dq = smem_desc(sbase + kOffQr, 16, 512, 4);  // the k^R query columns
 #pragma unroll
-        for (int ks = 0; ks < kKSteps; ++ks) {
-          const uint64_t bd = ks < 16 ? dc + (uint64_t)(((ks >> 2) * kBoxC + (ks & 3) * 32) >> 4)
-                                      : dr + (uint64_t)(((ks - 16) * 32) >> 4);
-          mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * ks, bd, kIdescQK, ks > 0 ? 1u : 0u);
-        }
+        for (int ks = 0; ks < 16; ++ks)
+          mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * ks, dc + (uint64_t)(((ks >> 2) * kBoxC + (ks & 3) * 32) >> 4),
+                 kIdescQK, ks > 0 ? 1u : 0u);
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+          mma_ss(tmem + kTmemS, dq + (uint64_t)((ks * 32) >> 4), dr + (uint64_t)((ks * 32) >> 4), kIdescQK, 1u);
         mma_commit(bar(kBarSFull + (g & 1u)));
         if (c.last()) mma_commit(bar(kBarQFree));
       }
@@ -408,12 +423,13 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
         if (c.first() && c.seg > 0 && !wait_bounded(bar(kBarOFree), (c.seg - 1) & 1u, guard)) break;
         tc_fence_after();
         const uint64_t dv = smem_desc(sbase + st * kStageBytes, kBoxC, 1024, 2);
+        const uint32_t pcol = kTmemP + (kT / 2) * (g & 1u);
 #pragma unroll
         for (int kk = 0; kk < kT / 16; ++kk)
-          mma_ts(tmem + kTmemO, tmem + kTmemP + 8 * kk, dv + (uint64_t)((kk * 2048) >> 4), kIdescPV,
+          mma_ts(tmem + kTmemO, tmem + pcol + 8 * kk, dv + (uint64_t)((kk * 2048) >> 4), kIdescPV,
                  (!c.first() || kk > 0) ? 1u : 0u);
         mma_commit(bar(kBarKvEmpty + st));
-        mma_commit(bar(kBarPvDone + (g & 1u)));
+        mma_commit(bar(kBarPvDone + (g & 3u)));
         if (c.last()) mma_commit(bar(kBarOFull));
       }
       mma_commit(bar(kBarFinal2));
@@ -614,8 +630,13 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
         l_own += ((sm[0].x + sm[0].y) + (sm[1].x + sm[1].y)) + ((sm[2].x + sm[2].y) + (sm[3].x + sm[3].y));
         const bool warp_need = __any_sync(0xffffffffu, need);
 
-        // PV(g-1) is done: O may be rescaled and P (read by PV(g-1)) overwritten
-        if (g > 0 && !wait_spin(bar(kBarPvDone + ((g - 1) & 1u)), ((g - 1) >> 1) & 1u, guard)) break;
+        // P(g) goes where P(g-2) was: PV(g-2) must be done (it nearly always is by now). O may be
+        // rescaled only once PV(g-1) is done as well; without a rescale, PV(g-1) may still run.
+        // PV(g) signals barrier g % 4: PV(g-4) is done (tile g's stage was refilled after it) and
+        // PV(g+3) cannot be (it needs P(g)), so each of these waits is at most one phase behind
+        // its barrier, which a phase parity can tell apart.
+        if (g > 1 && !wait_spin(bar(kBarPvDone + ((g - 2) & 3u)), ((g - 2) >> 2) & 1u, guard)) break;
+        if (warp_need && g > 0 && !wait_spin(bar(kBarPvDone + ((g - 1) & 3u)), ((g - 1) >> 2) & 1u, guard)) break;
         tc_fence_after();
         if (warp_need) {   // O (all 256 columns of this head) to the new max
 #pragma unroll 1
@@ -636,7 +657,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
             __nv_bfloat162 b2 = __floats2bfloat162_rn(sv[32 * hf + 2 * j], sv[32 * hf + 2 * j + 1]);
             pk[j] = *reinterpret_cast<uint32_t*>(&b2);
           }
-          tmem_st16(lanes | (tmem + kTmemP + 16 * hf), pk);
+          tmem_st16(lanes | (tmem + kTmemP + (kT / 2) * wg + 16 * hf), pk);
         }
         tmem_wait_st();
         if (r < kT) {
@@ -653,8 +674,23 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       }
       if (c.last()) {   // segment done: this warpgroup's (max, share) for the epilogue
         const bool mine = my_seg == c.seg;
+        // ml[seg % 2] was last read by the epilogue of segment seg - 2: wait for that read (a
+        // per-head counter, since the softmax may be more than one segment ahead of it)
+        if (c.seg >= 2) {
+          const long long t0 = clock64();
+          while (epi_seg[h] < (int)c.seg - 1) {
+            if (*abort_flag) { ok = false; break; }
+            if (clock64() - t0 > p.wait_limit) {
+              atomicOr(p.err, kErrTimeout);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+          }
+          if (!ok) break;
+        }
         ml[((c.seg & 1u) * 2 + wg) * 128 + h] = make_float2(mine ? m_own : -INFINITY, mine ? l_own : 0.f);
-        mbar_arrive(bar(kBarMlFull));
+        mbar_arrive(bar((c.seg & 1u) ? kBarMlFull1 : kBarMlFull));
       }
     }
     // after an abort: blocks the peer may still have in flight to us (it sends local tile u
@@ -677,10 +713,12 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     int prev_slot = -1;
     auto epilogue = [&](uint32_t seg, int slot) -> bool {
       if (!wait_bounded(bar(kBarOFull), seg & 1u, guard)) return false;
-      if (!wait_bounded(bar(kBarMlFull), seg & 1u, guard)) return false;
+      if (!wait_bounded(bar((seg & 1u) ? kBarMlFull1 : kBarMlFull), (seg >> 1) & 1u, guard)) return false;
       tc_fence_after();
       const float2 m0 = ml[((seg & 1u) * 2 + 0) * 128 + h];
       const float2 m1 = ml[((seg & 1u) * 2 + 1) * 128 + h];
+      __threadfence_block();
+      epi_seg[h] = (int)seg + 1;   // both warpgroups may now overwrite ml[seg % 2] for this head
       // O is relative to the last max used (the larger: the max only grows); each warpgroup's
       // share of the normaliser is relative to the max it used last
       const float mlast = fmaxf(m0.x, m1.x);
@@ -725,13 +763,15 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
           if (wait_bounded(bar(kBarQLanded), 0, guard)) {
             q_part_from_smem(smem, tmem, lanes, h, head_ok, 2);
             tmem_wait_st();
+            fence_proxy_async_smem();
           }
           tc_fence_before();
           mbar_arrive(bar(kBarQReady0));
         } else {
 #pragma unroll 1
-          for (int part = 0; part < 3; ++part) load_q_part(p, tmem, lanes, h, c.b, part, rank);
+          for (int part = 0; part < 3; ++part) load_q_part(p, smem, tmem, lanes, h, c.b, part, rank);
           tmem_wait_st();
+          fence_proxy_async_smem();   // the k^R query columns are read by the MMA (async proxy)
           tc_fence_before();
           mbar_arrive(bar(kBarQReady));
         }

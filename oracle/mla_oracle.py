@@ -43,6 +43,16 @@ Readings where the pages are silent (each is also listed in the design doc):
   * k^R in the cache is already rotated (it is rotated when it is written, [V3-walk]
     §2.2); the decode step reads it as it is.
   * kv_len == 0: the output is 0 and the log-sum-exp is -inf.
+  * YaRN ([V2-arch] pre-training: the context is extended from 4K to 128K with YaRN, applied
+    only to the decoupled RoPE part; s = 40, alpha = 1, beta = 32, target length 160K, and the
+    length scaling factor sqrt(t) = 0.0707 ln s + 1; [V2-notes] Long-Context Extension repeats
+    s, alpha, beta and the 160K target). The pages give only these hyper-parameters; the
+    frequencies follow the YaRN method ("NTK-by-parts", Peng et al. 2023): with the original
+    context L_0 (the 4K pre-training length) and a pair's wavelength 2 pi / theta_m, the ratio
+    r_m = L_0 theta_m / (2 pi) sets a weight g = clip((r_m - alpha) / (beta - alpha), 0, 1) and
+    theta'_m = (1 - g) theta_m / s + g theta_m: long wavelengths are interpolated by s, short
+    ones kept. The scores are multiplied by t = (0.0707 ln s + 1)^2, which the default softmax
+    scale takes in.
   * The cache row of a new token (the step before decode): c^KV = W^DKV h ([V2-arch] eq. 9,
     [V2-walk] §2.2), followed by an RMSNorm ([V2-notes] Architecture: an RMSNorm is added
     after the compressed latent vectors) with a learned scale gamma and eps = 1e-6 by default
@@ -59,6 +69,8 @@ A cache given as uint16 is read as bf16 bit patterns and widened exactly to floa
 from __future__ import annotations
 
 import math
+from dataclasses import dataclass
+from typing import Optional
 
 import numpy as np
 
@@ -118,20 +130,51 @@ def token_rows(cache, b: int, kv_len: int, page_table=None, page_size: int = 0) 
 # RoPE on the decoupled query  ([V2-walk] §2.4, [V3-walk] §2.3; convention: module doc)
 # ---------------------------------------------------------------------------
 
-def rope_angles(pos: int, d_rope: int, base: float) -> np.ndarray:
-    """Angles pos * theta_m for the d_rope/2 pairs, theta_m = base^(-2m/d_rope)."""
+@dataclass(frozen=True)
+class Yarn:
+    """YaRN context extension of the decoupled RoPE (module doc): scale factor s, the
+    original context L_0, the ramp bounds alpha < beta, and the coefficient of ln s in
+    sqrt(t)."""
+    factor: float
+    original_len: int = 4096
+    alpha: float = 1.0
+    beta: float = 32.0
+    mscale_coef: float = 0.0707
+
+
+def rope_theta(d_rope: int, base: float, yarn: Optional[Yarn] = None) -> np.ndarray:
+    """The d_rope/2 pair frequencies: theta_m = base^(-2m/d_rope), or with YaRN the blend of
+    theta_m / s and theta_m weighted by the ramp of r_m = L_0 theta_m / (2 pi)."""
     m = np.arange(d_rope // 2, dtype=np.float64)
     theta = base ** (-2.0 * m / d_rope)
-    return float(pos) * theta
+    if yarn is None or yarn.factor <= 1.0:
+        return theta
+    wavelength = 2.0 * math.pi / theta
+    r = yarn.original_len / wavelength
+    g = np.clip((r - yarn.alpha) / (yarn.beta - yarn.alpha), 0.0, 1.0)
+    return (1.0 - g) * theta / yarn.factor + g * theta
 
 
-def rope_rotate(x, pos: int, base: float) -> np.ndarray:
+def yarn_score_factor(yarn: Optional[Yarn]) -> float:
+    """t with sqrt(t) = coef * ln s + 1 (1 without YaRN): the factor on the scores."""
+    if yarn is None or yarn.factor <= 1.0:
+        return 1.0
+    root = yarn.mscale_coef * math.log(yarn.factor) + 1.0
+    return root * root
+
+
+def rope_angles(pos: int, d_rope: int, base: float, yarn: Optional[Yarn] = None) -> np.ndarray:
+    """Angles pos * theta_m for the d_rope/2 pairs (rope_theta)."""
+    return float(pos) * rope_theta(d_rope, base, yarn)
+
+
+def rope_rotate(x, pos: int, base: float, yarn: Optional[Yarn] = None) -> np.ndarray:
     """Rotate each interleaved pair (x[2m], x[2m+1]) of the last axis by pos * theta_m.
     base == 0 leaves x unchanged (RoPE off)."""
     x = widen(x)
     if base == 0:
         return x.copy()
-    ang = rope_angles(pos, x.shape[-1], base)
+    ang = rope_angles(pos, x.shape[-1], base, yarn)
     c, s = np.cos(ang), np.sin(ang)
     even, odd = x[..., 0::2], x[..., 1::2]
     y = np.empty_like(x)
@@ -171,7 +214,7 @@ def rms_norm(x, gamma, eps: float = 1e-6) -> np.ndarray:
 
 
 def cache_rows(hidden, w_dkv, w_kr, gamma, kv_lens, rope_base: float,
-               eps: float = 1e-6) -> np.ndarray:
+               eps: float = 1e-6, yarn: Optional[Yarn] = None) -> np.ndarray:
     """The row each sequence appends for its new token, [c^KV ; k^R] (576 values):
         c^KV = RMSNorm(W^DKV h_b) * gamma,   k^R = RoPE_{kv_len[b]-1}(W^KR h_b).
     hidden [B, d]; w_dkv [d_c, d]; w_kr [d_R, d]; gamma [d_c]. Returns [B, d_c + d_R]."""
@@ -180,21 +223,22 @@ def cache_rows(hidden, w_dkv, w_kr, gamma, kv_lens, rope_base: float,
     rows = np.zeros((hidden.shape[0], w_dkv.shape[0] + w_kr.shape[0]))
     for b in range(hidden.shape[0]):
         c = rms_norm(w_dkv @ hidden[b], gamma, eps)
-        kr = rope_rotate(w_kr @ hidden[b], int(kv_lens[b]) - 1, rope_base)
+        kr = rope_rotate(w_kr @ hidden[b], int(kv_lens[b]) - 1, rope_base, yarn)
         rows[b] = np.concatenate([c, kr])
     return rows
 
 
-def default_scale(d_head: int = D_HEAD, d_rope: int = D_ROPE) -> float:
-    """1/sqrt(d_h + d_h^R): the reading of the softmax scale (see module doc)."""
-    return 1.0 / math.sqrt(d_head + d_rope)
+def default_scale(d_head: int = D_HEAD, d_rope: int = D_ROPE, yarn: Optional[Yarn] = None) -> float:
+    """1/sqrt(d_h + d_h^R) (the reading of the softmax scale, module doc), times the YaRN
+    score factor t when YaRN is on."""
+    return yarn_score_factor(yarn) / math.sqrt(d_head + d_rope)
 
 
 # ---------------------------------------------------------------------------
 # the absorbed path, one stage at a time
 # ---------------------------------------------------------------------------
 
-def absorb_query(q_c, q_r, w_uk, kv_lens, rope_base: float) -> np.ndarray:
+def absorb_query(q_c, q_r, w_uk, kv_lens, rope_base: float, yarn: Optional[Yarn] = None) -> np.ndarray:
     """Absorbed query rows [B, n_h, d_c + d_R] in float64.
 
     q'_{b,i} = W_UK,i^T q^C_{b,i}   ([V2-walk] §2.3 displayed equation; [V3-walk] §2.3)
@@ -211,7 +255,7 @@ def absorb_query(q_c, q_r, w_uk, kv_lens, rope_base: float) -> np.ndarray:
         pos = max(int(kv_lens[b]) - 1, 0)
         for i in range(H):
             out[b, i, :d_c] = w_uk[i].T @ q_c[b, i]
-            out[b, i, d_c:] = rope_rotate(q_r[b, i], pos, rope_base)
+            out[b, i, d_c:] = rope_rotate(q_r[b, i], pos, rope_base, yarn)
     return out
 
 
@@ -256,7 +300,7 @@ def apply_wuv(latent, w_uv) -> np.ndarray:
 
 def mla_decode_nonabsorbed(q_c, q_r, w_uk, w_uv, cache, kv_lens, scale: float,
                            rope_base: float, page_table=None, page_size: int = 0,
-                           pairs=None) -> np.ndarray:
+                           pairs=None, yarn: Optional[Yarn] = None) -> np.ndarray:
     """Head outputs o [B, n_h, d_h] by the non-absorbed definition (module doc).
 
     Per (b, i): k^C_j = W_UK,i c_j and v_j = W_UV,i c_j are materialised for every cached
@@ -287,7 +331,7 @@ def mla_decode_nonabsorbed(q_c, q_r, w_uk, w_uv, cache, kv_lens, scale: float,
         for i in heads:
             k_content = c @ w_uk[i].T                                   # [L, d_h]
             v = c @ w_uv[i].T                                           # [L, d_h]
-            q = np.concatenate([q_c[b, i], rope_rotate(q_r[b, i], L - 1, rope_base)])
+            q = np.concatenate([q_c[b, i], rope_rotate(q_r[b, i], L - 1, rope_base, yarn)])
             keys = np.concatenate([k_content, k_r], axis=1)             # [L, d_h + d_R]
             p, _ = softmax_lse((keys @ q) * scale, axis=0)
             out[b, i] = p @ v
@@ -295,11 +339,12 @@ def mla_decode_nonabsorbed(q_c, q_r, w_uk, w_uv, cache, kv_lens, scale: float,
 
 
 def mla_decode_absorbed(q_c, q_r, w_uk, w_uv, cache, kv_lens, scale: float,
-                        rope_base: float, page_table=None, page_size: int = 0):
+                        rope_base: float, page_table=None, page_size: int = 0,
+                        yarn: Optional[Yarn] = None):
     """The absorbed path in float64: absorb_query -> latent_attention -> apply_wuv.
     Returns (out [B, n_h, d_h], latent [B, n_h, d_c], lse [B, n_h])."""
     d_latent = np.asarray(w_uk).shape[2]
-    q_abs = absorb_query(q_c, q_r, w_uk, kv_lens, rope_base)
+    q_abs = absorb_query(q_c, q_r, w_uk, kv_lens, rope_base, yarn)
     latent, lse = latent_attention(q_abs, cache, kv_lens, scale, page_table, page_size,
                                    d_latent=d_latent)
     return apply_wuv(latent, w_uv), latent, lse

@@ -73,3 +73,30 @@ def cache_row(h, w_dkv, w_kr, gamma, kv_len, rope_base, eps=1e-6):
     rms = math.sqrt(math.fsum(v * v for v in x) / len(x) + eps)
     c = [v / rms * g for v, g in zip(x, gamma)]
     return c + _rotate(_matvec(w_kr, h), kv_len - 1, rope_base)
+
+
+def yarn_theta(d, base, s, orig_len, alpha, beta):
+    """YaRN pair frequencies, written pair by pair from the method's definition: a pair whose
+    wavelength fits into the original context fewer than alpha times is slowed by s, more
+    than beta times is kept, and in between the two are blended linearly in that count."""
+    out = []
+    for m in range(d // 2):
+        theta = base ** (-2.0 * m / d)
+        fits = orig_len / (2.0 * math.pi / theta)
+        if fits <= alpha:
+            w = 0.0
+        elif fits >= beta:
+            w = 1.0
+        else:
+            w = (fits - alpha) / (beta - alpha)
+        out.append(w * theta + (1.0 - w) * theta / s)
+    return out
+
+
+def rotate_with(x, pos, thetas):
+    """RoPE as a complex product with the given pair frequencies."""
+    y = [0.0] * len(x)
+    for m, th in enumerate(thetas):
+        z = complex(x[2 * m], x[2 * m + 1]) * cmath.exp(1j * pos * th)
+        y[2 * m], y[2 * m + 1] = z.real, z.imag
+    return y

@@ -292,11 +292,11 @@ def test_planted_mistakes_are_caught(monkeypatch):
     ref = np.array(ref)
     good_rotate, good_rows = om.rope_rotate, om.token_rows
 
-    def wrong_sign(x, pos, base):
-        return good_rotate(x, -pos, base)
+    def wrong_sign(x, pos, base, yarn=None):
+        return good_rotate(x, -pos, base, yarn)
 
-    def off_by_one(x, pos, base):
-        return good_rotate(x, pos + 1, base)
+    def off_by_one(x, pos, base, yarn=None):
+        return good_rotate(x, pos + 1, base, yarn)
 
     def wrong_slot(cache, b, kv_len, page_table=None, page_size=0):
         # slot index off by one inside each page (the order of the rows alone would not
@@ -386,3 +386,100 @@ def test_cache_row_planted_mistakes_are_caught():
     # RoPE one position late (at kv_len instead of kv_len - 1)
     late = np.stack([oracle.rope_rotate(w_kr @ h[b], int(lens[b]), 10000.0) for b in range(len(lens))])
     assert np.max(np.abs(late - good[:, 8:])) > 1e-3
+
+
+# --- YaRN (context extension of the decoupled RoPE) --------------------------------
+
+YARN_GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "yarn.txt")
+
+
+def _yarn_golden():
+    vals = {}
+    with open(YARN_GOLDEN) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                key, value = line.split()[:2]
+                vals[key] = float(value)
+    return vals
+
+
+def _pages_yarn():
+    g = _yarn_golden()
+    return oracle.Yarn(factor=g["scale_factor_s"], original_len=int(g["original_length_tokens"]),
+                       alpha=g["alpha"], beta=g["beta"], mscale_coef=g["sqrt_t_coefficient"])
+
+
+def test_yarn_figures_are_consistent():
+    """The pages' target length is the scale factor times the original 4K context."""
+    g = _yarn_golden()
+    assert g["scale_factor_s"] * g["original_length_tokens"] == g["target_length_tokens"]
+
+
+def test_yarn_off_or_factor_one_is_plain_rope():
+    plain = oracle.rope_theta(64, 10000.0)
+    np.testing.assert_array_equal(oracle.rope_theta(64, 10000.0, None), plain)
+    np.testing.assert_allclose(oracle.rope_theta(64, 10000.0, oracle.Yarn(factor=1.0)), plain, rtol=0)
+    assert oracle.yarn_score_factor(None) == 1.0
+    assert oracle.yarn_score_factor(oracle.Yarn(factor=1.0)) == 1.0
+
+
+def test_yarn_keeps_fast_pairs_and_slows_slow_pairs_by_s():
+    """With the pages' s = 40 over a 4K context: pair 0 (wavelength 2 pi, fits 652 times)
+    is kept, pair 31 (wavelength ~47,000 > 4K) is slowed by exactly s, and every pair lies
+    between theta/s and theta, non-increasing in m."""
+    y = _pages_yarn()
+    plain = oracle.rope_theta(64, 10000.0)
+    th = oracle.rope_theta(64, 10000.0, y)
+    assert th[0] == plain[0]
+    np.testing.assert_allclose(th[31], plain[31] / 40.0, rtol=1e-15)
+    assert np.all(th <= plain * (1 + 1e-15)) and np.all(th >= plain / 40.0 * (1 - 1e-15))
+    assert np.all(np.diff(th) <= 0)
+    # some pairs sit on the ramp (neither kept nor fully slowed)
+    mid = (th < plain * (1 - 1e-12)) & (th > plain / 40.0 * (1 + 1e-12))
+    assert mid.sum() >= 3
+
+
+def test_yarn_theta_matches_python_loops():
+    for y in (_pages_yarn(), oracle.Yarn(factor=8.0, original_len=2048, alpha=2.0, beta=16.0)):
+        got = oracle.rope_theta(64, 10000.0, y)
+        ref = _bruteforce.yarn_theta(64, 10000.0, y.factor, y.original_len, y.alpha, y.beta)
+        np.testing.assert_allclose(got, ref, rtol=1e-14)
+        rng = np.random.default_rng(50)
+        x = rng.standard_normal(64)
+        np.testing.assert_allclose(oracle.rope_rotate(x, 100000, 10000.0, y),
+                                   _bruteforce.rotate_with(list(x), 100000, ref), atol=1e-9)
+
+
+def test_yarn_score_factor_special_points():
+    """sqrt(t) = c ln s + 1: t = 1 at s = 1, and t = 4 where c ln s = 1."""
+    c = 0.0707
+    assert oracle.yarn_score_factor(oracle.Yarn(factor=1.0, mscale_coef=c)) == 1.0
+    s = math.exp(1.0 / c)
+    assert abs(oracle.yarn_score_factor(oracle.Yarn(factor=s, mscale_coef=c)) - 4.0) < 1e-12
+    assert oracle.default_scale(yarn=oracle.Yarn(factor=s, mscale_coef=c)) == pytest.approx(4.0 / math.sqrt(192))
+
+
+def test_yarn_rotation_keeps_relative_position_property():
+    """Rotations with any fixed frequencies: q at p and k at p' give the same dot product as
+    q at p + d and k at p' + d."""
+    y = _pages_yarn()
+    rng = np.random.default_rng(51)
+    q, k = rng.standard_normal(64), rng.standard_normal(64)
+    a = oracle.rope_rotate(q, 5000, 10000.0, y) @ oracle.rope_rotate(k, 1234, 10000.0, y)
+    b = oracle.rope_rotate(q, 105000, 10000.0, y) @ oracle.rope_rotate(k, 101234, 10000.0, y)
+    assert abs(a - b) < 1e-9
+
+
+def test_yarn_planted_mistakes_are_caught():
+    y = _pages_yarn()
+    plain = oracle.rope_theta(64, 10000.0)
+    good = oracle.rope_theta(64, 10000.0, y)
+    r = y.original_len * plain / (2 * math.pi)
+    g = np.clip((r - y.alpha) / (y.beta - y.alpha), 0, 1)
+    reversed_ramp = g * plain / y.factor + (1 - g) * plain
+    multiplied = (1 - g) * plain * y.factor + g * plain
+    for bad in (reversed_ramp, multiplied):
+        assert not np.allclose(bad, good)
+        # ... and the pin on the end pairs sees it
+        assert bad[0] != plain[0] or abs(bad[31] - plain[31] / 40.0) > 1e-18

@@ -62,6 +62,19 @@ typedef struct {
   float softmax_scale;   /* 0 => 1/sqrt(d_h + d_h^R) = 1/sqrt(192)                    */
   float rope_base;       /* RoPE base (10000 for DeepSeek-V2); 0 => q^R not rotated   */
   int32_t max_splits;    /* upper bound on KV splits per sequence; 0 => automatic     */
+  /* YaRN context extension of the decoupled RoPE ([V2-arch] pre-training paragraph;
+   * [V2-notes] Long-Context Extension: s = 40, alpha = 1, beta = 32 over a 4K original
+   * context, sqrt(t) = 0.0707 ln s + 1). With yarn_factor s > 1, pair m's frequency
+   * theta_m = base^(-2m/64) becomes (1 - g) theta_m / s + g theta_m, where
+   * g = clamp((r - alpha) / (beta - alpha), 0, 1) and r = original_len * theta_m / (2 pi)
+   * (the YaRN method's blend), for the rotated query (mla_absorb_q) and the written key
+   * (mla_append_kv); and softmax_scale 0 then means t / sqrt(192), t = (coef ln s + 1)^2.
+   * yarn_factor 0 or 1 leaves RoPE and the scale as above. */
+  float yarn_factor;        /* s: 0 or 1 => off, else >= 1                              */
+  int32_t yarn_original_len;/* original context length (>= 1 when on; 4096)             */
+  float yarn_alpha;         /* ramp start, in wavelengths per original context (1)      */
+  float yarn_beta;          /* ramp end, > yarn_alpha (32)                               */
+  float yarn_mscale_coef;   /* coefficient of ln s in sqrt(t), >= 0 (0.0707)            */
 } mla_config_t;
 
 /*

@@ -42,6 +42,11 @@ class MlaConfig(ctypes.Structure):
         ("softmax_scale", ctypes.c_float),
         ("rope_base", ctypes.c_float),
         ("max_splits", ctypes.c_int32),
+        ("yarn_factor", ctypes.c_float),
+        ("yarn_original_len", ctypes.c_int32),
+        ("yarn_alpha", ctypes.c_float),
+        ("yarn_beta", ctypes.c_float),
+        ("yarn_mscale_coef", ctypes.c_float),
     ]
 
 
@@ -102,9 +107,13 @@ def _check(status: int, what: str) -> None:
 
 def make_config(n_heads: int, max_batch: int, max_kv_len: int, page_size: int = 0,
                 softmax_scale: float = 0.0, rope_base: float = 10000.0,
-                max_splits: int = 0) -> MlaConfig:
+                max_splits: int = 0, yarn_factor: float = 0.0, yarn_original_len: int = 4096,
+                yarn_alpha: float = 1.0, yarn_beta: float = 32.0,
+                yarn_mscale_coef: float = 0.0707) -> MlaConfig:
+    """yarn_factor > 1 turns on YaRN (DeepSeek-V2 uses 40 with the other defaults)."""
     return MlaConfig(n_heads, 128, 512, 64, page_size, max_batch, max_kv_len,
-                     softmax_scale, rope_base, max_splits)
+                     softmax_scale, rope_base, max_splits, yarn_factor, yarn_original_len,
+                     yarn_alpha, yarn_beta, yarn_mscale_coef)
 
 
 def check_config(cfg: MlaConfig) -> int:
@@ -132,10 +141,12 @@ class MlaDecode:
 
     def __init__(self, n_heads: int, max_batch: int, max_kv_len: int, page_size: int = 0,
                  softmax_scale: float = 0.0, rope_base: float = 10000.0, max_splits: int = 0,
-                 device: Optional[int] = None):
+                 device: Optional[int] = None, **yarn):
+        """`yarn`: yarn_factor, yarn_original_len, yarn_alpha, yarn_beta, yarn_mscale_coef
+        (make_config)."""
         self._lib = load_library()
         self.cfg = make_config(n_heads, max_batch, max_kv_len, page_size, softmax_scale,
-                               rope_base, max_splits)
+                               rope_base, max_splits, **yarn)
         self.device = torch.cuda.current_device() if device is None else int(device)
         h = ctypes.c_void_p()
         _check(self._lib.mla_decode_create(ctypes.byref(self.cfg), self.device, ctypes.byref(h)),

@@ -317,7 +317,7 @@ cudaError_t launch_append_kv(const mla_decode_s& h, int batch, int d_model,
   fp.c_kv = c_kv;
   fp.k_r = k_r;
   for (int m = 0; m < kDRope / 2; ++m)
-    fp.theta[m] = h.cfg.rope_base > 0.f ? std::pow((double)h.cfg.rope_base, -2.0 * m / kDRope) : 0.0;
+    fp.theta[m] = h.theta[m];
   fp.err = h.ws.err;
   return launch_pdl(kv_finalize, dim3(batch), dim3(kRow), 0, s, fp);
 }

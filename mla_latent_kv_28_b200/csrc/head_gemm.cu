@@ -281,7 +281,7 @@ cudaError_t launch(const mla_decode_s& h, int batch, const __nv_bfloat16* w, con
   p.q_r = q_r;
   p.kv_lens = kv_lens;
   for (int m = 0; m < kDRope / 2; ++m)
-    p.theta[m] = h.cfg.rope_base > 0.f ? std::pow((double)h.cfg.rope_base, -2.0 * m / kDRope) : 0.0;
+    p.theta[m] = h.theta[m];
   p.err = h.ws.err;
   p.wait_limit = 2000000000LL;
   const uint32_t smem = kWeightBytes + kXBoxes * n_tile * 128 + 64 + 1024;

@@ -31,7 +31,30 @@ int config_status(const mla_config_t* c) {
   if (c->page_size != 0 && c->page_size != 64) return MLA_ERR_UNSUPPORTED;
   if (c->max_kv_len > (int64_t)1 << 30) return MLA_ERR_UNSUPPORTED;
   if (c->max_splits > 64) return MLA_ERR_UNSUPPORTED;
+  if (!(c->yarn_factor >= 0.f) || !std::isfinite(c->yarn_factor) ||
+      (c->yarn_factor > 0.f && c->yarn_factor < 1.f))
+    return MLA_ERR_INVALID_ARG;
+  if (c->yarn_factor > 1.f &&
+      (c->yarn_original_len < 1 || !std::isfinite(c->yarn_alpha) || !std::isfinite(c->yarn_beta) ||
+       !(c->yarn_beta > c->yarn_alpha) || !(c->yarn_mscale_coef >= 0.f) ||
+       !std::isfinite(c->yarn_mscale_coef)))
+    return MLA_ERR_INVALID_ARG;
   return MLA_OK;
+}
+
+// Pair frequencies of the decoupled RoPE: base^(-2m/64), and with YaRN (factor s > 1) the
+// blend of theta/s (pairs whose wavelength fits into the original context at most alpha
+// times) and theta (at least beta times), linear in that count between the two.
+void rope_frequencies(const mla_config_t& c, double* theta) {
+  for (int m = 0; m < kDRope / 2; ++m) {
+    if (!(c.rope_base > 0.f)) { theta[m] = 0.0; continue; }
+    const double th = std::pow((double)c.rope_base, -2.0 * m / kDRope);
+    if (!(c.yarn_factor > 1.f)) { theta[m] = th; continue; }
+    const double fits = (double)c.yarn_original_len * th / (2.0 * 3.141592653589793);
+    double w = (fits - (double)c.yarn_alpha) / ((double)c.yarn_beta - (double)c.yarn_alpha);
+    w = std::min(1.0, std::max(0.0, w));
+    theta[m] = w * th + (1.0 - w) * th / (double)c.yarn_factor;
+  }
 }
 
 }  // namespace
@@ -69,8 +92,14 @@ int mla_decode_create(const mla_config_t* cfg, int device, mla_handle_t* out) {
   h->cfg = *cfg;
   h->device = device;
   h->num_sms = sms;
+  double t = 1.0;   // YaRN's factor on the scores
+  if (cfg->yarn_factor > 1.f) {
+    const double root = (double)cfg->yarn_mscale_coef * std::log((double)cfg->yarn_factor) + 1.0;
+    t = root * root;
+  }
   h->scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale
-                                      : (float)(1.0 / std::sqrt((double)(kDHead + kDRope)));
+                                      : (float)(t / std::sqrt((double)(kDHead + kDRope)));
+  rope_frequencies(*cfg, h->theta);
   h->units = sms / 2;  // the decode kernel runs one 2-CTA cluster per unit of work
 
   const int B = cfg->max_batch;

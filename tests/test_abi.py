@@ -62,7 +62,16 @@ def test_config_checks(lib):
         (binding.make_config(129, 1, 1), binding.MLA_ERR_UNSUPPORTED),
         (binding.make_config(8, 1, 1, page_size=16), binding.MLA_ERR_UNSUPPORTED),
         (binding.make_config(8, 4096, 1), binding.MLA_ERR_UNSUPPORTED),
+        # YaRN: a factor in (0, 1), a ramp that does not rise, a negative coefficient, no
+        # original length
+        (binding.make_config(8, 1, 1, yarn_factor=0.5), binding.MLA_ERR_INVALID_ARG),
+        (binding.make_config(8, 1, 1, yarn_factor=40.0, yarn_alpha=32.0, yarn_beta=32.0),
+         binding.MLA_ERR_INVALID_ARG),
+        (binding.make_config(8, 1, 1, yarn_factor=40.0, yarn_mscale_coef=-0.1), binding.MLA_ERR_INVALID_ARG),
+        (binding.make_config(8, 1, 1, yarn_factor=40.0, yarn_original_len=0), binding.MLA_ERR_INVALID_ARG),
     ]
+    assert binding.check_config(binding.make_config(128, 64, 131072, yarn_factor=40.0)) == binding.MLA_OK
+    assert binding.check_config(binding.make_config(8, 1, 1, yarn_factor=1.0)) == binding.MLA_OK
     for cfg, want in bad:
         assert binding.check_config(cfg) == want
     wrong_dims = binding.make_config(8, 1, 1)

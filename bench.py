@@ -429,10 +429,13 @@ def run_ours(args):
     del step_graph, attn_graph
 
     # End to end through the public API: every step uploads its inputs from pinned host
-    # memory and downloads its head outputs to pinned host memory. The copies run on their
-    # own stream, double-buffered, so step k+1's upload and step k's download overlap step
-    # k's kernels, as a serving loop would run them; every step's copies are inside the timed
-    # region (it ends when the last download has landed).
+    # memory and downloads its head outputs to pinned host memory. A serving loop would run
+    # the step as a CUDA graph with the copies on their own branch: graph k computes step k
+    # from the inputs uploaded by graph k-1, while uploading step k+1's inputs and downloading
+    # step k-1's outputs, so the copies overlap the kernels and one graph launch is all the
+    # host does per step. The graphs are captured from the public calls (MlaDecode.step and
+    # tensor copies); the timed region covers the first upload, K graphs, and the last
+    # download.
     hq_c = g.q_c.cpu().pin_memory()
     hq_r = g.q_r.cpu().pin_memory()
     hlens = g.kv_lens.cpu().pin_memory()
@@ -443,49 +446,58 @@ def run_ours(args):
     h2d = hq_c.numel() * 2 + hq_r.numel() * 2 + hlens.numel() * 4
     d2h = hout[0].numel() * 2
     copy = torch.cuda.Stream(dev)
-    uploaded = [torch.cuda.Event() for _ in range(2)]
-    computed = [torch.cuda.Event() for _ in range(2)]
-    downloaded = [torch.cuda.Event() for _ in range(2)]
 
     def upload(slot):
+        for d, hsrc in zip(din[slot], (hq_c, hq_r, hlens)):
+            d.copy_(hsrc, non_blocking=True)
+
+    def e2e_step(k):
+        slot = k % 2
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        copy.wait_event(fork)
         with torch.cuda.stream(copy):
-            copy.wait_event(computed[slot])       # the step that last read this slot is done
-            for d, hsrc in zip(din[slot], (hq_c, hq_r, hlens)):
-                d.copy_(hsrc, non_blocking=True)
-            uploaded[slot].record(copy)
+            upload(1 - slot)                                        # inputs of step k+1
+            hout[1 - slot].copy_(dout[1 - slot], non_blocking=True)  # outputs of step k-1
+            join = torch.cuda.Event()
+            join.record(copy)
+        dq_c, dq_r, dlens = din[slot]
+        h.step(dq_c, dq_r, g.w_uk, g.w_uv, caches[k % copies], dlens, g.page_table, stream,
+               dict(bufs, out=dout[slot]))
+        stream.wait_event(join)
 
-    def e2e_run(n, e_start=None, e_end=None):
-        if e_start is not None:
-            e_start.record(copy)
+    n_graphs = 2 * copies // math.gcd(2, copies)   # input slot and cache copy both cycle
+    with torch.cuda.stream(stream):
         upload(0)
-        for k in range(n):
-            slot = k % 2
-            stream.wait_event(uploaded[slot])
-            stream.wait_event(downloaded[slot])   # step k-2's output has left dout[slot]
-            dq_c, dq_r, dlens = din[slot]
-            out = h.step(dq_c, dq_r, g.w_uk, g.w_uv, caches[k % copies], dlens, g.page_table,
-                         stream, dict(bufs, out=dout[slot]))
-            computed[slot].record(stream)
-            if k + 1 < n:
-                upload(1 - slot)
-            with torch.cuda.stream(copy):
-                copy.wait_event(computed[slot])
-                hout[slot].copy_(out, non_blocking=True)
-                downloaded[slot].record(copy)
-        if e_end is not None:
-            e_end.record(copy)
-
-    for ev in computed + downloaded:
-        ev.record(stream)
-    e2e_run(args.warmup)
+        for k in range(max(args.warmup, n_graphs)):
+            e2e_step(k)
     torch.cuda.synchronize(dev)
+    e2e_graphs = []
+    for k in range(n_graphs):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            e2e_step(k)
+        e2e_graphs.append(gr)
+    with torch.cuda.stream(stream):
+        upload(0)
+        for k in range(n_graphs):
+            e2e_graphs[k].replay()
+    torch.cuda.synchronize(dev)
+    h.check_device_errors(stream)
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world, local, True)
     torch.cuda.synchronize(dev)
-    e2e_run(args.steps, e_start, e_end)
+    with torch.cuda.stream(stream):
+        e_start.record(stream)
+        upload(0)
+        for k in range(args.steps):
+            e2e_graphs[k % n_graphs].replay()
+        hout[(args.steps - 1) % 2].copy_(dout[(args.steps - 1) % 2], non_blocking=True)
+        e_end.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world, local, True)
     h.check_device_errors(stream)
+    del e2e_graphs
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / args.steps, world, dev)
     clocks.stop()
 

@@ -43,6 +43,10 @@ Readings where the pages are silent (each is also listed in the design doc):
   * k^R in the cache is already rotated (it is rotated when it is written, [V3-walk]
     §2.2); the decode step reads it as it is.
   * kv_len == 0: the output is 0 and the log-sum-exp is -inf.
+  * Several new tokens per sequence (multi-token prediction, speculative decoding; the
+    pages' MTP modules, [V3-walk] section 4.1, predict extra tokens that the main model then
+    verifies): the T new tokens are the last T of the kv_len cached rows, and token t sees
+    rows 0 .. kv_len - T + t (see "several new tokens per sequence" below).
   * YaRN ([V2-arch] pre-training: the context is extended from 4K to 128K with YaRN, applied
     only to the decoupled RoPE part; s = 40, alpha = 1, beta = 32, target length 160K, and the
     length scaling factor sqrt(t) = 0.0707 ln s + 1; [V2-notes] Long-Context Extension repeats
@@ -335,6 +339,88 @@ def mla_decode_nonabsorbed(q_c, q_r, w_uk, w_uv, cache, kv_lens, scale: float,
             keys = np.concatenate([k_content, k_r], axis=1)             # [L, d_h + d_R]
             p, _ = softmax_lse((keys @ q) * scale, axis=0)
             out[b, i] = p @ v
+    return out
+
+
+# ---------------------------------------------------------------------------
+# several new tokens per sequence (multi-token prediction / speculative decoding)
+# ---------------------------------------------------------------------------
+# A sequence whose kv_len = L cached rows include T new tokens holds them at positions
+# L - T + t, t = 0..T-1. Token t attends to the rows at positions 0 .. L - T + t: itself and
+# what came before it, not the new tokens after it (the causal mask of [V2-arch]'s MHA
+# equation, Softmax_j over j = 1..t, applied to each new token). A token with no visible row
+# (L < T) gets a zero output and a log-sum-exp of -inf; its q^R is rotated at position 0.
+
+def token_visible_rows(kv_len: int, q_len: int, t: int) -> int:
+    """Rows that new token t (0-based, of q_len) of a sequence with kv_len rows sees."""
+    return max(0, int(kv_len) - int(q_len) + t + 1)
+
+
+def absorb_query_tokens(q_c, q_r, w_uk, kv_lens, rope_base: float,
+                        yarn: Optional[Yarn] = None) -> np.ndarray:
+    """q_c [B, T, n_h, d_h], q_r [B, T, n_h, d_R] -> absorbed rows [B, T, n_h, d_c + d_R]:
+    W_UK,i^T q^C and q^R rotated at token t's position max(L - T + t, 0)."""
+    q_c, q_r, w_uk = widen(q_c), widen(q_r), widen(w_uk)
+    kv_lens = np.asarray(kv_lens)
+    B, T, H, _ = q_c.shape
+    d_c, d_r = w_uk.shape[2], q_r.shape[3]
+    out = np.zeros((B, T, H, d_c + d_r))
+    for b in range(B):
+        for t in range(T):
+            pos = max(int(kv_lens[b]) - T + t, 0)
+            for i in range(H):
+                out[b, t, i, :d_c] = w_uk[i].T @ q_c[b, t, i]
+                out[b, t, i, d_c:] = rope_rotate(q_r[b, t, i], pos, rope_base, yarn)
+    return out
+
+
+def latent_attention_tokens(q_abs, cache, kv_lens, scale: float, page_table=None,
+                            page_size: int = 0, d_latent: int = D_LATENT):
+    """q_abs [B, T, n_h, 576] -> (latent [B, T, n_h, d_c], lse [B, T, n_h]); token t of
+    sequence b attends to its first token_visible_rows(L, T, t) rows."""
+    q_abs = widen(q_abs)
+    kv_lens = np.asarray(kv_lens)
+    B, T, H, _ = q_abs.shape
+    latent = np.zeros((B, T, H, d_latent))
+    lse = np.full((B, T, H), -np.inf)
+    for b in range(B):
+        L = int(kv_lens[b])
+        rows = token_rows(cache, b, L, page_table, page_size) if L > 0 else None
+        for t in range(T):
+            n = token_visible_rows(L, T, t)
+            if n == 0:
+                continue
+            s = (rows[:n] @ q_abs[b, t].T) * scale                   # [n, H]
+            p, lse[b, t] = softmax_lse(s, axis=0)
+            latent[b, t] = p.T @ rows[:n, :d_latent]
+    return latent, lse
+
+
+def mla_decode_nonabsorbed_tokens(q_c, q_r, w_uk, w_uv, cache, kv_lens, scale: float,
+                                  rope_base: float, page_table=None, page_size: int = 0,
+                                  yarn: Optional[Yarn] = None) -> np.ndarray:
+    """Head outputs o [B, T, n_h, d_h] by the non-absorbed definition (materialised keys and
+    values per head), each new token over its visible rows."""
+    q_c, q_r = widen(q_c), widen(q_r)
+    w_uk, w_uv = widen(w_uk), widen(w_uv)
+    kv_lens = np.asarray(kv_lens)
+    B, T, H, d_h = q_c.shape
+    d_c = w_uk.shape[2]
+    out = np.zeros((B, T, H, d_h))
+    for b in range(B):
+        L = int(kv_lens[b])
+        rows = token_rows(cache, b, L, page_table, page_size) if L > 0 else None
+        for t in range(T):
+            n = token_visible_rows(L, T, t)
+            if n == 0:
+                continue
+            c, k_r = rows[:n, :d_c], rows[:n, d_c:]
+            pos = L - T + t
+            for i in range(H):
+                keys = np.concatenate([c @ w_uk[i].T, k_r], axis=1)
+                q = np.concatenate([q_c[b, t, i], rope_rotate(q_r[b, t, i], pos, rope_base, yarn)])
+                p, _ = softmax_lse((keys @ q) * scale, axis=0)
+                out[b, t, i] = p @ (c @ w_uv[i].T)
     return out
 
 

@@ -483,3 +483,74 @@ def test_yarn_planted_mistakes_are_caught():
         assert not np.allclose(bad, good)
         # ... and the pin on the end pairs sees it
         assert bad[0] != plain[0] or abs(bad[31] - plain[31] / 40.0) > 1e-18
+
+
+# --- several new tokens per sequence (multi-token / speculative decoding) ----------
+
+def _tiny_tokens(seed=60, B=2, T=3, H=2, d_h=4, d_c=8, d_r=4, L=(7, 2)):
+    rng = np.random.default_rng(seed)
+    Lmax = max(L)
+    return dict(q_c=rng.standard_normal((B, T, H, d_h)), q_r=rng.standard_normal((B, T, H, d_r)),
+                w_uk=rng.standard_normal((H, d_h, d_c)), w_uv=rng.standard_normal((H, d_h, d_c)),
+                cache=rng.standard_normal((B, Lmax, d_c + d_r)), kv_lens=np.array(L))
+
+
+def test_tokens_with_one_token_equal_single_token_decode():
+    a = _tiny_tokens(T=1, L=(7, 3))
+    q1 = oracle.absorb_query(a["q_c"][:, 0], a["q_r"][:, 0], a["w_uk"], a["kv_lens"], 10.0)
+    qt = oracle.absorb_query_tokens(a["q_c"], a["q_r"], a["w_uk"], a["kv_lens"], 10.0)
+    np.testing.assert_array_equal(qt[:, 0], q1)
+    l1, s1 = oracle.latent_attention(q1, a["cache"], a["kv_lens"], 0.3, d_latent=8)
+    lt, st = oracle.latent_attention_tokens(qt, a["cache"], a["kv_lens"], 0.3, d_latent=8)
+    np.testing.assert_allclose(lt[:, 0], l1, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(st[:, 0], s1, rtol=1e-13)
+
+
+def test_each_new_token_is_a_single_token_decode_on_the_truncated_cache():
+    """Token t of T over L rows is exactly the one-token decode over the first L - T + t + 1
+    rows (its position is the last of them): checked against the pure-Python brute force."""
+    a = _tiny_tokens()
+    B, T, H = a["q_c"].shape[:3]
+    got = oracle.mla_decode_nonabsorbed_tokens(a["q_c"], a["q_r"], a["w_uk"], a["w_uv"], a["cache"],
+                                               a["kv_lens"], 0.41, 10.0)
+    for b in range(B):
+        for t in range(T):
+            n = int(a["kv_lens"][b]) - T + t + 1
+            if n <= 0:
+                np.testing.assert_array_equal(got[b, t], 0.0)
+                continue
+            out, _ = _bruteforce.decode(
+                [a["q_c"][b, t].tolist()], [a["q_r"][b, t].tolist()], a["w_uk"].tolist(),
+                a["w_uv"].tolist(), lambda _b, b=b, n=n: a["cache"][b, :n].tolist(), [n], 0.41, 10.0)
+            np.testing.assert_allclose(got[b, t], np.array(out[0]), rtol=1e-12, atol=1e-12)
+
+
+def test_tokens_absorbed_equals_nonabsorbed():
+    a = _tiny_tokens(seed=61, L=(9, 3))
+    q = oracle.absorb_query_tokens(a["q_c"], a["q_r"], a["w_uk"], a["kv_lens"], 10.0)
+    lat, _ = oracle.latent_attention_tokens(q, a["cache"], a["kv_lens"], 0.41, d_latent=8)
+    out_abs = np.einsum("btic,idc->btid", lat, a["w_uv"])
+    out = oracle.mla_decode_nonabsorbed_tokens(a["q_c"], a["q_r"], a["w_uk"], a["w_uv"], a["cache"],
+                                               a["kv_lens"], 0.41, 10.0)
+    np.testing.assert_allclose(out_abs, out, rtol=1e-11, atol=1e-12)
+
+
+def test_new_tokens_do_not_see_later_new_tokens():
+    a = _tiny_tokens(seed=62, L=(9, 5))
+    q = oracle.absorb_query_tokens(a["q_c"], a["q_r"], a["w_uk"], a["kv_lens"], 10.0)
+    base, _ = oracle.latent_attention_tokens(q, a["cache"], a["kv_lens"], 0.41, d_latent=8)
+    changed = a["cache"].copy()
+    changed[0, 8] += 5.0          # the last new token of sequence 0 (position 8 of 9)
+    lat, _ = oracle.latent_attention_tokens(q, changed, a["kv_lens"], 0.41, d_latent=8)
+    np.testing.assert_array_equal(lat[0, :2], base[0, :2])   # tokens 0 and 1 do not see it
+    assert not np.allclose(lat[0, 2], base[0, 2])            # token 2 (itself) does
+    np.testing.assert_array_equal(lat[1], base[1])
+
+
+def test_tokens_without_visible_rows():
+    a = _tiny_tokens(seed=63, T=3, L=(1, 0))
+    q = oracle.absorb_query_tokens(a["q_c"], a["q_r"], a["w_uk"], a["kv_lens"], 10.0)
+    lat, lse = oracle.latent_attention_tokens(q, a["cache"], a["kv_lens"], 0.41, d_latent=8)
+    assert np.all(lat[0, :2] == 0) and np.all(np.isneginf(lse[0, :2]))
+    assert np.all(np.isfinite(lse[0, 2]))
+    assert np.all(lat[1] == 0) and np.all(np.isneginf(lse[1]))

@@ -75,6 +75,16 @@ typedef struct {
   float yarn_alpha;         /* ramp start, in wavelengths per original context (1)      */
   float yarn_beta;          /* ramp end, > yarn_alpha (32)                               */
   float yarn_mscale_coef;   /* coefficient of ln s in sqrt(t), >= 0 (0.0707)            */
+  /* New tokens per sequence per call, T (multi-token prediction / speculative decoding:
+   * [V3-walk] §4.1, the MTP modules' extra tokens verified by the main model). 0 or 1 =>
+   * one. With T > 1 every per-sequence array below gains a token axis after the batch axis
+   * (q_c [batch, T, n_h, 128], q_abs [batch, T, n_h, 576], out_latent [batch, T, n_h, 512],
+   * lse [batch, T, n_h], latent/out of mla_apply_wuv, hidden [batch, T, d] of
+   * mla_append_kv); kv_lens counts the T new tokens, which sit at positions kv_len - T + t;
+   * token t attends to rows 0 .. kv_len - T + t (a token with none: latent 0, lse -inf) and
+   * its q^R is rotated at max(kv_len - T + t, 0). Limits: n_heads * T <= 128 and
+   * max_batch * T <= 1024. */
+  int32_t q_len;
 } mla_config_t;
 
 /*

@@ -47,6 +47,7 @@ class MlaConfig(ctypes.Structure):
         ("yarn_alpha", ctypes.c_float),
         ("yarn_beta", ctypes.c_float),
         ("yarn_mscale_coef", ctypes.c_float),
+        ("q_len", ctypes.c_int32),
     ]
 
 
@@ -109,11 +110,12 @@ def make_config(n_heads: int, max_batch: int, max_kv_len: int, page_size: int = 
                 softmax_scale: float = 0.0, rope_base: float = 10000.0,
                 max_splits: int = 0, yarn_factor: float = 0.0, yarn_original_len: int = 4096,
                 yarn_alpha: float = 1.0, yarn_beta: float = 32.0,
-                yarn_mscale_coef: float = 0.0707) -> MlaConfig:
-    """yarn_factor > 1 turns on YaRN (DeepSeek-V2 uses 40 with the other defaults)."""
+                yarn_mscale_coef: float = 0.0707, q_len: int = 1) -> MlaConfig:
+    """yarn_factor > 1 turns on YaRN (DeepSeek-V2 uses 40 with the other defaults); q_len > 1
+    makes every call take q_len new tokens per sequence (a token axis after the batch axis)."""
     return MlaConfig(n_heads, 128, 512, 64, page_size, max_batch, max_kv_len,
                      softmax_scale, rope_base, max_splits, yarn_factor, yarn_original_len,
-                     yarn_alpha, yarn_beta, yarn_mscale_coef)
+                     yarn_alpha, yarn_beta, yarn_mscale_coef, q_len)
 
 
 def check_config(cfg: MlaConfig) -> int:
@@ -141,12 +143,14 @@ class MlaDecode:
 
     def __init__(self, n_heads: int, max_batch: int, max_kv_len: int, page_size: int = 0,
                  softmax_scale: float = 0.0, rope_base: float = 10000.0, max_splits: int = 0,
-                 device: Optional[int] = None, **yarn):
+                 device: Optional[int] = None, q_len: int = 1, **yarn):
         """`yarn`: yarn_factor, yarn_original_len, yarn_alpha, yarn_beta, yarn_mscale_coef
-        (make_config)."""
+        (make_config). With q_len > 1 the per-sequence tensors carry a token axis:
+        q_c [B, q_len, n_h, 128], q_abs [B, q_len, n_h, 576], latent [B, q_len, n_h, 512], ..."""
         self._lib = load_library()
+        self.q_len = max(1, int(q_len))
         self.cfg = make_config(n_heads, max_batch, max_kv_len, page_size, softmax_scale,
-                               rope_base, max_splits, **yarn)
+                               rope_base, max_splits, q_len=q_len, **yarn)
         self.device = torch.cuda.current_device() if device is None else int(device)
         h = ctypes.c_void_p()
         _check(self._lib.mla_decode_create(ctypes.byref(self.cfg), self.device, ctypes.byref(h)),
@@ -179,12 +183,12 @@ class MlaDecode:
     def absorb_q(self, q_c: torch.Tensor, q_r: torch.Tensor, w_uk: torch.Tensor,
                  kv_lens: torch.Tensor, q_abs: Optional[torch.Tensor] = None,
                  stream=None) -> torch.Tensor:
-        B, H = q_c.shape[0], q_c.shape[1]
+        B = q_c.shape[0]
         for t, n in ((q_c, "q_c"), (q_r, "q_r"), (w_uk, "w_uk")):
             _need(t, torch.bfloat16, n)
         _need(kv_lens, torch.int32, "kv_lens")
         if q_abs is None:
-            q_abs = torch.empty((B, H, ROW), dtype=torch.bfloat16, device=q_c.device)
+            q_abs = torch.empty(tuple(q_c.shape[:-1]) + (ROW,), dtype=torch.bfloat16, device=q_c.device)
         _need(q_abs, torch.bfloat16, "q_abs")
         _check(self._lib.mla_absorb_q(self._h, B, _ptr(q_c), _ptr(q_r), _ptr(w_uk), _ptr(kv_lens),
                                       _ptr(q_abs), _stream(stream)), "mla_absorb_q")
@@ -197,7 +201,7 @@ class MlaDecode:
         """Write the new token's cache row [RMSNorm(W_DKV h)*gamma ; RoPE(W_KR h)] as token
         kv_lens[b]-1 of every sequence b. hidden [B, d] bf16; w_dkv [512, d]; w_kr [64, d];
         gamma [512]; cache as for decode_attn. Returns the cache."""
-        B, d = hidden.shape
+        B, d = hidden.shape[0], hidden.shape[-1]
         for t, n in ((hidden, "hidden"), (w_dkv, "w_dkv"), (w_kr, "w_kr"), (gamma, "gamma")):
             _need(t, torch.bfloat16, n)
         _need(kv_lens, torch.int32, "kv_lens")
@@ -230,14 +234,15 @@ class MlaDecode:
                     want_lse: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
         """cache: contiguous [B, Lmax, 576] or paged [num_pages, page_size, 576] bf16 rows
         [c^KV ; k^R]. Returns (out_latent [B, n_h, 512] bf16, lse [B, n_h] fp32 or None)."""
-        B, H = q_abs.shape[0], q_abs.shape[1]
+        B = q_abs.shape[0]
         _need(q_abs, torch.bfloat16, "q_abs")
         _need(kv_lens, torch.int32, "kv_lens")
         row_stride, seq_stride, c_kv, k_r, max_pages, num_pages = self._cache_view(cache, page_table)
         if out_latent is None:
-            out_latent = torch.empty((B, H, D_LATENT), dtype=torch.bfloat16, device=q_abs.device)
+            out_latent = torch.empty(tuple(q_abs.shape[:-1]) + (D_LATENT,), dtype=torch.bfloat16,
+                                     device=q_abs.device)
         if lse is None and want_lse:
-            lse = torch.empty((B, H), dtype=torch.float32, device=q_abs.device)
+            lse = torch.empty(tuple(q_abs.shape[:-1]), dtype=torch.float32, device=q_abs.device)
         _check(self._lib.mla_decode_attn(
             self._h, B, _ptr(q_abs), ctypes.c_void_p(c_kv), ctypes.c_void_p(k_r), row_stride,
             seq_stride, _ptr(kv_lens), _ptr(page_table), max_pages, num_pages, _ptr(out_latent),
@@ -246,11 +251,11 @@ class MlaDecode:
 
     def apply_wuv(self, latent: torch.Tensor, w_uv: torch.Tensor,
                   out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-        B, H = latent.shape[0], latent.shape[1]
+        B = latent.shape[0]
         _need(latent, torch.bfloat16, "latent")
         _need(w_uv, torch.bfloat16, "w_uv")
         if out is None:
-            out = torch.empty((B, H, 128), dtype=torch.bfloat16, device=latent.device)
+            out = torch.empty(tuple(latent.shape[:-1]) + (128,), dtype=torch.bfloat16, device=latent.device)
         _need(out, torch.bfloat16, "out")
         _check(self._lib.mla_apply_wuv(self._h, B, _ptr(latent), _ptr(w_uv), _ptr(out),
                                        _stream(stream)), "mla_apply_wuv")

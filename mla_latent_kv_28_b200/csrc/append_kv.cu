@@ -160,7 +160,7 @@ kv_down_tc(const __grid_constant__ CUtensorMap tmap_wd, const __grid_constant__ 
 
 struct FinalParams {
   const float* part;
-  int slices, part_batch;
+  int slices, part_batch, q_len;
   const __nv_bfloat16* gamma;
   float eps;
   const int32_t* kv_lens;
@@ -176,15 +176,16 @@ __global__ void __launch_bounds__(kRow)
 kv_finalize(const FinalParams p) {
   __shared__ float xs[kRow];
   __shared__ float red[kDLatent / 32];
-  const int b = blockIdx.x, f = threadIdx.x, warp = f >> 5, lane = f & 31;
+  // block = one (sequence, new token) row: sequence blockIdx.x / q_len, token blockIdx.x % q_len
+  const int bt = blockIdx.x, b = bt / p.q_len, f = threadIdx.x, warp = f >> 5, lane = f & 31;
   grid_dependency_wait();   // the partial sums of kv_down_tc
   allow_dependent_launch();
   const int64_t L = p.kv_lens[b];
-  if (L < 1 || L > p.max_kv_len) {   // no new token to place
+  if (L < p.q_len || L > p.max_kv_len) {   // no room for the new tokens
     if (f == 0) atomicOr(p.err, kErrBadKvLen);
     return;
   }
-  const int64_t pos = L - 1;
+  const int64_t pos = L - p.q_len + bt % p.q_len;
   int64_t row;
   if (p.cv.page_table == nullptr) {
     row = (int64_t)b * p.cv.seq_stride + pos;
@@ -200,7 +201,7 @@ kv_finalize(const FinalParams p) {
   float v[kAppendSlices];
 #pragma unroll
   for (int s = 0; s < kAppendSlices; ++s)
-    v[s] = s < p.slices ? p.part[((int64_t)s * p.part_batch + b) * kRow + f] : 0.f;
+    v[s] = s < p.slices ? p.part[((int64_t)s * p.part_batch + bt) * kRow + f] : 0.f;
   float x = v[0];
 #pragma unroll
   for (int s = 1; s < kAppendSlices; ++s) x += v[s];
@@ -275,12 +276,13 @@ cudaError_t launch_append_kv(const mla_decode_s& h, int batch, int d_model,
   // finer, to fill every SM, measured slower: the work is latency-bound at these sizes and
   // more slices mean more partial sums to write and add.)
   const int slice = std::max(64, (d_model / kAppendSlices + 63) / 64 * 64);
+  const int rows = batch * h.q_len;   // one row per (sequence, new token)
   const int slices = (d_model + slice - 1) / slice;
-  const int n_tile = std::min(64, (batch + 15) / 16 * 16);
+  const int n_tile = std::min(64, (rows + 15) / 16 * 16);
   CUtensorMap twd, twr, th;
   if (!encode(&twd, w_dkv, kDLatent, (uint64_t)d_model, 128) ||
       !encode(&twr, w_kr, kDRope, (uint64_t)d_model, 128) ||
-      !encode(&th, hidden, (uint64_t)batch, (uint64_t)d_model, (uint32_t)n_tile))
+      !encode(&th, hidden, (uint64_t)rows, (uint64_t)d_model, (uint32_t)n_tile))
     return cudaErrorInvalidValue;
   const int nbox = slice / 64;
   const uint32_t smem = nbox * (kWBox + (uint32_t)n_tile * 128) + 128 + 1024;
@@ -293,22 +295,23 @@ cudaError_t launch_append_kv(const mla_decode_s& h, int batch, int d_model,
   if (attr != cudaSuccess) return attr;
 
   DownParams dp{};
-  dp.batch = batch;
+  dp.batch = rows;
   dp.n_tile = n_tile;
   dp.slice = slice;
   dp.idesc = idesc_bf16_f32(128, n_tile, false, false);
   dp.part = h.ws.append_part;
-  dp.part_batch = h.cfg.max_batch;
+  dp.part_batch = h.cfg.max_batch * h.q_len;
   dp.err = h.ws.err;
   dp.wait_limit = 2000000000LL;
-  cudaError_t e = launch_pdl(kv_down_tc, dim3(kFeatBlocks, slices, (batch + n_tile - 1) / n_tile),
+  cudaError_t e = launch_pdl(kv_down_tc, dim3(kFeatBlocks, slices, (rows + n_tile - 1) / n_tile),
                              dim3(kThreads), smem, s, twd, twr, th, dp);
   if (e != cudaSuccess) return e;
 
   FinalParams fp{};
   fp.part = h.ws.append_part;
   fp.slices = slices;
-  fp.part_batch = h.cfg.max_batch;
+  fp.part_batch = h.cfg.max_batch * h.q_len;
+  fp.q_len = h.q_len;
   fp.gamma = gamma;
   fp.eps = eps;
   fp.kv_lens = kv_lens;
@@ -319,7 +322,7 @@ cudaError_t launch_append_kv(const mla_decode_s& h, int batch, int d_model,
   for (int m = 0; m < kDRope / 2; ++m)
     fp.theta[m] = h.theta[m];
   fp.err = h.ws.err;
-  return launch_pdl(kv_finalize, dim3(batch), dim3(kRow), 0, s, fp);
+  return launch_pdl(kv_finalize, dim3(rows), dim3(kRow), 0, s, fp);
 }
 
 }  // namespace mla

@@ -119,7 +119,7 @@ combine_kernel(PlanView plan, int n_heads, int slot_lanes, int groups_per_block,
 
 cudaError_t launch_combine(const mla_decode_s& h, int batch, __nv_bfloat16* out_latent,
                            float* lse, cudaStream_t s) {
-  const int n_heads = h.cfg.n_heads;
+  const int n_heads = h.n_rows;   // attention rows per sequence (heads x new tokens)
   const int per_block = n_heads >= kThreads ? 1 : kThreads / n_heads;   // head rows per block
   // the most slots one sequence can have: balanced units overlap about units / batch + 1 of a
   // sequence's tiles; capped plans give at most max_splits

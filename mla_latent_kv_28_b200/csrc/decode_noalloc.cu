@@ -126,6 +126,8 @@ extern "C" int mla_decode_attn_noalloc(int32_t n_heads, float softmax_scale, int
 
   mla_decode_s h;  // a handle on the stack: no allocation, scratch pointers into g_scratch
   h.cfg.n_heads = n_heads;
+  h.q_len = 1;
+  h.n_rows = n_heads;
   h.cfg.d_head = kDHead;
   h.cfg.d_latent = kDLatent;
   h.cfg.d_rope = kDRope;

@@ -122,7 +122,8 @@ constexpr float kRescaleThreshold = 8.f;   // log2 units: rescale O only when th
 struct Params {
   const __nv_bfloat16* q_abs;
   PlanView plan;
-  int batch, n_heads;
+  int batch, n_heads;      // n_heads: attention rows per sequence, token-major (heads x new tokens)
+  int q_len, heads_per_token;   // new tokens per sequence; row r is token r / heads_per_token
   int64_t seq_stride;
   const int32_t* page_table;
   int max_pages, num_pages;
@@ -533,6 +534,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
         const uint32_t st = g % kStages, u = g >> 1, xb = u & 1u;
         if (!wait_spin(bar(kBarKvFull + st), (g / kStages) & 1u, guard)) break;
         const int r = tile_valid[st] ? c.rows() : 0;   // valid tokens of the tile
+        // ... of which this row sees those up to its own token's position: new token t of
+        // q_len sits at len - q_len + t and does not see the new tokens after it
+        const int rr = max(0, min(r, c.len - (p.q_len - 1 - h / p.heads_per_token) - c.j()));
         // own partial S out of TMEM (S is free for the next QK once we have it)
         float sv[kT];
         {
@@ -546,9 +550,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
 #pragma unroll
           for (int j = 0; j < 32; ++j) { sv[j] = __uint_as_float(a[j]); sv[32 + j] = __uint_as_float(b[j]); }
         }
-        if (r < kT) {   // the last tile of a sequence (or a skipped page): what is not there is 0 ...
+        if (rr < kT) {   // the last tile of a sequence (or a skipped page): what is not there is 0 ...
 #pragma unroll
-          for (int j = 0; j < kT; ++j) sv[j] = j < r ? sv[j] : 0.f;
+          for (int j = 0; j < kT; ++j) sv[j] = j < rr ? sv[j] : 0.f;
         }
         {   // ... to the peer, then the peer's partial back: S = own + peer
           uint32_t qv[kT / 2];
@@ -578,9 +582,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
           }
           consumed = u + 1;
         }
-        if (r < kT) {
+        if (rr < kT) {
 #pragma unroll
-          for (int j = 0; j < kT; ++j) sv[j] = j < r ? sv[j] : -INFINITY;
+          for (int j = 0; j < kT; ++j) sv[j] = j < rr ? sv[j] : -INFINITY;
         }
         float mx[8];
 #pragma unroll
@@ -857,7 +861,7 @@ cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfl
                                                 : (int64_t)batch * cv.seq_stride;
   if (rows <= 0 || rows >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
   CUtensorMap tc, tr, tq, tqr;
-  const uint64_t qrows = (uint64_t)batch * h.cfg.n_heads;   // q_abs as [B * n_h, 576]
+  const uint64_t qrows = (uint64_t)batch * h.n_rows;   // q_abs as [B * rows, 576]
   if (!encode_latent_groups(&tc, cv.c_kv, (uint64_t)rows, cv.row_stride) ||
       !encode_rows(&tr, cv.k_r, kDRope, (uint64_t)rows, cv.row_stride, 32, CU_TENSOR_MAP_SWIZZLE_64B) ||
       !encode_rows(&tq, q_abs, kRow, qrows, kRow, 64, CU_TENSOR_MAP_SWIZZLE_128B, 128) ||
@@ -868,7 +872,9 @@ cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfl
   p.q_abs = q_abs;
   p.plan = h.ws.plan;
   p.batch = batch;
-  p.n_heads = h.cfg.n_heads;
+  p.n_heads = h.n_rows;
+  p.q_len = h.q_len;
+  p.heads_per_token = h.cfg.n_heads;
   p.seq_stride = cv.seq_stride;
   p.page_table = cv.page_table;
   p.max_pages = cv.max_pages;

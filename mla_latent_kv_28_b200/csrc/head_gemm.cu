@@ -34,7 +34,8 @@ constexpr uint32_t kWeightBytes = 8 * kWeightBox;  // one head's 128 x 512 matri
 enum Mode { kAbsorb = 0, kUpProject = 1 };
 
 struct GemmParams {
-  int batch, n_heads, n_tile;     // n_tile: sequences per CTA (multiple of 16, <= 128)
+  int batch, n_heads, n_tile;     // n_tile: rows per CTA (multiple of 16, <= 128); a row is
+  int q_len;                      // one (sequence, new token): row = sequence * q_len + token
   uint32_t idesc;
   __nv_bfloat16* out;             // q_abs [B, n_h, 576] or out [B, n_h, 128]
   const __nv_bfloat16* q_r;       // absorb only
@@ -55,8 +56,8 @@ __device__ __forceinline__ bool wait_simple(uint32_t bar, uint32_t parity, const
   return true;
 }
 
-// RoPE of the decoupled query of this head for the CTA's sequences, rotated to position
-// kv_len - 1. The angle pos * theta_m reaches ~1.3e5 rad at 128K tokens, so it is formed in
+// RoPE of the decoupled query of this head for the CTA's rows, rotated to the row's token
+// position max(kv_len - q_len + token, 0) (kv_len - 1 for one new token). The angle pos * theta_m reaches ~1.3e5 rad at 128K tokens, so it is formed in
 // double and brought into [-pi, pi] by Cody-Waite reduction with a two-term 2*pi before the
 // sine and cosine are taken; the result is exact to far below bf16 resolution.
 __device__ __forceinline__ void rope_rows(const GemmParams& p, int h, int b0) {
@@ -71,7 +72,8 @@ __device__ __forceinline__ void rope_rows(const GemmParams& p, int h, int b0) {
     const float x0 = __low2float(x), x1 = __high2float(x);
     double y0 = x0, y1 = x1;
     if (p.theta[m] != 0.0) {
-      const double a = (double)max(p.kv_lens[b] - 1, 0) * p.theta[m];
+      const int pos = max(p.kv_lens[b / p.q_len] - p.q_len + b % p.q_len, 0);
+      const double a = (double)pos * p.theta[m];
       const double k = rint(a * kInvTwoPi);
       const double r = fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, a));
       double sn, cs;
@@ -276,6 +278,7 @@ cudaError_t launch(const mla_decode_s& h, int batch, const __nv_bfloat16* w, con
   p.batch = batch;
   p.n_heads = h.cfg.n_heads;
   p.n_tile = n_tile;
+  p.q_len = h.q_len;
   p.idesc = idesc_bf16_f32(128, n_tile, MODE == kAbsorb, false);
   p.out = out;
   p.q_r = q_r;

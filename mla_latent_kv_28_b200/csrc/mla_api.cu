@@ -31,6 +31,12 @@ int config_status(const mla_config_t* c) {
   if (c->page_size != 0 && c->page_size != 64) return MLA_ERR_UNSUPPORTED;
   if (c->max_kv_len > (int64_t)1 << 30) return MLA_ERR_UNSUPPORTED;
   if (c->max_splits > 64) return MLA_ERR_UNSUPPORTED;
+  if (c->q_len < 0) return MLA_ERR_INVALID_ARG;
+  {
+    const int64_t T = c->q_len > 1 ? c->q_len : 1;
+    if ((int64_t)c->n_heads * T > mla::kMaxHeads || (int64_t)c->max_batch * T > mla::kMaxBatch)
+      return MLA_ERR_UNSUPPORTED;
+  }
   if (!(c->yarn_factor >= 0.f) || !std::isfinite(c->yarn_factor) ||
       (c->yarn_factor > 0.f && c->yarn_factor < 1.f))
     return MLA_ERR_INVALID_ARG;
@@ -100,6 +106,8 @@ int mla_decode_create(const mla_config_t* cfg, int device, mla_handle_t* out) {
   h->scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale
                                       : (float)(t / std::sqrt((double)(kDHead + kDRope)));
   rope_frequencies(*cfg, h->theta);
+  h->q_len = cfg->q_len > 1 ? cfg->q_len : 1;
+  h->n_rows = cfg->n_heads * h->q_len;
   h->units = sms / 2;  // the decode kernel runs one 2-CTA cluster per unit of work
 
   const int B = cfg->max_batch;
@@ -114,9 +122,9 @@ int mla_decode_create(const mla_config_t* cfg, int device, mla_handle_t* out) {
   const size_t o_seq_unit = off;  off = round_up(off + 4 * B, 256);
   const size_t o_ubegin = off;    off = round_up(off + 4 * (max_units + 1), 256);
   const size_t o_useq = off;      off = round_up(off + 4 * max_units, 256);
-  const size_t o_plse = off;      off = round_up(off + 4 * (size_t)max_slots * cfg->n_heads, 256);
-  const size_t o_po = off;        off = round_up(off + 4 * (size_t)max_slots * cfg->n_heads * kDLatent, 256);
-  const size_t o_ap = off;        off = round_up(off + 4 * (size_t)mla::kAppendSlices * B * mla::kRow, 256);
+  const size_t o_plse = off;      off = round_up(off + 4 * (size_t)max_slots * h->n_rows, 256);
+  const size_t o_po = off;        off = round_up(off + 4 * (size_t)max_slots * h->n_rows * kDLatent, 256);
+  const size_t o_ap = off;        off = round_up(off + 4 * (size_t)mla::kAppendSlices * B * h->q_len * mla::kRow, 256);
 
   void* base = nullptr;
   if (cudaMalloc(&base, off) != cudaSuccess) {
@@ -169,8 +177,9 @@ int mla_absorb_q(mla_handle_t h, int32_t batch, const void* q_c, const void* q_r
   if (batch < 1 || batch > h->cfg.max_batch) return MLA_ERR_INVALID_ARG;
   if (!aligned16(q_c) || !aligned16(q_r) || !aligned16(w_uk) || !aligned16(q_abs))
     return MLA_ERR_INVALID_ARG;
+  // one GEMM row per (sequence, new token)
   const cudaError_t e = mla::launch_absorb_q(
-      *h, batch, static_cast<const __nv_bfloat16*>(q_c), static_cast<const __nv_bfloat16*>(q_r),
+      *h, batch * h->q_len, static_cast<const __nv_bfloat16*>(q_c), static_cast<const __nv_bfloat16*>(q_r),
       static_cast<const __nv_bfloat16*>(w_uk), kv_lens, static_cast<__nv_bfloat16*>(q_abs), stream);
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
@@ -256,7 +265,7 @@ int mla_apply_wuv(mla_handle_t h, int32_t batch, const void* latent, const void*
   if (batch < 1 || batch > h->cfg.max_batch) return MLA_ERR_INVALID_ARG;
   if (!aligned16(latent) || !aligned16(w_uv) || !aligned16(out)) return MLA_ERR_INVALID_ARG;
   const cudaError_t e = mla::launch_apply_wuv(
-      *h, batch, static_cast<const __nv_bfloat16*>(latent),
+      *h, batch * h->q_len, static_cast<const __nv_bfloat16*>(latent),
       static_cast<const __nv_bfloat16*>(w_uv), static_cast<__nv_bfloat16*>(out), stream);
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }

@@ -61,6 +61,8 @@ struct mla_decode_s {
   int device = 0;
   int num_sms = 0;
   float scale = 0.f;
+  int q_len = 1;    // new tokens per sequence per call
+  int n_rows = 0;   // attention rows per sequence: n_heads * q_len (token-major)
   double theta[mla::kDRope / 2] = {};  // RoPE pair frequencies (0: no rotation), YaRN applied
   int units = 0;  // units the balanced plan cuts the tile space into
   mla::Workspace ws;

@@ -205,3 +205,12 @@ def draw_append_inputs(batch: int, d_model: int = 5120, seed: int = 3) -> dict:
     w_kr = (torch.randn((D_ROPE, d_model), generator=gen) * wstd).to(torch.bfloat16)
     gamma = (1.0 + 0.1 * torch.randn((D_LATENT,), generator=gen)).to(torch.bfloat16)
     return {"hidden": hidden, "w_dkv": w_dkv, "w_kr": w_kr, "gamma": gamma}
+
+
+def draw_token_queries(batch: int, q_len: int, n_heads: int, seed: int = 4):
+    """Queries of q_len new tokens per sequence: q^C [B, T, n_h, 128] and q^R [B, T, n_h, 64],
+    N(0, 1) rounded to bf16 (the one-token recipe with a token axis)."""
+    gen = torch.Generator().manual_seed(seed)
+    q_c = _randn_bf16((batch, q_len, n_heads, D_HEAD), gen)
+    q_r = _randn_bf16((batch, q_len, n_heads, D_ROPE), gen)
+    return q_c, q_r

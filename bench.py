@@ -445,7 +445,8 @@ def run_ours(args):
     dout = [torch.empty((B, H, 128), dtype=torch.bfloat16, device=dev) for _ in range(2)]
     h2d = hq_c.numel() * 2 + hq_r.numel() * 2 + hlens.numel() * 4
     d2h = hout[0].numel() * 2
-    copy = torch.cuda.Stream(dev)
+    copy = torch.cuda.Stream(dev)       # uploads
+    copy_out = torch.cuda.Stream(dev)   # downloads, on another copy engine
 
     def upload(slot):
         for d, hsrc in zip(din[slot], (hq_c, hq_r, hlens)):
@@ -456,15 +457,20 @@ def run_ours(args):
         fork = torch.cuda.Event()
         fork.record(stream)
         copy.wait_event(fork)
+        copy_out.wait_event(fork)
         with torch.cuda.stream(copy):
             upload(1 - slot)                                        # inputs of step k+1
+            join_in = torch.cuda.Event()
+            join_in.record(copy)
+        with torch.cuda.stream(copy_out):
             hout[1 - slot].copy_(dout[1 - slot], non_blocking=True)  # outputs of step k-1
-            join = torch.cuda.Event()
-            join.record(copy)
+            join_out = torch.cuda.Event()
+            join_out.record(copy_out)
         dq_c, dq_r, dlens = din[slot]
         h.step(dq_c, dq_r, g.w_uk, g.w_uv, caches[k % copies], dlens, g.page_table, stream,
                dict(bufs, out=dout[slot]))
-        stream.wait_event(join)
+        stream.wait_event(join_in)
+        stream.wait_event(join_out)
 
     n_graphs = 2 * copies // math.gcd(2, copies)   # input slot and cache copy both cycle
     with torch.cuda.stream(stream):

@@ -152,6 +152,36 @@ int mla_decode_attn(mla_handle_t h, int32_t batch, const void* q_abs, const void
                     int32_t num_pages, void* out_latent, float* lse, mla_stream_t stream);
 
 /*
+ * mla_decode_attn over one shard of each sequence's cache, for a request whose tokens are
+ * spread over several GPUs: the same attention over the rows this caller holds (kv_lens =
+ * the rows held, 0 allowed), with out_latent as fp32 [batch, (T,) n_h, 512] (normalised over
+ * the shard) and lse required. q_abs must be rotated at the request's global position
+ * (mla_absorb_q with the global kv_lens): the cached k^R rows carry their global positions.
+ * The shards' results are merged with mla_merge_partials. Not on the pages: the split-KV
+ * log-sum-exp merge across GPUs is this library's. MLA_ERR_UNSUPPORTED with q_len > 1 (the
+ * causal limits of several new tokens follow their global positions).
+ */
+int mla_decode_attn_partial(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
+                            const void* k_r, int64_t row_stride, int64_t seq_stride,
+                            const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                            int32_t num_pages, float* out_latent, float* lse, mla_stream_t stream);
+
+/*
+ * Log-sum-exp merge of n_parts partial results over disjoint pieces of each sequence's cache:
+ *   lse* = max_p lse_p, w_p = exp(lse_p - lse*),
+ *   out_latent = sum_p w_p latent_p / sum_p w_p (bf16), lse = lse* + log sum_p w_p (fp32).
+ * latent_parts fp32 [n_parts][batch][(T,) n_h][512], lse_parts fp32 [n_parts][batch][(T,) n_h]
+ * (the outputs of mla_decode_attn_partial stacked part by part, e.g. by an all-gather across
+ * GPUs); out_latent bf16 [batch, (T,) n_h, 512]; lse fp32 or NULL. Parts are added in part
+ * order, so the result does not depend on timing. A row whose parts are all empty (lse -inf)
+ * gets latent 0 and lse -inf.
+ * Errors: MLA_ERR_INVALID_ARG for NULL pointers, batch outside 1..max_batch, n_parts < 1,
+ * misalignment.
+ */
+int mla_merge_partials(mla_handle_t h, int32_t batch, int32_t n_parts, const float* latent_parts,
+                       const float* lse_parts, void* out_latent, float* lse, mla_stream_t stream);
+
+/*
  * V up-projection ([V2-walk] §2.3: W_UV is applied last; [V2-arch] eq. 11 v^C = W^UV c^KV):
  *   out[b,i,:] = W_UV,i latent[b,i,:]                               (fp32 accumulation)
  * latent bf16 [batch, n_h, 512]; w_uv bf16 [n_h, 128, 512]; out bf16 [batch, n_h, 128].

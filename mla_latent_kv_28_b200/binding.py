@@ -63,6 +63,9 @@ SIGNATURES = {
     "mla_absorb_q": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P, _P, _P]),
     "mla_decode_attn": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32, _P, _P, _P]),
     "mla_apply_wuv": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P]),
+    "mla_decode_attn_partial": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32,
+                                               _P, _P, _P]),
+    "mla_merge_partials": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _P, _P, _P]),
     "mla_append_kv": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _P, _P, ctypes.c_float, _P, _P,
                                      _I64, _I64, _P, _P, _I32, _I32, _P]),
     "mla_decode_attn_noalloc": (ctypes.c_int, [_I32, ctypes.c_float, _I32, _I64, _I32, _P, _P, _P,
@@ -247,6 +250,50 @@ class MlaDecode:
             self._h, B, _ptr(q_abs), ctypes.c_void_p(c_kv), ctypes.c_void_p(k_r), row_stride,
             seq_stride, _ptr(kv_lens), _ptr(page_table), max_pages, num_pages, _ptr(out_latent),
             _ptr(lse), _stream(stream)), "mla_decode_attn")
+        return out_latent, lse
+
+    def decode_attn_partial(self, q_abs: torch.Tensor, cache: torch.Tensor, kv_lens: torch.Tensor,
+                            page_table: Optional[torch.Tensor] = None,
+                            out_latent: Optional[torch.Tensor] = None,
+                            lse: Optional[torch.Tensor] = None,
+                            stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+        """Attention over the cache rows this caller holds (one shard of each sequence):
+        (latent fp32 [B, (T,) n_h, 512], lse fp32 [B, (T,) n_h]), to be merged across shards
+        with merge_partials. q_abs is rotated at the request's global positions."""
+        B = q_abs.shape[0]
+        _need(q_abs, torch.bfloat16, "q_abs")
+        _need(kv_lens, torch.int32, "kv_lens")
+        row_stride, seq_stride, c_kv, k_r, max_pages, num_pages = self._cache_view(cache, page_table)
+        if out_latent is None:
+            out_latent = torch.empty(tuple(q_abs.shape[:-1]) + (D_LATENT,), dtype=torch.float32,
+                                     device=q_abs.device)
+        if lse is None:
+            lse = torch.empty(tuple(q_abs.shape[:-1]), dtype=torch.float32, device=q_abs.device)
+        _need(out_latent, torch.float32, "out_latent")
+        _need(lse, torch.float32, "lse")
+        _check(self._lib.mla_decode_attn_partial(
+            self._h, B, _ptr(q_abs), ctypes.c_void_p(c_kv), ctypes.c_void_p(k_r), row_stride,
+            seq_stride, _ptr(kv_lens), _ptr(page_table), max_pages, num_pages, _ptr(out_latent),
+            _ptr(lse), _stream(stream)), "mla_decode_attn_partial")
+        return out_latent, lse
+
+    def merge_partials(self, latent_parts: torch.Tensor, lse_parts: torch.Tensor,
+                       out_latent: Optional[torch.Tensor] = None,
+                       lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+                       stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+        """latent_parts fp32 [P, B, (T,) n_h, 512], lse_parts fp32 [P, B, (T,) n_h] ->
+        (latent bf16 [B, (T,) n_h, 512], lse fp32 or None)."""
+        _need(latent_parts, torch.float32, "latent_parts")
+        _need(lse_parts, torch.float32, "lse_parts")
+        P, B = latent_parts.shape[0], latent_parts.shape[1]
+        if out_latent is None:
+            out_latent = torch.empty(tuple(latent_parts.shape[1:]), dtype=torch.bfloat16,
+                                     device=latent_parts.device)
+        if lse is None and want_lse:
+            lse = torch.empty(tuple(lse_parts.shape[1:]), dtype=torch.float32, device=lse_parts.device)
+        _check(self._lib.mla_merge_partials(self._h, B, P, _ptr(latent_parts), _ptr(lse_parts),
+                                            _ptr(out_latent), _ptr(lse), _stream(stream)),
+               "mla_merge_partials")
         return out_latent, lse
 
     def apply_wuv(self, latent: torch.Tensor, w_uv: torch.Tensor,

@@ -184,10 +184,14 @@ int mla_absorb_q(mla_handle_t h, int32_t batch, const void* q_c, const void* q_r
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
-int mla_decode_attn(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
-                    const void* k_r, int64_t row_stride, int64_t seq_stride,
-                    const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
-                    int32_t num_pages, void* out_latent, float* lse, mla_stream_t stream) {
+namespace {
+
+// The shared body of mla_decode_attn (bf16 latent) and mla_decode_attn_partial (fp32).
+int decode_attn_common(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
+                       const void* k_r, int64_t row_stride, int64_t seq_stride,
+                       const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                       int32_t num_pages, void* out_latent, bool out_f32, float* lse,
+                       mla_stream_t stream) {
   if (h == nullptr || q_abs == nullptr || c_kv == nullptr || k_r == nullptr ||
       kv_lens == nullptr || out_latent == nullptr)
     return MLA_ERR_INVALID_ARG;
@@ -215,7 +219,44 @@ int mla_decode_attn(mla_handle_t h, int32_t batch, const void* q_abs, const void
   if (e == cudaSuccess)
     e = mla::launch_decode_split(*h, batch, static_cast<const __nv_bfloat16*>(q_abs), cv, stream);
   if (e == cudaSuccess)
-    e = mla::launch_combine(*h, batch, static_cast<__nv_bfloat16*>(out_latent), lse, stream);
+    e = out_f32 ? mla::launch_combine_f32(*h, batch, static_cast<float*>(out_latent), lse, stream)
+                : mla::launch_combine(*h, batch, static_cast<__nv_bfloat16*>(out_latent), lse, stream);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace
+
+int mla_decode_attn(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
+                    const void* k_r, int64_t row_stride, int64_t seq_stride,
+                    const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                    int32_t num_pages, void* out_latent, float* lse, mla_stream_t stream) {
+  return decode_attn_common(h, batch, q_abs, c_kv, k_r, row_stride, seq_stride, kv_lens, page_table,
+                            max_pages, num_pages, out_latent, false, lse, stream);
+}
+
+int mla_decode_attn_partial(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
+                            const void* k_r, int64_t row_stride, int64_t seq_stride,
+                            const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                            int32_t num_pages, float* out_latent, float* lse, mla_stream_t stream) {
+  if (h == nullptr || lse == nullptr) return MLA_ERR_INVALID_ARG;
+  // several new tokens attend causally by their global positions, which a shard's local row
+  // count does not carry
+  if (h->q_len > 1) return MLA_ERR_UNSUPPORTED;
+  return decode_attn_common(h, batch, q_abs, c_kv, k_r, row_stride, seq_stride, kv_lens, page_table,
+                            max_pages, num_pages, out_latent, true, lse, stream);
+}
+
+int mla_merge_partials(mla_handle_t h, int32_t batch, int32_t n_parts, const float* latent_parts,
+                       const float* lse_parts, void* out_latent, float* lse, mla_stream_t stream) {
+  if (h == nullptr || latent_parts == nullptr || lse_parts == nullptr || out_latent == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > h->cfg.max_batch || n_parts < 1) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(latent_parts) || !aligned16(out_latent) ||
+      (reinterpret_cast<uintptr_t>(lse_parts) & 3) != 0 ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3) != 0))
+    return MLA_ERR_INVALID_ARG;
+  const cudaError_t e = mla::launch_merge_parts(*h, batch, n_parts, latent_parts, lse_parts,
+                                                static_cast<__nv_bfloat16*>(out_latent), lse, stream);
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

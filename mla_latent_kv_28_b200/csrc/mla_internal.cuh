@@ -124,6 +124,13 @@ cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfl
 cudaError_t launch_combine(const mla_decode_s& h, int batch, __nv_bfloat16* out_latent,
                            float* lse, cudaStream_t s);
 
+cudaError_t launch_combine_f32(const mla_decode_s& h, int batch, float* out_latent, float* lse,
+                               cudaStream_t s);
+
+cudaError_t launch_merge_parts(const mla_decode_s& h, int batch, int n_parts, const float* latent_parts,
+                               const float* lse_parts, __nv_bfloat16* out_latent, float* lse_out,
+                               cudaStream_t s);
+
 cudaError_t launch_append_kv(const mla_decode_s& h, int batch, int d_model,
                              const __nv_bfloat16* hidden, const __nv_bfloat16* w_dkv,
                              const __nv_bfloat16* w_kr, const __nv_bfloat16* gamma, float eps,

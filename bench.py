@@ -352,6 +352,56 @@ def append_kv_measure(h, w, g, caches, copies, stream, args, world, local, dev,
             "kernels": "kv_down_tc + kv_finalize", "gpu_launches": 2 * args.steps}
 
 
+def graph_ms(fn, stream, args, world, local, dev):
+    """Device time of fn(k), k = 0..K-1, replayed from one CUDA graph after W eager calls."""
+    with torch.cuda.stream(stream):
+        for k in range(args.warmup):
+            fn(k)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for k in range(args.steps):
+            fn(k)
+    with torch.cuda.stream(stream):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, local, True)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, local, True)
+    del graph
+    return max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+
+
+def multi_token_measure(w, g, caches, copies, stream, args, world, local, dev,
+                        n_heads: int = 16, q_len: int = 8):
+    """Several new tokens per sequence on the same cache: 16 heads x 8 new tokens (128
+    attention rows, e.g. one tensor-parallel shard of the 128 heads verifying 8 draft tokens),
+    the attention call alone, timed like the step. Every token's rows come from the cache
+    once for all its tokens, so the cache bytes per call are those of one-token decode."""
+    from mla_latent_kv_28_b200 import binding
+    hm = binding.MlaDecode(n_heads, w.batch, w.max_kv_len, page_size=w.page_size,
+                           rope_base=w.rope_base, q_len=q_len)
+    qa = wl.draw_q_abs(w.batch, n_heads * q_len, seed=9).view(w.batch, q_len, n_heads, 576).to(dev)
+    lat = torch.empty((w.batch, q_len, n_heads, 512), dtype=torch.bfloat16, device=dev)
+    ms = graph_ms(lambda k: hm.decode_attn(qa, caches[k % copies], g.kv_lens, g.page_table, lat,
+                                           None, want_lse=False, stream=stream),
+                  stream, args, world, local, dev)
+    hm.check_device_errors(stream)
+    hm.close()
+    cache_bytes = w.cached_tokens * ROW_BYTES
+    hbm_gbs, _, peak_kind = measured_peaks()
+    gbs = cache_bytes / (ms * 1e-3) / 1e9
+    return {"n_heads": n_heads, "q_len": q_len, "attn_us": ms * 1e3,
+            "query_tokens_per_s": world * w.batch * q_len / (ms * 1e-3),
+            "kv_gbs": gbs, "frac_of_hbm": gbs / hbm_gbs, "peak_source": f"{peak_kind} hbm_gbs",
+            "gpu_launches": 3 * args.steps}
+
+
 def run_ours(args):
     rank, world, local = dist_env()
     if not torch.cuda.is_available():
@@ -508,6 +558,7 @@ def run_ours(args):
     clocks.stop()
 
     append = append_kv_measure(h, w, g, caches, copies, stream, args, world, local, dev)
+    tokens = multi_token_measure(w, g, caches, copies, stream, args, world, local, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -542,6 +593,7 @@ def run_ours(args):
         "clocks": clocks.summary(w0, w1),
     }
     line["append_kv"] = append
+    line["multi_token"] = tokens
     if cpu is not None:
         line["cpu_baseline"] = cpu
     h.close()

@@ -62,3 +62,21 @@ def test_job_throughput_counts_all_ranks():
 def test_single_rank_needs_no_process_group():
     assert bench.max_over_ranks(3.5, 1, torch.device("cpu")) == 3.5
     bench.barrier(1, 0, cuda=False)  # a no-op without a process group
+
+
+def test_committed_decode_profile_parses():
+    """The ncu summary bench.py reads roofline.traffic from has its hash and byte count lines."""
+    import bench
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "profiles",
+                        "decode_attn_v2_b32_l4096.txt")
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    assert len(vals["kernel_sources_sha"]) == 16
+    assert float(vals["dram_bytes_per_launch"]) > float(vals["algorithmic_bytes_per_launch"]) * 0.9
+    # while the kernel sources are the profiled ones, bench reports the traffic
+    if vals["kernel_sources_sha"] == bench.kernel_sources_sha():
+        assert bench.profiled_traffic("v2_b32_l4096") == float(vals["dram_bytes_per_launch"])

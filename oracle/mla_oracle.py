@@ -32,7 +32,7 @@ decoupled key of [V2-notes] / [V3-walk] §2.3):
 The absorbed form ([V2-walk] §2.3 displayed equation, [V3-walk] §2.3) reaches the same
 o_i through q'_i = W_UK,i^T q^C_i, a latent output sum_j p_j c_j, and W_UV,i last.
 
-Readings where the pages are silent (each is also listed in the design doc):
+Readings where the pages are silent:
   * scale = 1/sqrt(d_h + d_h^R). The pages print only the MHA 1/sqrt(d_h); the MLA
     equations that would fix it are omitted or lost in extraction.
   * RoPE: interleaved pairs (x[2m], x[2m+1]), theta_m = base^(-2m/d_R), angle pos*theta_m,

@@ -232,6 +232,80 @@ def cache_rows(hidden, w_dkv, w_kr, gamma, kv_lens, rope_base: float,
     return rows
 
 
+# ---------------------------------------------------------------------------
+# the quantised latent cache (FP8 rows with one power-of-two scale per token)
+# ---------------------------------------------------------------------------
+# The pages quantise the deployed KV cache to about 6 bits per element on average ([V2-notes]
+# Inference cost; [V2-arch] summary) without giving the format. Reading: each cached row of
+# 576 values is stored as OCP FP8 E4M3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa
+# bits; subnormals; no infinities; S.1111.111 is NaN; largest finite 448) and one scale 2^e
+# per token, e an integer. The quantiser takes the smallest e with max|row| / 2^e <= 448 and
+# rounds row / 2^e to the nearest code, ties to the even code. A power-of-two scale keeps
+# the dequantised values exact in bf16 and fp32.
+
+E4M3_MAX = 448.0
+
+
+def e4m3_value(code: int) -> float:
+    """The value of one E4M3 code, from the format's definition."""
+    code = int(code) & 0xFF
+    sign = -1.0 if code & 0x80 else 1.0
+    exp, man = (code >> 3) & 0xF, code & 0x7
+    if exp == 0xF and man == 0x7:
+        return math.nan
+    if exp == 0:
+        return sign * man * 2.0 ** -9            # subnormal: (man / 8) * 2^(1 - 7)
+    return sign * (1.0 + man / 8.0) * 2.0 ** (exp - 7)
+
+
+_E4M3_TABLE = np.array([e4m3_value(c) for c in range(256)])
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    return _E4M3_TABLE[np.asarray(codes, dtype=np.uint8)]
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Nearest finite E4M3 code to each value (|x| <= 448), ties to the code with an even last
+    bit; found by comparing with every finite code's value."""
+    x = np.asarray(x, dtype=np.float64)
+    codes = np.array([c for c in range(256) if np.isfinite(_E4M3_TABLE[c])], dtype=np.int64)
+    vals = _E4M3_TABLE[codes]
+    d = np.abs(x[..., None] - vals)                                 # [..., finite codes]
+    best = d.min(axis=-1, keepdims=True)
+    tie = d == best
+    # among equally near codes prefer an even code, then the one whose value has x's sign
+    # (the two zeros, 0x00 and 0x80, are both even: keep +0 for x >= 0 and -0 for x < 0)
+    score = tie * 4 + tie * ((codes & 1) == 0) * 2 + tie * (np.signbit(vals) == np.signbit(x)[..., None])
+    return codes[np.argmax(score, axis=-1)].astype(np.uint8)
+
+
+def fp8_row_exponent(row) -> int:
+    """Smallest e with max|row| / 2^e <= 448 (0 for an all-zero row)."""
+    amax = float(np.max(np.abs(widen(row))))
+    if amax == 0.0:
+        return 0
+    e = math.ceil(math.log2(amax / E4M3_MAX))
+    while amax / 2.0 ** e > E4M3_MAX:             # guard against log2 rounding
+        e += 1
+    while e > -200 and amax / 2.0 ** (e - 1) <= E4M3_MAX:
+        e -= 1
+    return e
+
+
+def quantize_rows_fp8(rows):
+    """rows [N, 576] -> (codes uint8 [N, 576], exponents int [N])."""
+    rows = widen(rows)
+    exps = np.array([fp8_row_exponent(r) for r in rows], dtype=np.int64)
+    codes = np.stack([e4m3_encode(r / 2.0 ** e) for r, e in zip(rows, exps)])
+    return codes, exps
+
+
+def dequantize_rows_fp8(codes, exps) -> np.ndarray:
+    """codes [..., 576] uint8, exps [...] -> rows in float64: 2^e * value(code)."""
+    return e4m3_decode(codes) * np.exp2(np.asarray(exps, dtype=np.float64))[..., None]
+
+
 def default_scale(d_head: int = D_HEAD, d_rope: int = D_ROPE, yarn: Optional[Yarn] = None) -> float:
     """1/sqrt(d_h + d_h^R) (the reading of the softmax scale, module doc), times the YaRN
     score factor t when YaRN is on."""

@@ -11,6 +11,7 @@ import os
 
 import numpy as np
 import pytest
+import torch
 
 import oracle
 from oracle import mla_oracle as om
@@ -554,3 +555,47 @@ def test_tokens_without_visible_rows():
     assert np.all(lat[0, :2] == 0) and np.all(np.isneginf(lse[0, :2]))
     assert np.all(np.isfinite(lse[0, 2]))
     assert np.all(lat[1] == 0) and np.all(np.isneginf(lse[1]))
+
+
+# --- the quantised latent cache (E4M3 rows, one power-of-two scale per token) ------------
+
+def test_e4m3_values_at_defining_codes():
+    v = oracle.e4m3_value
+    assert v(0x00) == 0.0 and math.copysign(1.0, v(0x80)) == -1.0
+    assert v(0x01) == 2.0 ** -9          # smallest subnormal
+    assert v(0x08) == 2.0 ** -6          # smallest normal
+    assert v(0x38) == 1.0
+    assert v(0x7E) == 448.0 and v(0xFE) == -448.0
+    assert math.isnan(v(0x7F)) and math.isnan(v(0xFF))
+
+
+def test_e4m3_matches_torch_float8_cast():
+    """Every code decodes as torch's float8_e4m3fn does, and round-to-nearest-even encoding of
+    random values agrees with torch's cast (both the library routine and the definition)."""
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = oracle.e4m3_decode(codes.numpy())
+    assert np.array_equal(np.isnan(ref), np.isnan(got))
+    assert np.array_equal(ref[~np.isnan(ref)], got[~np.isnan(got)])
+    rng = np.random.default_rng(90)
+    x = np.concatenate([rng.uniform(-448, 448, 4000), rng.standard_normal(4000) * 0.01,
+                        rng.standard_normal(2000) * 2.0 ** -8])
+    ours = oracle.e4m3_encode(x)
+    theirs = torch.from_numpy(x).to(torch.float32).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, theirs)
+
+
+def test_fp8_rows_quantise_within_half_a_step():
+    rng = np.random.default_rng(91)
+    rows = rng.standard_normal((20, 576)) * np.exp(rng.uniform(-8, 8, (20, 1)))
+    rows[3] = 0.0
+    codes, exps = oracle.quantize_rows_fp8(rows)
+    deq = oracle.dequantize_rows_fp8(codes, exps)
+    for r, e, d in zip(rows, exps, deq):
+        amax = np.max(np.abs(r))
+        if amax == 0:
+            assert np.all(d == 0)
+            continue
+        assert 224.0 < amax / 2.0 ** e <= 448.0          # the smallest exponent that fits
+        step = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(r) / 2.0 ** e, 2.0 ** -6))) - 3) * 2.0 ** e
+        assert np.all(np.abs(d - r) <= step / 2 * (1 + 1e-12))

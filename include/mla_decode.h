@@ -152,6 +152,21 @@ int mla_decode_attn(mla_handle_t h, int32_t batch, const void* q_abs, const void
                     int32_t num_pages, void* out_latent, float* lse, mla_stream_t stream);
 
 /*
+ * mla_decode_attn over a quantised cache ([V2-notes] Inference cost: the deployed KV cache is
+ * quantised, to about 6 bits per element on average; the format is this library's reading):
+ * cached row r is 576 OCP FP8 E4M3 codes [c^KV (512) ; k^R (64)] at kv_codes + r*row_stride
+ * (bytes) and one power-of-two scale 2^kv_exp[r]; its values are 2^kv_exp[r] times the codes'
+ * values. Row r is indexed as for mla_decode_attn (b*seq_stride + j, or the page table). The
+ * scores, softmax and latent sum are those of mla_decode_attn on the dequantised rows (which
+ * are exact in bf16). kv_exp int8, one per row; row_stride a multiple of 16, >= 576. Outputs,
+ * kv_lens, page table and errors as for mla_decode_attn.
+ */
+int mla_decode_attn_fp8(mla_handle_t h, int32_t batch, const void* q_abs, const void* kv_codes,
+                        const int8_t* kv_exp, int64_t row_stride, int64_t seq_stride,
+                        const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                        int32_t num_pages, void* out_latent, float* lse, mla_stream_t stream);
+
+/*
  * mla_decode_attn over one shard of each sequence's cache, for a request whose tokens are
  * spread over several GPUs: the same attention over the rows this caller holds (kv_lens =
  * the rows held, 0 allowed), with out_latent as fp32 [batch, (T,) n_h, 512] (normalised over

@@ -63,6 +63,7 @@ SIGNATURES = {
     "mla_absorb_q": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P, _P, _P]),
     "mla_decode_attn": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32, _P, _P, _P]),
     "mla_apply_wuv": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P]),
+    "mla_decode_attn_fp8": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32, _P, _P, _P]),
     "mla_decode_attn_partial": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32,
                                                _P, _P, _P]),
     "mla_merge_partials": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _P, _P, _P]),
@@ -250,6 +251,39 @@ class MlaDecode:
             self._h, B, _ptr(q_abs), ctypes.c_void_p(c_kv), ctypes.c_void_p(k_r), row_stride,
             seq_stride, _ptr(kv_lens), _ptr(page_table), max_pages, num_pages, _ptr(out_latent),
             _ptr(lse), _stream(stream)), "mla_decode_attn")
+        return out_latent, lse
+
+    def decode_attn_fp8(self, q_abs: torch.Tensor, codes: torch.Tensor, exps: torch.Tensor,
+                        kv_lens: torch.Tensor, page_table: Optional[torch.Tensor] = None,
+                        out_latent: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                        want_lse: bool = True, stream=None):
+        """Attention over a quantised cache: codes uint8 [B, Lmax, 576] or [P, 64, 576] (E4M3),
+        exps int8 [B, Lmax] or [P, 64] (row r is 2^exps[r] times its codes' values)."""
+        B = q_abs.shape[0]
+        _need(q_abs, torch.bfloat16, "q_abs")
+        _need(kv_lens, torch.int32, "kv_lens")
+        if not codes.is_cuda or codes.dtype != torch.uint8 or codes.dim() != 3 or codes.stride(-1) != 1:
+            raise ValueError("codes: expected a CUDA uint8 [*, *, 576] tensor with unit inner stride")
+        _need(exps, torch.int8, "exps")
+        if exps.stride(-1) != 1 or exps.shape != codes.shape[:2]:
+            raise ValueError("exps: one int8 per cached row, shaped like codes[..., 0]")
+        row_stride = codes.stride(1)
+        seq_stride = codes.stride(0) // row_stride
+        if exps.stride(0) != seq_stride:
+            raise ValueError("exps must index rows as codes does")
+        max_pages = num_pages = 0
+        if page_table is not None:
+            _need(page_table, torch.int32, "page_table")
+            max_pages, num_pages, seq_stride = page_table.shape[1], codes.shape[0], 0
+        if out_latent is None:
+            out_latent = torch.empty(tuple(q_abs.shape[:-1]) + (D_LATENT,), dtype=torch.bfloat16,
+                                     device=q_abs.device)
+        if lse is None and want_lse:
+            lse = torch.empty(tuple(q_abs.shape[:-1]), dtype=torch.float32, device=q_abs.device)
+        _check(self._lib.mla_decode_attn_fp8(
+            self._h, B, _ptr(q_abs), _ptr(codes), _ptr(exps), row_stride, seq_stride, _ptr(kv_lens),
+            _ptr(page_table), max_pages, num_pages, _ptr(out_latent), _ptr(lse), _stream(stream)),
+            "mla_decode_attn_fp8")
         return out_latent, lse
 
     def decode_attn_partial(self, q_abs: torch.Tensor, cache: torch.Tensor, kv_lens: torch.Tensor,

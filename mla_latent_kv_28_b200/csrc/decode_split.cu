@@ -44,6 +44,8 @@
 #include <algorithm>
 #include <mutex>
 
+#include <cuda_fp16.h>
+
 #include "mla_internal.cuh"
 #include "sm100.cuh"
 
@@ -93,7 +95,9 @@ constexpr int kBarQReady0 = kBarXFull + 16;      // the first segment's query co
 constexpr int kBarQLanded = kBarQReady0 + 1;     // ... and in shared memory (stages 1-2)
 constexpr int kBarMHand = kBarQLanded + 1;       // [4 head quarters] running max of tile g-1 published
 constexpr int kBarMlFull1 = kBarMHand + 4;      // ... of a finished odd segment
-constexpr int kNumBars = kBarMlFull1 + 1;
+constexpr int kBarKvConv = kBarMlFull1 + 1;     // [kStages] quantised cache: the tile expanded to bf16
+constexpr int kBarConvSync = kBarKvConv + kStages;   // quantised cache: the expanding warpgroup's codes are read
+constexpr int kNumBars = kBarConvSync + 1;
 // The first segment's query columns arrive by TMA in stages 1-2 (exactly 72 KB: four 64-column
 // boxes of 128 heads with 128-byte swizzle, then one 32-column k^R box with 64-byte swizzle);
 // the producer fills those stages with cache tiles only after the query has moved to TMEM.
@@ -132,6 +136,9 @@ struct Params {
   float* part_lse;
   uint32_t* err;
   long long wait_limit;
+  // quantised cache (E4M3 codes + one power-of-two scale per row), else kv_exp == nullptr
+  const int8_t* kv_exp;
+  int64_t kv_rows;          // rows of the cache, for the bounds of the exponent loads
 };
 
 // Walks this cluster's work tile by tile: units in turn, the segments (one sequence's
@@ -254,6 +261,63 @@ __device__ __forceinline__ void q_part_from_smem(uint8_t* smem, uint32_t tmem, u
   q_chunks_out(v, smem, tmem, lanes, h, part);
 }
 
+// The quantised cache's tile in a stage: each 64-column box's E4M3 codes (64 rows x 64 bytes,
+// landed by TMA) sit in the upper half of that box's bf16 slot, the k^R codes (64 rows x 32
+// bytes) in the upper half of the k^R slot. The transition warpgroup expands them in place
+// into the layout the bf16 cache lands in (128- and 64-byte swizzles): every thread first
+// reads its codes (thread t: row t/2, half t%2 of each box), the warpgroup meets, then the
+// threads write; so no code is overwritten before it is read.
+constexpr uint32_t kQ8StageBytes = 4 * (kBoxC / 2) + kBoxR / 2;   // 18 KB of codes per tile
+struct TileCodes {
+  uint4 c[4][2];   // 32 c^KV codes of each box
+  uint4 r;         // 16 k^R codes
+};
+
+__device__ __forceinline__ void read_codes(const uint8_t* stage, int t, TileCodes& v) {
+  const int row = t >> 1, half = t & 1;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+      v.c[i][k] = *reinterpret_cast<const uint4*>(stage + i * kBoxC + kBoxC / 2 + row * 64 + half * 32 + 16 * k);
+  v.r = *reinterpret_cast<const uint4*>(stage + 4 * kBoxC + kBoxR / 2 + row * 32 + half * 16);
+}
+
+// Two E4M3 codes (low byte first) -> their values times 2^e as a bf16 pair. E4M3 -> f16 is
+// exact (the hardware conversion), f16 -> f32 too, and a power-of-two scale keeps the
+// product exact in bf16 (3 mantissa bits), so the expansion adds no rounding.
+__device__ __forceinline__ uint32_t e4m3x2_bf16x2(uint32_t codes2, float scale) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((unsigned short)(codes2 & 0xFFFFu)));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+  __nv_bfloat162 b = __floats2bfloat162_rn(f.x * scale, f.y * scale);
+  return *reinterpret_cast<uint32_t*>(&b);
+}
+
+__device__ __forceinline__ uint4 expand8(uint32_t lo4, uint32_t hi4, float scale) {
+  return make_uint4(e4m3x2_bf16x2(lo4, scale), e4m3x2_bf16x2(lo4 >> 16, scale),
+                    e4m3x2_bf16x2(hi4, scale), e4m3x2_bf16x2(hi4 >> 16, scale));
+}
+
+__device__ __forceinline__ void write_bf16(uint8_t* stage, int t, const TileCodes& v, float scale) {
+  const int row = t >> 1, half = t & 1;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {   // 16-byte chunk half*4 + k of the row: 8 columns
+      const uint4 w = v.c[i][k >> 1];
+      const int chunk = half * 4 + k;
+      *reinterpret_cast<uint4*>(stage + i * kBoxC + row * 128 + ((chunk ^ (row & 7)) << 4)) =
+          (k & 1) ? expand8(w.z, w.w, scale) : expand8(w.x, w.y, scale);
+    }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int chunk = half * 2 + k;
+    *reinterpret_cast<uint4*>(stage + 4 * kBoxC + row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4)) =
+        k ? expand8(v.r.z, v.r.w, scale) : expand8(v.r.x, v.r.y, scale);
+  }
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constant__ CUtensorMap tmap_r,
                 const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_qr,
@@ -266,6 +330,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   volatile int* tile_valid = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);  // [kStages]
+  volatile long long* tile_row_s = reinterpret_cast<volatile long long*>(smem + kOffMisc + 24);  // [kStages]
+  const bool q8 = p.kv_exp != nullptr;   // quantised cache
   float2* ml = reinterpret_cast<float2*>(smem + kOffMl);                             // [2][2][128]
   volatile float* mh = reinterpret_cast<volatile float*>(smem + kOffMh);             // [128]
   volatile int* epi_seg = reinterpret_cast<volatile int*>(smem + kOffEpi);           // [128]
@@ -298,6 +364,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     mbar_init(bar(kBarOFree), 128);
     mbar_init(bar(kBarMlFull), 256);
     mbar_init(bar(kBarMlFull1), 256);
+    for (int i = 0; i < kStages; ++i) mbar_init(bar(kBarKvConv + i), 128);
+    mbar_init(bar(kBarConvSync), 128);
     for (int i = 0; i < 128; ++i) epi_seg[i] = 0;
     mbar_init(bar(kBarFinal), 1);
     *abort_flag = 0;
@@ -354,8 +422,16 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
         const bool ok = row >= 0;
         if (!ok) atomicOr(p.err, kErrBadPage);
         tile_valid[st] = ok ? 1 : 0;
+        tile_row_s[st] = row;
         const uint32_t dst = sbase + st * kStageBytes;
-        if (ok) {
+        if (ok && q8) {   // the codes, each box's into the upper half of its bf16 slot
+          mbar_arrive_expect_tx(bar(kBarKvFull + st), kQ8StageBytes);
+          for (int i = 0; i < 4; ++i)
+            tma_load_2d(dst + i * kBoxC + kBoxC / 2, &tmap_c, 256 * (int)rank + 64 * i, (int)row,
+                        bar(kBarKvFull + st));
+          tma_load_2d(dst + 4 * kBoxC + kBoxR / 2, &tmap_r, kDLatent + 32 * (int)rank, (int)row,
+                      bar(kBarKvFull + st));
+        } else if (ok) {
           mbar_arrive_expect_tx(bar(kBarKvFull + st), kStageBytes);
           // the CTA's four 64-column c^KV boxes in one copy (3-D map: column, row, column group),
           // then its 32 k^R columns: two TMA instructions per tile keep the producer's warp
@@ -381,7 +457,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       c.init(p);
       for (; c.valid; c.next(p)) {
         const uint32_t g = c.g, st = g % kStages;
-        if (!wait_bounded(bar(kBarKvFull + st), (g / kStages) & 1u, guard)) break;
+        // the tile in bf16: landed, or (quantised cache) landed and expanded
+        if (!wait_bounded(bar((q8 ? kBarKvConv : kBarKvFull) + st), (g / kStages) & 1u, guard)) break;
         // S is free once the softmax copied S(g-1) out (tile g-1's warpgroup)
         if (g > 0 && !wait_bounded(bar(kBarSEmpty + ((g - 1) & 1u)), ((g - 1) >> 1) & 1u, guard)) break;
         if (c.first() && !wait_bounded(c.seg == 0 ? bar(kBarQReady0) : bar(kBarQReady),
@@ -754,6 +831,27 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       mbar_arrive(bar(kBarOFree));
       return true;
     };
+    // Quantised cache: expand tile g's codes in place (see read_codes), then let its QK go.
+    uint32_t n_expanded = 0;
+    auto expand_tile = [&](uint32_t g) -> bool {
+      const uint32_t st = g % kStages;
+      if (!wait_bounded(bar(kBarKvFull + st), (g / kStages) & 1u, guard)) return false;
+      const int t = (int)threadIdx.x - 384;   // 0..127 within this warpgroup
+      const int64_t row0 = tile_row_s[st];
+      const int64_t row = row0 + (t >> 1);
+      const int e = (row0 >= 0 && row < p.kv_rows) ? (int)p.kv_exp[row] : 0;
+      const float scale = __uint_as_float((uint32_t)(min(max(e, -126), 127) + 127) << 23);   // 2^e
+      uint8_t* stage = smem + st * kStageBytes;
+      TileCodes v;
+      read_codes(stage, t, v);
+      mbar_arrive(bar(kBarConvSync));
+      if (!wait_bounded(bar(kBarConvSync), n_expanded & 1u, guard)) return false;
+      ++n_expanded;
+      write_bf16(stage, t, v, scale);
+      fence_proxy_async_smem();   // read by the MMAs (async proxy)
+      mbar_arrive(bar(kBarKvConv + st));
+      return true;
+    };
     bool ok = true;
     while (ok && c.valid) {
       const uint32_t seg = c.seg;
@@ -780,11 +878,23 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
           mbar_arrive(bar(kBarQReady));
         }
       }
-      // the previous segment's output, while this one runs
-      if (seg > 0) ok = epilogue(seg - 1, prev_slot);
-      prev_slot = c.slot;
-      // skip to the next segment, and pull its query rows into L2 while this one runs
-      while (c.valid && c.seg == seg) c.next(p);
+      // the previous segment's output, while this one runs (with a quantised cache, after
+      // this segment's first tile is expanded, so that its QK does not wait for the epilogue)
+      if (seg > 0 && !q8) ok = epilogue(seg - 1, prev_slot);
+      const int seg_slot = c.slot;
+      // walk to the next segment (expanding each quantised tile on the way), and pull its
+      // query rows into L2 while this one runs
+      bool first_tile = true;
+      while (ok && c.valid && c.seg == seg) {
+        if (q8) {
+          if (!expand_tile(c.g)) { ok = false; break; }
+          if (first_tile && seg > 0) ok = epilogue(seg - 1, prev_slot);
+        }
+        first_tile = false;
+        c.next(p);
+      }
+      prev_slot = seg_slot;
+      if (!ok) break;
       if (c.valid && head_ok) {
         const __nv_bfloat16* qrow = p.q_abs + ((int64_t)c.b * p.n_heads + h) * kRow;
         asm volatile("prefetch.global.L2 [%0];" :: "l"(qrow + 256 * (int)rank) : "memory");
@@ -845,6 +955,21 @@ bool encode_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The quantised cache's codes as a 2-D byte tensor [rows, 576] with {box_cols, 64} boxes, no
+// swizzle: a box lands as 64 dense rows of box_cols bytes.
+bool encode_codes(CUtensorMap* m, const void* base, uint64_t rows, int64_t row_stride_bytes,
+                  uint32_t box_cols) {
+  const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)kRow, rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)row_stride_bytes};
+  const cuuint32_t box[2] = {box_cols, (cuuint32_t)kT};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfloat16* q_abs,
@@ -862,8 +987,13 @@ cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfl
   if (rows <= 0 || rows >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
   CUtensorMap tc, tr, tq, tqr;
   const uint64_t qrows = (uint64_t)batch * h.n_rows;   // q_abs as [B * rows, 576]
-  if (!encode_latent_groups(&tc, cv.c_kv, (uint64_t)rows, cv.row_stride) ||
-      !encode_rows(&tr, cv.k_r, kDRope, (uint64_t)rows, cv.row_stride, 32, CU_TENSOR_MAP_SWIZZLE_64B) ||
+  const bool cache_ok =
+      cv.kv_exp != nullptr
+          ? encode_codes(&tc, cv.c_kv, (uint64_t)rows, cv.row_stride, 64) &&
+                encode_codes(&tr, cv.c_kv, (uint64_t)rows, cv.row_stride, 32)
+          : encode_latent_groups(&tc, cv.c_kv, (uint64_t)rows, cv.row_stride) &&
+                encode_rows(&tr, cv.k_r, kDRope, (uint64_t)rows, cv.row_stride, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (!cache_ok ||
       !encode_rows(&tq, q_abs, kRow, qrows, kRow, 64, CU_TENSOR_MAP_SWIZZLE_128B, 128) ||
       !encode_rows(&tqr, q_abs, kRow, qrows, kRow, 32, CU_TENSOR_MAP_SWIZZLE_64B, 128))
     return cudaErrorInvalidValue;
@@ -884,6 +1014,8 @@ cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfl
   p.part_lse = h.ws.part_lse;
   p.err = h.ws.err;
   p.wait_limit = 2000000000LL;  // SM cycles, about a second
+  p.kv_exp = cv.kv_exp;
+  p.kv_rows = rows;
 
   const int pairs = std::max(1, std::min(h.units, h.num_sms / 2));
   // the 2-CTA cluster shape is compiled into the kernel

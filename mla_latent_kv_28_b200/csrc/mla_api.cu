@@ -234,6 +234,42 @@ int mla_decode_attn(mla_handle_t h, int32_t batch, const void* q_abs, const void
                             max_pages, num_pages, out_latent, false, lse, stream);
 }
 
+int mla_decode_attn_fp8(mla_handle_t h, int32_t batch, const void* q_abs, const void* kv_codes,
+                        const int8_t* kv_exp, int64_t row_stride, int64_t seq_stride,
+                        const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                        int32_t num_pages, void* out_latent, float* lse, mla_stream_t stream) {
+  if (h == nullptr || q_abs == nullptr || kv_codes == nullptr || kv_exp == nullptr ||
+      kv_lens == nullptr || out_latent == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > h->cfg.max_batch) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_abs) || !aligned16(kv_codes) || !aligned16(out_latent) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3) != 0))
+    return MLA_ERR_INVALID_ARG;
+  if (row_stride < mla::kRow || row_stride % 16 != 0) return MLA_ERR_INVALID_ARG;   // bytes
+  mla::CacheView cv{};
+  cv.c_kv = static_cast<const __nv_bfloat16*>(kv_codes);   // read as bytes by the kernel
+  cv.k_r = nullptr;
+  cv.row_stride = row_stride;
+  cv.page_size = h->cfg.page_size;
+  cv.kv_exp = kv_exp;
+  if (h->cfg.page_size == 0) {
+    if (page_table != nullptr || seq_stride < h->cfg.max_kv_len) return MLA_ERR_INVALID_ARG;
+    cv.seq_stride = seq_stride;
+  } else {
+    const int64_t need = (h->cfg.max_kv_len + h->cfg.page_size - 1) / h->cfg.page_size;
+    if (page_table == nullptr || max_pages < need || num_pages < 1) return MLA_ERR_INVALID_ARG;
+    cv.page_table = page_table;
+    cv.max_pages = max_pages;
+    cv.num_pages = num_pages;
+  }
+  cudaError_t e = mla::launch_split_plan(*h, batch, kv_lens, stream);
+  if (e == cudaSuccess)
+    e = mla::launch_decode_split(*h, batch, static_cast<const __nv_bfloat16*>(q_abs), cv, stream);
+  if (e == cudaSuccess)
+    e = mla::launch_combine(*h, batch, static_cast<__nv_bfloat16*>(out_latent), lse, stream);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 int mla_decode_attn_partial(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
                             const void* k_r, int64_t row_stride, int64_t seq_stride,
                             const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,

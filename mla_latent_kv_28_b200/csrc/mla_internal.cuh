@@ -116,6 +116,9 @@ struct CacheView {
   int32_t max_pages;
   int32_t num_pages;
   int32_t page_size;
+  // quantised cache: c_kv / k_r point at E4M3 codes (row_stride in bytes), and row r's values
+  // are 2^kv_exp[r] times its codes' values
+  const int8_t* kv_exp = nullptr;
 };
 
 cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfloat16* q_abs,

@@ -28,3 +28,5 @@ def test_bench_json_line():
     assert app["us"] > 0 and 0 < app["frac_of_hbm"] < 1.5 and app["gpu_launches"] == 2 * 5
     mt = line["multi_token"]
     assert mt["q_len"] == 8 and mt["attn_us"] > 0 and mt["query_tokens_per_s"] > 0
+    q8 = line["fp8_cache"]
+    assert q8["attn_us"] > 0 and 0 < q8["frac_of_hbm"] < 1.5

@@ -44,8 +44,6 @@
 #include <algorithm>
 #include <mutex>
 
-#include <cuda_fp16.h>
-
 #include "mla_internal.cuh"
 #include "sm100.cuh"
 
@@ -283,23 +281,34 @@ __device__ __forceinline__ void read_codes(const uint8_t* stage, int t, TileCode
   v.r = *reinterpret_cast<const uint4*>(stage + 4 * kBoxC + kBoxR / 2 + row * 32 + half * 16);
 }
 
-// Two E4M3 codes (low byte first) -> their values times 2^e as a bf16 pair. E4M3 -> f16 is
-// exact (the hardware conversion), f16 -> f32 too, and a power-of-two scale keeps the
-// product exact in bf16 (3 mantissa bits), so the expansion adds no rounding.
-__device__ __forceinline__ uint32_t e4m3x2_bf16x2(uint32_t codes2, float scale) {
-  uint32_t h2;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((unsigned short)(codes2 & 0xFFFFu)));
-  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
-  __nv_bfloat162 b = __floats2bfloat162_rn(f.x * scale, f.y * scale);
-  return *reinterpret_cast<uint32_t*>(&b);
+// An E4M3 code as fp32 bits, exponent and mantissa fields moved 20 bits up and the sign to
+// bit 31: that fp32 is the code's value times 2^-120 for every finite code (the normal ones,
+// whose fp32 exponent field is theirs, and the subnormal ones and zero, which land on fp32
+// subnormals and zero). A multiply by 2^120 gives the code's value (normal, at most 448), a
+// second by 2^e the scaled value, both exactly, and the product's upper 16 bits are its bf16
+// (4 significant bits survive any power-of-two scale that keeps the value a normal bf16:
+// e in [-117, 118], far wider than a quantised row needs). No conversion instructions:
+// shifts, logic and two multiplies per value. (The NaN codes 0x7F and 0xFF, which the
+// quantiser never writes, read as 480.)
+__device__ __forceinline__ float e4m3_scaled(uint32_t byte_in_top, float scale) {
+  const uint32_t bits = (byte_in_top & 0x80000000u) | ((byte_in_top >> 4) & 0x07F00000u);
+  return __uint_as_float(bits) * 0x1p120f * scale;
 }
 
-__device__ __forceinline__ uint4 expand8(uint32_t lo4, uint32_t hi4, float scale) {
-  return make_uint4(e4m3x2_bf16x2(lo4, scale), e4m3x2_bf16x2(lo4 >> 16, scale),
-                    e4m3x2_bf16x2(hi4, scale), e4m3x2_bf16x2(hi4 >> 16, scale));
+// Four codes (one word, low byte first) -> two bf16 pairs, in order.
+__device__ __forceinline__ uint2 expand4(uint32_t w, float scale120) {
+  const float v0 = e4m3_scaled(w << 24, scale120), v1 = e4m3_scaled(w << 16, scale120);
+  const float v2 = e4m3_scaled(w << 8, scale120), v3 = e4m3_scaled(w, scale120);
+  return make_uint2(__byte_perm(__float_as_uint(v0), __float_as_uint(v1), 0x7632),
+                    __byte_perm(__float_as_uint(v2), __float_as_uint(v3), 0x7632));
 }
 
-__device__ __forceinline__ void write_bf16(uint8_t* stage, int t, const TileCodes& v, float scale) {
+__device__ __forceinline__ uint4 expand8(uint32_t lo4, uint32_t hi4, float scale120) {
+  const uint2 a = expand4(lo4, scale120), b = expand4(hi4, scale120);
+  return make_uint4(a.x, a.y, b.x, b.y);
+}
+
+__device__ __forceinline__ void write_bf16(uint8_t* stage, int t, const TileCodes& v, float scale120) {
   const int row = t >> 1, half = t & 1;
 #pragma unroll
   for (int i = 0; i < 4; ++i)
@@ -308,16 +317,19 @@ __device__ __forceinline__ void write_bf16(uint8_t* stage, int t, const TileCode
       const uint4 w = v.c[i][k >> 1];
       const int chunk = half * 4 + k;
       *reinterpret_cast<uint4*>(stage + i * kBoxC + row * 128 + ((chunk ^ (row & 7)) << 4)) =
-          (k & 1) ? expand8(w.z, w.w, scale) : expand8(w.x, w.y, scale);
+          (k & 1) ? expand8(w.z, w.w, scale120) : expand8(w.x, w.y, scale120);
     }
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const int chunk = half * 2 + k;
     *reinterpret_cast<uint4*>(stage + 4 * kBoxC + row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4)) =
-        k ? expand8(v.r.z, v.r.w, scale) : expand8(v.r.x, v.r.y, scale);
+        k ? expand8(v.r.z, v.r.w, scale120) : expand8(v.r.x, v.r.y, scale120);
   }
 }
 
+// kQ8: the cache is quantised (E4M3 codes expanded in shared memory); a separate
+// instantiation, so that the bf16 kernel carries none of that code.
+template <bool kQ8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constant__ CUtensorMap tmap_r,
                 const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_qr,
@@ -331,7 +343,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   volatile int* tile_valid = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);  // [kStages]
   volatile long long* tile_row_s = reinterpret_cast<volatile long long*>(smem + kOffMisc + 24);  // [kStages]
-  const bool q8 = p.kv_exp != nullptr;   // quantised cache
+  constexpr bool q8 = kQ8;   // quantised cache
   float2* ml = reinterpret_cast<float2*>(smem + kOffMl);                             // [2][2][128]
   volatile float* mh = reinterpret_cast<volatile float*>(smem + kOffMh);             // [128]
   volatile int* epi_seg = reinterpret_cast<volatile int*>(smem + kOffEpi);           // [128]
@@ -840,14 +852,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       const int64_t row0 = tile_row_s[st];
       const int64_t row = row0 + (t >> 1);
       const int e = (row0 >= 0 && row < p.kv_rows) ? (int)p.kv_exp[row] : 0;
-      const float scale = __uint_as_float((uint32_t)(min(max(e, -126), 127) + 127) << 23);   // 2^e
+      const float scale120 = __uint_as_float((uint32_t)(min(max(e, -126), 127) + 127) << 23);   // 2^e
       uint8_t* stage = smem + st * kStageBytes;
       TileCodes v;
       read_codes(stage, t, v);
       mbar_arrive(bar(kBarConvSync));
       if (!wait_bounded(bar(kBarConvSync), n_expanded & 1u, guard)) return false;
       ++n_expanded;
-      write_bf16(stage, t, v, scale);
+      write_bf16(stage, t, v, scale120);
       fence_proxy_async_smem();   // read by the MMAs (async proxy)
       mbar_arrive(bar(kBarKvConv + st));
       return true;
@@ -977,8 +989,11 @@ cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfl
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(decode_split_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr_err = cudaFuncSetAttribute(decode_split_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)kSmemAlloc);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(decode_split_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kSmemAlloc);
   });
   if (attr_err != cudaSuccess) return attr_err;
 
@@ -1019,7 +1034,9 @@ cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfl
 
   const int pairs = std::max(1, std::min(h.units, h.num_sms / 2));
   // the 2-CTA cluster shape is compiled into the kernel
-  return launch_pdl(decode_split_tc, dim3(2 * pairs), dim3(kThreads), kSmemAlloc, s, tc, tr, tq, tqr, p);
+  return cv.kv_exp != nullptr
+             ? launch_pdl(decode_split_tc<true>, dim3(2 * pairs), dim3(kThreads), kSmemAlloc, s, tc, tr, tq, tqr, p)
+             : launch_pdl(decode_split_tc<false>, dim3(2 * pairs), dim3(kThreads), kSmemAlloc, s, tc, tr, tq, tqr, p);
 }
 
 }  // namespace mla

@@ -36,10 +36,16 @@
 // the two softmax warpgroups, one thread per head (= TMEM lane) and all 64 tokens of a tile;
 // 12..15 segment transitions (query load, epilogue).
 //
+// A quantised cache (E4M3 codes, one power-of-two scale per row) runs through a second
+// instantiation: the producer lands each tile's codes in the upper halves of the stage's bf16
+// boxes, the transition warpgroup expands them in place to exactly the bf16 rows (see
+// e4m3_expand.cuh) and only then lets the tile's QK go; the rest is the same kernel.
+//
 // Every wait is bounded: after about a second it sets the device error word (timeout bit)
 // and the CTA's abort flag, all roles leave their loops, wait for their own copies and
 // MMAs in flight, and the CTA frees its tensor memory and exits.
 #include <cudaTypedefs.h>
+#include <cuda_fp16.h>
 
 #include <algorithm>
 #include <mutex>
@@ -259,73 +265,8 @@ __device__ __forceinline__ void q_part_from_smem(uint8_t* smem, uint32_t tmem, u
   q_chunks_out(v, smem, tmem, lanes, h, part);
 }
 
-// The quantised cache's tile in a stage: each 64-column box's E4M3 codes (64 rows x 64 bytes,
-// landed by TMA) sit in the upper half of that box's bf16 slot, the k^R codes (64 rows x 32
-// bytes) in the upper half of the k^R slot. The transition warpgroup expands them in place
-// into the layout the bf16 cache lands in (128- and 64-byte swizzles): every thread first
-// reads its codes (thread t: row t/2, half t%2 of each box), the warpgroup meets, then the
-// threads write; so no code is overwritten before it is read.
-constexpr uint32_t kQ8StageBytes = 4 * (kBoxC / 2) + kBoxR / 2;   // 18 KB of codes per tile
-struct TileCodes {
-  uint4 c[4][2];   // 32 c^KV codes of each box
-  uint4 r;         // 16 k^R codes
-};
+#include "e4m3_expand.cuh"   // the quantised cache's in-place expansion
 
-__device__ __forceinline__ void read_codes(const uint8_t* stage, int t, TileCodes& v) {
-  const int row = t >> 1, half = t & 1;
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int k = 0; k < 2; ++k)
-      v.c[i][k] = *reinterpret_cast<const uint4*>(stage + i * kBoxC + kBoxC / 2 + row * 64 + half * 32 + 16 * k);
-  v.r = *reinterpret_cast<const uint4*>(stage + 4 * kBoxC + kBoxR / 2 + row * 32 + half * 16);
-}
-
-// An E4M3 code as fp32 bits, exponent and mantissa fields moved 20 bits up and the sign to
-// bit 31: that fp32 is the code's value times 2^-120 for every finite code (the normal ones,
-// whose fp32 exponent field is theirs, and the subnormal ones and zero, which land on fp32
-// subnormals and zero). A multiply by 2^120 gives the code's value (normal, at most 448), a
-// second by 2^e the scaled value, both exactly, and the product's upper 16 bits are its bf16
-// (4 significant bits survive any power-of-two scale that keeps the value a normal bf16:
-// e in [-117, 118], far wider than a quantised row needs). No conversion instructions:
-// shifts, logic and two multiplies per value. (The NaN codes 0x7F and 0xFF, which the
-// quantiser never writes, read as 480.)
-__device__ __forceinline__ float e4m3_scaled(uint32_t byte_in_top, float scale) {
-  const uint32_t bits = (byte_in_top & 0x80000000u) | ((byte_in_top >> 4) & 0x07F00000u);
-  return __uint_as_float(bits) * 0x1p120f * scale;
-}
-
-// Four codes (one word, low byte first) -> two bf16 pairs, in order.
-__device__ __forceinline__ uint2 expand4(uint32_t w, float scale120) {
-  const float v0 = e4m3_scaled(w << 24, scale120), v1 = e4m3_scaled(w << 16, scale120);
-  const float v2 = e4m3_scaled(w << 8, scale120), v3 = e4m3_scaled(w, scale120);
-  return make_uint2(__byte_perm(__float_as_uint(v0), __float_as_uint(v1), 0x7632),
-                    __byte_perm(__float_as_uint(v2), __float_as_uint(v3), 0x7632));
-}
-
-__device__ __forceinline__ uint4 expand8(uint32_t lo4, uint32_t hi4, float scale120) {
-  const uint2 a = expand4(lo4, scale120), b = expand4(hi4, scale120);
-  return make_uint4(a.x, a.y, b.x, b.y);
-}
-
-__device__ __forceinline__ void write_bf16(uint8_t* stage, int t, const TileCodes& v, float scale120) {
-  const int row = t >> 1, half = t & 1;
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {   // 16-byte chunk half*4 + k of the row: 8 columns
-      const uint4 w = v.c[i][k >> 1];
-      const int chunk = half * 4 + k;
-      *reinterpret_cast<uint4*>(stage + i * kBoxC + row * 128 + ((chunk ^ (row & 7)) << 4)) =
-          (k & 1) ? expand8(w.z, w.w, scale120) : expand8(w.x, w.y, scale120);
-    }
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int chunk = half * 2 + k;
-    *reinterpret_cast<uint4*>(stage + 4 * kBoxC + row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4)) =
-        k ? expand8(v.r.z, v.r.w, scale120) : expand8(v.r.x, v.r.y, scale120);
-  }
-}
 
 // kQ8: the cache is quantised (E4M3 codes expanded in shared memory); a separate
 // instantiation, so that the bf16 kernel carries none of that code.
@@ -852,14 +793,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       const int64_t row0 = tile_row_s[st];
       const int64_t row = row0 + (t >> 1);
       const int e = (row0 >= 0 && row < p.kv_rows) ? (int)p.kv_exp[row] : 0;
-      const float scale120 = __uint_as_float((uint32_t)(min(max(e, -126), 127) + 127) << 23);   // 2^e
+      const float scale = __uint_as_float((uint32_t)(min(max(e, -126), 127) + 127) << 23);   // 2^e
       uint8_t* stage = smem + st * kStageBytes;
       TileCodes v;
       read_codes(stage, t, v);
       mbar_arrive(bar(kBarConvSync));
       if (!wait_bounded(bar(kBarConvSync), n_expanded & 1u, guard)) return false;
       ++n_expanded;
-      write_bf16(stage, t, v, scale120);
+      write_bf16(stage, t, v, scale);
       fence_proxy_async_smem();   // read by the MMAs (async proxy)
       mbar_arrive(bar(kBarKvConv + st));
       return true;

@@ -236,6 +236,20 @@ int mla_append_kv(mla_handle_t h, int32_t batch, int32_t d_model, const void* hi
                   int32_t num_pages, mla_stream_t stream);
 
 /*
+ * mla_append_kv into a quantised cache (the layout of mla_decode_attn_fp8): the new row's 576
+ * values, computed as above in fp32, get the smallest power-of-two scale 2^e with
+ * max|row| / 2^e <= 448 (e in -126..127, 0 for an all-zero row), and each value / 2^e is
+ * rounded to the nearest E4M3 code, ties to even (saturating at +-448). Codes go to
+ * kv_codes + r*row_stride (bytes; a multiple of 16, >= 576), e to kv_exp[r]. Other arguments
+ * and errors as for mla_append_kv.
+ */
+int mla_append_kv_fp8(mla_handle_t h, int32_t batch, int32_t d_model, const void* hidden,
+                      const void* w_dkv, const void* w_kr, const void* gamma, float rms_eps,
+                      void* kv_codes, int8_t* kv_exp, int64_t row_stride, int64_t seq_stride,
+                      const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                      int32_t num_pages, mla_stream_t stream);
+
+/*
  * mla_decode_attn for callers that cannot allocate device memory. The pages have no
  * counterpart to this call: it exists for library users whose device memory is owned by
  * someone else (a serving engine that has reserved nearly all of HBM for its own KV-cache

@@ -63,6 +63,8 @@ SIGNATURES = {
     "mla_absorb_q": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P, _P, _P]),
     "mla_decode_attn": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32, _P, _P, _P]),
     "mla_apply_wuv": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P]),
+    "mla_append_kv_fp8": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _P, _P, ctypes.c_float, _P, _P,
+                                         _I64, _I64, _P, _P, _I32, _I32, _P]),
     "mla_decode_attn_fp8": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32, _P, _P, _P]),
     "mla_decode_attn_partial": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32,
                                                _P, _P, _P]),
@@ -215,6 +217,33 @@ class MlaDecode:
             ctypes.c_void_p(c_kv), ctypes.c_void_p(k_r), row_stride, seq_stride, _ptr(kv_lens),
             _ptr(page_table), max_pages, num_pages, _stream(stream)), "mla_append_kv")
         return cache
+
+    def append_kv_fp8(self, hidden: torch.Tensor, w_dkv: torch.Tensor, w_kr: torch.Tensor,
+                      gamma: torch.Tensor, codes: torch.Tensor, exps: torch.Tensor,
+                      kv_lens: torch.Tensor, page_table: Optional[torch.Tensor] = None,
+                      eps: float = 1e-6, stream=None):
+        """append_kv into a quantised cache: codes uint8 [B, Lmax, 576] or [P, 64, 576], exps
+        int8 shaped like codes[..., 0] (the layout of decode_attn_fp8)."""
+        B, d = hidden.shape[0], hidden.shape[-1]
+        for t, n in ((hidden, "hidden"), (w_dkv, "w_dkv"), (w_kr, "w_kr"), (gamma, "gamma")):
+            _need(t, torch.bfloat16, n)
+        _need(kv_lens, torch.int32, "kv_lens")
+        if not codes.is_cuda or codes.dtype != torch.uint8 or codes.dim() != 3 or codes.stride(-1) != 1:
+            raise ValueError("codes: expected a CUDA uint8 [*, *, 576] tensor with unit inner stride")
+        _need(exps, torch.int8, "exps")
+        row_stride = codes.stride(1)
+        seq_stride = codes.stride(0) // row_stride
+        if exps.shape != codes.shape[:2] or exps.stride(0) != seq_stride:
+            raise ValueError("exps must index rows as codes does")
+        max_pages = num_pages = 0
+        if page_table is not None:
+            _need(page_table, torch.int32, "page_table")
+            max_pages, num_pages, seq_stride = page_table.shape[1], codes.shape[0], 0
+        _check(self._lib.mla_append_kv_fp8(
+            self._h, B, d, _ptr(hidden), _ptr(w_dkv), _ptr(w_kr), _ptr(gamma), float(eps),
+            _ptr(codes), _ptr(exps), row_stride, seq_stride, _ptr(kv_lens), _ptr(page_table),
+            max_pages, num_pages, _stream(stream)), "mla_append_kv_fp8")
+        return codes, exps
 
     @staticmethod
     def _cache_view(cache: torch.Tensor, page_table: Optional[torch.Tensor]):

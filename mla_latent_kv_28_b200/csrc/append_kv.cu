@@ -168,6 +168,8 @@ struct FinalParams {
   CacheView cv;
   __nv_bfloat16* c_kv;   // writable views of the cache rows
   __nv_bfloat16* k_r;
+  uint8_t* codes;        // quantised cache (else nullptr): E4M3 codes of row r at codes + r*row_stride
+  int8_t* kv_exp;        // ... and its scale exponent
   double theta[kDRope / 2];
   uint32_t* err;
 };
@@ -176,6 +178,7 @@ __global__ void __launch_bounds__(kRow)
 kv_finalize(const FinalParams p) {
   __shared__ float xs[kRow];
   __shared__ float red[kDLatent / 32];
+  __shared__ float red_max[kRow / 32];
   // block = one (sequence, new token) row: sequence blockIdx.x / q_len, token blockIdx.x % q_len
   const int bt = blockIdx.x, b = bt / p.q_len, f = threadIdx.x, warp = f >> 5, lane = f & 31;
   grid_dependency_wait();   // the partial sums of kv_down_tc
@@ -212,12 +215,13 @@ kv_finalize(const FinalParams p) {
   for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
   if (f < kDLatent && lane == 0) red[warp] = sq;
   __syncthreads();
+  double val;   // this thread's value of the row
   if (f < kDLatent) {
     float tot = 0.f;
 #pragma unroll
     for (int w = 0; w < kDLatent / 32; ++w) tot += red[w];
     const float y = x * rsqrtf(tot / kDLatent + p.eps) * __bfloat162float(p.gamma[f]);
-    p.c_kv[row * p.cv.row_stride + f] = __float2bfloat16_rn(y);
+    val = y;
   } else {
     // RoPE of the pair (2m, 2m+1) at the new token's position, angle reduced as in absorb
     constexpr double kTwoPiHi = 6.283185307179586;
@@ -234,8 +238,35 @@ kv_finalize(const FinalParams p) {
       sincos(r, &sn, &cs);
       y = (i & 1) ? x0 * sn + x1 * cs : x0 * cs - x1 * sn;
     }
-    p.k_r[row * p.cv.row_stride + i] = __double2bfloat16(y);
+    val = y;
   }
+  if (p.codes == nullptr) {   // bf16 row, one rounding from the computed value
+    if (f < kDLatent) p.c_kv[row * p.cv.row_stride + f] = __float2bfloat16_rn((float)val);
+    else p.k_r[row * p.cv.row_stride + (f - kDLatent)] = __double2bfloat16(val);
+    return;
+  }
+  // Quantised row: the smallest power-of-two scale 2^e with max|row| / 2^e <= 448, then each
+  // value / 2^e (exact) rounded to the nearest E4M3 code, ties to even.
+  float am = fabsf((float)val);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  if (lane == 0) red_max[warp] = am;
+  __syncthreads();
+  float amax = 0.f;
+#pragma unroll
+  for (int w = 0; w < kRow / 32; ++w) amax = fmaxf(amax, red_max[w]);
+  int e = 0;
+  if (amax > 0.f) {
+    e = (int)ceil(log2((double)amax / 448.0));
+    while ((double)amax * exp2(-(double)e) > 448.0) ++e;
+    while ((double)amax * exp2(-(double)(e - 1)) <= 448.0) --e;
+    e = min(max(e, -126), 127);
+  }
+  const float q = (float)(val * exp2(-(double)e));
+  uint32_t c2;
+  asm("{ .reg .b16 t; cvt.rn.satfinite.e4m3x2.f32 t, %1, %2; cvt.u32.u16 %0, t; }" : "=r"(c2) : "f"(0.f), "f"(q));
+  p.codes[row * p.cv.row_stride + f] = (uint8_t)(c2 & 0xFFu);
+  if (f == 0) p.kv_exp[row] = (int8_t)e;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encoder() {
@@ -319,6 +350,10 @@ cudaError_t launch_append_kv(const mla_decode_s& h, int batch, int d_model,
   fp.cv = cv;
   fp.c_kv = c_kv;
   fp.k_r = k_r;
+  if (cv.kv_exp != nullptr) {   // quantised cache: c_kv is the codes' base
+    fp.codes = reinterpret_cast<uint8_t*>(c_kv);
+    fp.kv_exp = const_cast<int8_t*>(cv.kv_exp);
+  }
   for (int m = 0; m < kDRope / 2; ++m)
     fp.theta[m] = h.theta[m];
   fp.err = h.ws.err;

@@ -296,11 +296,15 @@ int mla_merge_partials(mla_handle_t h, int32_t batch, int32_t n_parts, const flo
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
-int mla_append_kv(mla_handle_t h, int32_t batch, int32_t d_model, const void* hidden,
-                  const void* w_dkv, const void* w_kr, const void* gamma, float rms_eps,
-                  void* c_kv, void* k_r, int64_t row_stride, int64_t seq_stride,
-                  const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
-                  int32_t num_pages, mla_stream_t stream) {
+namespace {
+
+// The shared body of mla_append_kv (bf16 rows) and mla_append_kv_fp8 (kv_exp != nullptr:
+// E4M3 codes at c_kv, row_stride in bytes).
+int append_kv_common(mla_handle_t h, int32_t batch, int32_t d_model, const void* hidden,
+                     const void* w_dkv, const void* w_kr, const void* gamma, float rms_eps,
+                     void* c_kv, void* k_r, int8_t* kv_exp, int64_t row_stride, int64_t seq_stride,
+                     const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                     int32_t num_pages, mla_stream_t stream) {
   if (h == nullptr || hidden == nullptr || w_dkv == nullptr || w_kr == nullptr ||
       gamma == nullptr || c_kv == nullptr || k_r == nullptr || kv_lens == nullptr)
     return MLA_ERR_INVALID_ARG;
@@ -311,12 +315,15 @@ int mla_append_kv(mla_handle_t h, int32_t batch, int32_t d_model, const void* hi
   if (!aligned16(hidden) || !aligned16(w_dkv) || !aligned16(w_kr) || !aligned16(gamma) ||
       !aligned16(c_kv) || !aligned16(k_r))
     return MLA_ERR_INVALID_ARG;
-  if (row_stride < kDLatent || row_stride % 8 != 0) return MLA_ERR_INVALID_ARG;
+  if (kv_exp == nullptr ? (row_stride < kDLatent || row_stride % 8 != 0)
+                        : (row_stride < mla::kRow || row_stride % 16 != 0))
+    return MLA_ERR_INVALID_ARG;
   mla::CacheView cv{};
   cv.c_kv = static_cast<const __nv_bfloat16*>(c_kv);
   cv.k_r = static_cast<const __nv_bfloat16*>(k_r);
   cv.row_stride = row_stride;
   cv.page_size = h->cfg.page_size;
+  cv.kv_exp = kv_exp;
   if (h->cfg.page_size == 0) {
     if (page_table != nullptr || seq_stride < h->cfg.max_kv_len) return MLA_ERR_INVALID_ARG;
     cv.seq_stride = seq_stride;
@@ -333,6 +340,28 @@ int mla_append_kv(mla_handle_t h, int32_t batch, int32_t d_model, const void* hi
       static_cast<const __nv_bfloat16*>(gamma), rms_eps, cv, static_cast<__nv_bfloat16*>(c_kv),
       static_cast<__nv_bfloat16*>(k_r), kv_lens, stream);
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace
+
+int mla_append_kv(mla_handle_t h, int32_t batch, int32_t d_model, const void* hidden,
+                  const void* w_dkv, const void* w_kr, const void* gamma, float rms_eps,
+                  void* c_kv, void* k_r, int64_t row_stride, int64_t seq_stride,
+                  const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                  int32_t num_pages, mla_stream_t stream) {
+  return append_kv_common(h, batch, d_model, hidden, w_dkv, w_kr, gamma, rms_eps, c_kv, k_r, nullptr,
+                          row_stride, seq_stride, kv_lens, page_table, max_pages, num_pages, stream);
+}
+
+int mla_append_kv_fp8(mla_handle_t h, int32_t batch, int32_t d_model, const void* hidden,
+                      const void* w_dkv, const void* w_kr, const void* gamma, float rms_eps,
+                      void* kv_codes, int8_t* kv_exp, int64_t row_stride, int64_t seq_stride,
+                      const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                      int32_t num_pages, mla_stream_t stream) {
+  if (kv_exp == nullptr) return MLA_ERR_INVALID_ARG;
+  return append_kv_common(h, batch, d_model, hidden, w_dkv, w_kr, gamma, rms_eps, kv_codes,
+                          kv_codes, kv_exp, row_stride, seq_stride, kv_lens, page_table, max_pages,
+                          num_pages, stream);
 }
 
 int mla_apply_wuv(mla_handle_t h, int32_t batch, const void* latent, const void* w_uv,

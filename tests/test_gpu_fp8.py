@@ -93,3 +93,50 @@ def test_argument_errors():
     with pytest.raises(binding.MlaError, match="INVALID_ARG"):   # a row pitch that is not 16-byte
         wide = torch.zeros((1, 64, 584), dtype=torch.uint8, device=DEV)[..., :576]
         h.decode_attn_fp8(qa, wide, torch.zeros((1, 64), dtype=torch.int8, device=DEV), lens)
+
+
+@pytest.mark.parametrize("page_size", [0, 64])
+def test_cache_write_into_the_quantised_cache(page_size):
+    """mla_append_kv_fp8: the new rows' exponents are the oracle's, their codes dequantise to
+    within half a step of the oracle's rows, no other row changes, and the decode over the
+    quantised cache then matches the oracle over the dequantised rows."""
+    lens = [5, 64, 130]
+    w = wl.make_workload(3, 32, lens, page_size=page_size, seed=100, max_kv_len=192)
+    g = w.to(DEV)
+    codes, exps, _, deq64 = _quantise(w.cache)
+    codes, exps = codes.to(DEV), exps.to(DEV)
+    before_c, before_e = codes.clone(), exps.clone()
+    inp = wl.draw_append_inputs(3, 1024, seed=101)
+    h = binding.MlaDecode(32, 3, w.max_kv_len, page_size=page_size)
+    dev = {k: v.to(DEV) for k, v in inp.items()}
+    h.append_kv_fp8(dev["hidden"], dev["w_dkv"], dev["w_kr"], dev["gamma"], codes, exps, g.kv_lens,
+                    g.page_table)
+    h.check_device_errors()
+    ref = oracle.cache_rows(to_np(inp["hidden"]), to_np(inp["w_dkv"]), to_np(inp["w_kr"]),
+                            to_np(inp["gamma"]), lens, w.rope_base)
+
+    def at(b):
+        pos = lens[b] - 1
+        if w.page_table is None:
+            return b, pos
+        return int(w.page_table[b, pos // 64]), pos % 64
+
+    mask = torch.ones(codes.shape[:2], dtype=torch.bool, device=DEV)
+    for b in range(3):
+        i, j = at(b)
+        mask[i, j] = False
+        e = int(exps[i, j])
+        assert e == oracle.fp8_row_exponent(ref[b]), b
+        got = oracle.dequantize_rows_fp8(codes[i, j].cpu().numpy()[None], np.array([e]))[0]
+        step = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ref[b]) / 2.0 ** e, 2.0 ** -6))) - 3) * 2.0 ** e
+        assert np.all(np.abs(got - ref[b]) <= step / 2 + 1e-6 * np.abs(ref[b]).max()), b
+        deq64[i, j] = got
+    assert torch.equal(codes[mask], before_c[mask]) and torch.equal(exps[mask], before_e[mask])
+    qa = wl.draw_q_abs(3, 32, seed=102)
+    lat, lse = h.decode_attn_fp8(qa.to(DEV), codes, exps, g.kv_lens, g.page_table)
+    h.check_device_errors()
+    a = workload_np(w)
+    ref_lat, ref_lse = oracle.latent_attention(to_np(qa), deq64, a["kv_lens"], oracle.default_scale(),
+                                               a["page_table"], a["page_size"])
+    assert_close(f64(lat), ref_lat, "decode after the quantised cache write: latent")
+    assert_close(lse.cpu().numpy(), ref_lse, "decode after the quantised cache write: lse")

@@ -101,7 +101,8 @@ def test_cache_write_into_the_quantised_cache(page_size):
     within half a step of the oracle's rows, no other row changes, and the decode over the
     quantised cache then matches the oracle over the dequantised rows."""
     lens = [5, 64, 130]
-    w = wl.make_workload(3, 32, lens, page_size=page_size, seed=100, max_kv_len=192)
+    w = wl.make_workload(3, 32, lens, page_size=page_size, seed=100,
+                         max_kv_len=192 if page_size else None)
     g = w.to(DEV)
     codes, exps, _, deq64 = _quantise(w.cache)
     codes, exps = codes.to(DEV), exps.to(DEV)

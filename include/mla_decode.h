@@ -82,8 +82,9 @@ typedef struct {
    * lse [batch, T, n_h], latent/out of mla_apply_wuv, hidden [batch, T, d] of
    * mla_append_kv); kv_lens counts the T new tokens, which sit at positions kv_len - T + t;
    * token t attends to rows 0 .. kv_len - T + t (a token with none: latent 0, lse -inf) and
-   * its q^R is rotated at max(kv_len - T + t, 0). Limits: n_heads * T <= 128 and
-   * max_batch * T <= 1024. */
+   * its q^R is rotated at max(kv_len - T + t, 0). Limits: n_heads * T <= 1024 and
+   * max_batch * T <= 1024; mla_decode_attn runs more than 128 attention rows per sequence in
+   * groups of 128, each reading the cache. */
   int32_t q_len;
 } mla_config_t;
 

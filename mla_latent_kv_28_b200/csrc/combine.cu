@@ -12,6 +12,7 @@
 //   many splits (QG = 1): the slots are dealt round-robin to SL threads per (head, quad),
 //   which meet in shared memory for the max, the weights and the sums, so a single long
 //   sequence split ~70 ways still has thousands of loads in flight.
+#include <algorithm>
 #include <type_traits>
 
 #include "mla_internal.cuh"
@@ -28,7 +29,9 @@ template <int QG, typename OutT>
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(PlanView plan, int n_heads, int slot_lanes, int groups_per_block,
                const float* __restrict__ part_o, const float* __restrict__ part_lse,
-               OutT* __restrict__ out_latent, float* __restrict__ lse_out) {
+               OutT* __restrict__ out_latent, float* __restrict__ lse_out, int row_base, int out_rows) {
+  // n_heads: the rows of the partials (one launch's group); out_rows: rows per sequence of the
+  // outputs, of which this launch writes [row_base, row_base + n_heads)
   constexpr int kGroups = kQuads / QG;
   __shared__ float s_m[kThreads];
   __shared__ float4 s_acc[kThreads][QG];
@@ -99,13 +102,13 @@ combine_kernel(PlanView plan, int n_heads, int slot_lanes, int groups_per_block,
   if (!work || sl != 0) return;
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
   if constexpr (std::is_same<OutT, float>::value) {
-    float* dst = out_latent + ((int64_t)b * n_heads + h) * kDLatent + grp * 4 * QG;
+    float* dst = out_latent + ((int64_t)b * out_rows + row_base + h) * kDLatent + grp * 4 * QG;
 #pragma unroll
     for (int q = 0; q < QG; ++q)
       reinterpret_cast<float4*>(dst)[q] =
           make_float4(acc[q].x * inv, acc[q].y * inv, acc[q].z * inv, acc[q].w * inv);
     if (lse_out != nullptr && grp == 0)
-      lse_out[(int64_t)b * n_heads + h] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
+      lse_out[(int64_t)b * out_rows + row_base + h] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
     return;
   }
   uint32_t packed[2 * QG];
@@ -116,7 +119,7 @@ combine_kernel(PlanView plan, int n_heads, int slot_lanes, int groups_per_block,
     packed[2 * q] = *reinterpret_cast<uint32_t*>(&lo);
     packed[2 * q + 1] = *reinterpret_cast<uint32_t*>(&hi);
   }
-  __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(out_latent) + ((int64_t)b * n_heads + h) * kDLatent + grp * 4 * QG;
+  __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(out_latent) + ((int64_t)b * out_rows + row_base + h) * kDLatent + grp * 4 * QG;
   if (QG == 4) {
     reinterpret_cast<uint4*>(dst)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     reinterpret_cast<uint4*>(dst)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
@@ -126,15 +129,15 @@ combine_kernel(PlanView plan, int n_heads, int slot_lanes, int groups_per_block,
       reinterpret_cast<uint2*>(dst)[q] = make_uint2(packed[2 * q], packed[2 * q + 1]);
   }
   if (lse_out != nullptr && grp == 0)
-    lse_out[(int64_t)b * n_heads + h] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
+    lse_out[(int64_t)b * out_rows + row_base + h] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
 }
 
 }  // namespace
 
 template <typename OutT>
 cudaError_t launch_combine_t(const mla_decode_s& h, int batch, OutT* out_latent, float* lse,
-                             cudaStream_t s) {
-  const int n_heads = h.n_rows;   // attention rows per sequence (heads x new tokens)
+                             int row_base, cudaStream_t s) {
+  const int n_heads = std::min(h.group_rows, h.n_rows - row_base);   // this group's rows
   const int per_block = n_heads >= kThreads ? 1 : kThreads / n_heads;   // head rows per block
   // the most slots one sequence can have: balanced units overlap about units / batch + 1 of a
   // sequence's tiles; capped plans give at most max_splits
@@ -144,21 +147,21 @@ cudaError_t launch_combine_t(const mla_decode_s& h, int batch, OutT* out_latent,
     const int bps = (kG + per_block - 1) / per_block;
     return launch_pdl(combine_kernel<4, OutT>, dim3(batch * bps), dim3(kThreads), 0, s, h.ws.plan, n_heads,
                       1, per_block, (const float*)h.ws.part_o, (const float*)h.ws.part_lse,
-                      out_latent, lse);
+                      out_latent, lse, row_base, h.n_rows);
   }
   return launch_pdl(combine_kernel<1, OutT>, dim3(batch * kQuads), dim3(kThreads), 0, s, h.ws.plan, n_heads,
                     per_block, 1, (const float*)h.ws.part_o, (const float*)h.ws.part_lse, out_latent,
-                    lse);
+                    lse, row_base, h.n_rows);
 }
 
 cudaError_t launch_combine(const mla_decode_s& h, int batch, __nv_bfloat16* out_latent,
-                           float* lse, cudaStream_t s) {
-  return launch_combine_t(h, batch, out_latent, lse, s);
+                           float* lse, int row_base, cudaStream_t s) {
+  return launch_combine_t(h, batch, out_latent, lse, row_base, s);
 }
 
 cudaError_t launch_combine_f32(const mla_decode_s& h, int batch, float* out_latent, float* lse,
-                               cudaStream_t s) {
-  return launch_combine_t(h, batch, out_latent, lse, s);
+                               int row_base, cudaStream_t s) {
+  return launch_combine_t(h, batch, out_latent, lse, row_base, s);
 }
 
 }  // namespace mla

@@ -128,6 +128,7 @@ extern "C" int mla_decode_attn_noalloc(int32_t n_heads, float softmax_scale, int
   h.cfg.n_heads = n_heads;
   h.q_len = 1;
   h.n_rows = n_heads;
+  h.group_rows = n_heads;
   h.cfg.d_head = kDHead;
   h.cfg.d_latent = kDLatent;
   h.cfg.d_rope = kDRope;
@@ -169,8 +170,8 @@ extern "C" int mla_decode_attn_noalloc(int32_t n_heads, float softmax_scale, int
   if (cudaMemsetAsync(h.ws.err, 0, sizeof(uint32_t), stream) != cudaSuccess) return MLA_ERR_CUDA;
   cudaError_t e = launch_split_plan(h, batch, kv_lens, stream);
   if (e == cudaSuccess)
-    e = launch_decode_split(h, batch, static_cast<const __nv_bfloat16*>(q_abs), cv, stream);
+    e = launch_decode_split(h, batch, static_cast<const __nv_bfloat16*>(q_abs), cv, 0, stream);
   if (e == cudaSuccess)
-    e = launch_combine(h, batch, static_cast<__nv_bfloat16*>(out_latent), lse, stream);
+    e = launch_combine(h, batch, static_cast<__nv_bfloat16*>(out_latent), lse, 0, stream);
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }

@@ -132,6 +132,7 @@ struct Params {
   PlanView plan;
   int batch, n_heads;      // n_heads: attention rows per sequence, token-major (heads x new tokens)
   int q_len, heads_per_token;   // new tokens per sequence; row r is token r / heads_per_token
+  int row_base, q_row_stride;   // this launch's rows: [row_base, row_base + n_heads) of q_row_stride
   int64_t seq_stride;
   const int32_t* page_table;
   int max_pages, num_pages;
@@ -237,7 +238,7 @@ __device__ __forceinline__ void q_chunks_out(const uint4 (&v)[12], uint8_t* smem
 __device__ __forceinline__ void load_q_part(const Params& p, uint8_t* smem, uint32_t tmem, uint32_t lanes,
                                             int h, int b, int part, uint32_t rank) {
   const bool head_ok = h < p.n_heads;
-  const __nv_bfloat16* qrow = p.q_abs + ((int64_t)b * p.n_heads + (head_ok ? h : 0)) * kRow;
+  const __nv_bfloat16* qrow = p.q_abs + ((int64_t)b * p.q_row_stride + p.row_base + (head_ok ? h : 0)) * kRow;
   uint4 v[12];
 #pragma unroll
   for (int i = 0; i < 12; ++i) {
@@ -359,7 +360,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       TileCursor c;
       c.init(p);
       if (c.valid) {   // the first segment's query columns: one request, ahead of the tiles
-        const int qrow = c.b * p.n_heads;
+        const int qrow = c.b * p.q_row_stride + p.row_base;
         const uint32_t qdst = sbase + kStageBytes;
         mbar_arrive_expect_tx(bar(kBarQLanded), kQBytes);
         for (int i = 0; i < 4; ++i)
@@ -566,7 +567,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
         const int r = tile_valid[st] ? c.rows() : 0;   // valid tokens of the tile
         // ... of which this row sees those up to its own token's position: new token t of
         // q_len sits at len - q_len + t and does not see the new tokens after it
-        const int rr = max(0, min(r, c.len - (p.q_len - 1 - h / p.heads_per_token) - c.j()));
+        const int rr = max(0, min(r, c.len - (p.q_len - 1 - (p.row_base + h) / p.heads_per_token) - c.j()));
         // own partial S out of TMEM (S is free for the next QK once we have it)
         float sv[kT];
         {
@@ -849,7 +850,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       prev_slot = seg_slot;
       if (!ok) break;
       if (c.valid && head_ok) {
-        const __nv_bfloat16* qrow = p.q_abs + ((int64_t)c.b * p.n_heads + h) * kRow;
+        const __nv_bfloat16* qrow = p.q_abs + ((int64_t)c.b * p.q_row_stride + p.row_base + h) * kRow;
         asm volatile("prefetch.global.L2 [%0];" :: "l"(qrow + 256 * (int)rank) : "memory");
         asm volatile("prefetch.global.L2 [%0];" :: "l"(qrow + 256 * (int)rank + 64) : "memory");
         asm volatile("prefetch.global.L2 [%0];" :: "l"(qrow + 256 * (int)rank + 128) : "memory");
@@ -926,7 +927,7 @@ bool encode_codes(CUtensorMap* m, const void* base, uint64_t rows, int64_t row_s
 }  // namespace
 
 cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfloat16* q_abs,
-                                const CacheView& cv, cudaStream_t s) {
+                                const CacheView& cv, int row_base, cudaStream_t s) {
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
@@ -958,7 +959,9 @@ cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfl
   p.q_abs = q_abs;
   p.plan = h.ws.plan;
   p.batch = batch;
-  p.n_heads = h.n_rows;
+  p.n_heads = std::min(h.group_rows, h.n_rows - row_base);
+  p.row_base = row_base;
+  p.q_row_stride = h.n_rows;
   p.q_len = h.q_len;
   p.heads_per_token = h.cfg.n_heads;
   p.seq_stride = cv.seq_stride;

@@ -1,6 +1,7 @@
 // The C ABI of libmla_decode.so: argument checks, the workspace, and the launches.
 // Every compute call validates on the host, then enqueues kernels on the caller's stream;
 // nothing here allocates after mla_decode_create.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <new>
@@ -34,7 +35,7 @@ int config_status(const mla_config_t* c) {
   if (c->q_len < 0) return MLA_ERR_INVALID_ARG;
   {
     const int64_t T = c->q_len > 1 ? c->q_len : 1;
-    if ((int64_t)c->n_heads * T > mla::kMaxHeads || (int64_t)c->max_batch * T > mla::kMaxBatch)
+    if ((int64_t)c->n_heads * T > mla::kMaxRows || (int64_t)c->max_batch * T > mla::kMaxBatch)
       return MLA_ERR_UNSUPPORTED;
   }
   if (!(c->yarn_factor >= 0.f) || !std::isfinite(c->yarn_factor) ||
@@ -108,6 +109,7 @@ int mla_decode_create(const mla_config_t* cfg, int device, mla_handle_t* out) {
   rope_frequencies(*cfg, h->theta);
   h->q_len = cfg->q_len > 1 ? cfg->q_len : 1;
   h->n_rows = cfg->n_heads * h->q_len;
+  h->group_rows = std::min(h->n_rows, mla::kMaxHeads);
   h->units = sms / 2;  // the decode kernel runs one 2-CTA cluster per unit of work
 
   const int B = cfg->max_batch;
@@ -122,8 +124,8 @@ int mla_decode_create(const mla_config_t* cfg, int device, mla_handle_t* out) {
   const size_t o_seq_unit = off;  off = round_up(off + 4 * B, 256);
   const size_t o_ubegin = off;    off = round_up(off + 4 * (max_units + 1), 256);
   const size_t o_useq = off;      off = round_up(off + 4 * max_units, 256);
-  const size_t o_plse = off;      off = round_up(off + 4 * (size_t)max_slots * h->n_rows, 256);
-  const size_t o_po = off;        off = round_up(off + 4 * (size_t)max_slots * h->n_rows * kDLatent, 256);
+  const size_t o_plse = off;      off = round_up(off + 4 * (size_t)max_slots * h->group_rows, 256);
+  const size_t o_po = off;        off = round_up(off + 4 * (size_t)max_slots * h->group_rows * kDLatent, 256);
   const size_t o_ap = off;        off = round_up(off + 4 * (size_t)mla::kAppendSlices * B * h->q_len * mla::kRow, 256);
 
   void* base = nullptr;
@@ -216,11 +218,14 @@ int decode_attn_common(mla_handle_t h, int32_t batch, const void* q_abs, const v
     cv.num_pages = num_pages;
   }
   cudaError_t e = mla::launch_split_plan(*h, batch, kv_lens, stream);
-  if (e == cudaSuccess)
-    e = mla::launch_decode_split(*h, batch, static_cast<const __nv_bfloat16*>(q_abs), cv, stream);
-  if (e == cudaSuccess)
-    e = out_f32 ? mla::launch_combine_f32(*h, batch, static_cast<float*>(out_latent), lse, stream)
-                : mla::launch_combine(*h, batch, static_cast<__nv_bfloat16*>(out_latent), lse, stream);
+  // more than 128 attention rows per sequence (several new tokens): one decode + combine per
+  // group of 128 rows, each over the same cache and plan
+  for (int rb = 0; e == cudaSuccess && rb < h->n_rows; rb += h->group_rows) {
+    e = mla::launch_decode_split(*h, batch, static_cast<const __nv_bfloat16*>(q_abs), cv, rb, stream);
+    if (e == cudaSuccess)
+      e = out_f32 ? mla::launch_combine_f32(*h, batch, static_cast<float*>(out_latent), lse, rb, stream)
+                  : mla::launch_combine(*h, batch, static_cast<__nv_bfloat16*>(out_latent), lse, rb, stream);
+  }
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -263,10 +268,11 @@ int mla_decode_attn_fp8(mla_handle_t h, int32_t batch, const void* q_abs, const 
     cv.num_pages = num_pages;
   }
   cudaError_t e = mla::launch_split_plan(*h, batch, kv_lens, stream);
-  if (e == cudaSuccess)
-    e = mla::launch_decode_split(*h, batch, static_cast<const __nv_bfloat16*>(q_abs), cv, stream);
-  if (e == cudaSuccess)
-    e = mla::launch_combine(*h, batch, static_cast<__nv_bfloat16*>(out_latent), lse, stream);
+  for (int rb = 0; e == cudaSuccess && rb < h->n_rows; rb += h->group_rows) {
+    e = mla::launch_decode_split(*h, batch, static_cast<const __nv_bfloat16*>(q_abs), cv, rb, stream);
+    if (e == cudaSuccess)
+      e = mla::launch_combine(*h, batch, static_cast<__nv_bfloat16*>(out_latent), lse, rb, stream);
+  }
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

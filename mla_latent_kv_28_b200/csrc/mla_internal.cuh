@@ -16,6 +16,7 @@ constexpr int kDLatent = 512;  // d_c
 constexpr int kDRope = 64;     // d_h^R
 constexpr int kRow = kDLatent + kDRope;  // one cache row: [c^KV ; k^R]
 constexpr int kMaxHeads = 128;
+constexpr int kMaxRows = 1024;   // attention rows per sequence (heads x new tokens), in groups of 128
 constexpr int kMaxBatch = 1024;
 constexpr int kTileTokens = 64;  // tokens per KV tile: the unit of the work plan
 constexpr int kAppendSlices = 16;  // the cache write's projection is split over at most 16 slices of d
@@ -63,6 +64,7 @@ struct mla_decode_s {
   float scale = 0.f;
   int q_len = 1;    // new tokens per sequence per call
   int n_rows = 0;   // attention rows per sequence: n_heads * q_len (token-major)
+  int group_rows = 0;   // rows per decode launch (the MMA's M = 128 at most); n_rows in groups
   double theta[mla::kDRope / 2] = {};  // RoPE pair frequencies (0: no rotation), YaRN applied
   int units = 0;  // units the balanced plan cuts the tile space into
   mla::Workspace ws;
@@ -121,14 +123,16 @@ struct CacheView {
   const int8_t* kv_exp = nullptr;
 };
 
+// row_base: the first of the (at most group_rows) attention rows of each sequence this launch
+// takes; the partials it writes hold just those rows.
 cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfloat16* q_abs,
-                                const CacheView& cache, cudaStream_t s);
+                                const CacheView& cache, int row_base, cudaStream_t s);
 
 cudaError_t launch_combine(const mla_decode_s& h, int batch, __nv_bfloat16* out_latent,
-                           float* lse, cudaStream_t s);
+                           float* lse, int row_base, cudaStream_t s);
 
 cudaError_t launch_combine_f32(const mla_decode_s& h, int batch, float* out_latent, float* lse,
-                               cudaStream_t s);
+                               int row_base, cudaStream_t s);
 
 cudaError_t launch_merge_parts(const mla_decode_s& h, int batch, int n_parts, const float* latent_parts,
                                const float* lse_parts, __nv_bfloat16* out_latent, float* lse_out,

@@ -69,8 +69,8 @@ def test_config_checks(lib):
          binding.MLA_ERR_INVALID_ARG),
         (binding.make_config(8, 1, 1, yarn_factor=40.0, yarn_mscale_coef=-0.1), binding.MLA_ERR_INVALID_ARG),
         (binding.make_config(8, 1, 1, yarn_factor=40.0, yarn_original_len=0), binding.MLA_ERR_INVALID_ARG),
-        # several new tokens: at most 128 attention rows and 1024 (sequence, token) rows
-        (binding.make_config(128, 1, 16, q_len=2), binding.MLA_ERR_UNSUPPORTED),
+        # several new tokens: at most 1024 attention rows and 1024 (sequence, token) rows
+        (binding.make_config(128, 1, 16, q_len=9), binding.MLA_ERR_UNSUPPORTED),
         (binding.make_config(16, 512, 16, q_len=4), binding.MLA_ERR_UNSUPPORTED),
         (binding.make_config(16, 1, 16, q_len=-1), binding.MLA_ERR_INVALID_ARG),
     ]

@@ -49,6 +49,17 @@ def test_eight_tokens_sixteen_heads_contiguous():
     _step_vs_oracle(16, 8, [8, 100, 700, 3], 0, 70)
 
 
+def test_two_tokens_all_128_heads_in_two_row_groups():
+    """DeepSeek-V2's 128 heads with 2 new tokens: 256 attention rows, run as two groups of 128
+    over the same cache and plan."""
+    _step_vs_oracle(128, 2, [300, 64, 1000], 0, 76)
+
+
+def test_five_tokens_64_heads_uneven_groups():
+    """320 rows: groups of 128, 128 and 64, on a paged cache."""
+    _step_vs_oracle(64, 5, [5, 129, 700], 64, 77, max_kv_len=700)
+
+
 def test_two_tokens_paged_ragged():
     _step_vs_oracle(32, 2, [int(x) for x in np.random.default_rng(71).integers(1, 500, 20)], 64, 72,
                     max_kv_len=500)

@@ -269,6 +269,26 @@ __device__ __forceinline__ void q_part_from_smem(uint8_t* smem, uint32_t tmem, u
 #include "e4m3_expand.cuh"   // the quantised cache's in-place expansion
 
 
+// Rare paths of the softmax loop, kept out of line so that the loop's code stays small.
+__device__ __noinline__ void rescale_o(uint32_t taddr, float alpha) {
+#pragma unroll 1
+  for (int cc = 0; cc < 8; ++cc) {
+    uint32_t o[32];
+    tmem_ld32_sync(taddr + kTmemO + 32 * cc, o);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+    tmem_st32(taddr + kTmemO + 32 * cc, o);
+  }
+}
+
+__device__ __noinline__ void zero_tail(uint8_t* stage, int r, int tid) {
+  for (int i = tid; i < (kT - r) * 32; i += 128) {
+    const int row = r + (i >> 5), box = (i >> 3) & 3, chunk = i & 7;
+    *reinterpret_cast<uint4*>(stage + box * kBoxC + row * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async_smem();
+}
+
 // kQ8: the cache is quantised (E4M3 codes expanded in shared memory); a separate
 // instantiation, so that the bf16 kernel carries none of that code.
 template <bool kQ8>
@@ -673,17 +693,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
         if (g > 1 && !wait_spin(bar(kBarPvDone + ((g - 2) & 3u)), ((g - 2) >> 2) & 1u, guard)) break;
         if (warp_need && g > 0 && !wait_spin(bar(kBarPvDone + ((g - 1) & 3u)), ((g - 1) >> 2) & 1u, guard)) break;
         tc_fence_after();
-        if (warp_need) {   // O (all 256 columns of this head) to the new max
-#pragma unroll 1
-          for (int cc = 0; cc < 8; ++cc) {
-            uint32_t o[32];
-            const uint32_t col = kTmemO + 32 * cc;
-            tmem_ld32_sync(lanes | (tmem + col), o);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-            tmem_st32(lanes | (tmem + col), o);
-          }
-        }
+        if (warp_need) rescale_o(lanes | tmem, alpha);   // O (all 256 columns of this head) to the new max
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {   // P as bf16 pairs, 32 columns
           uint32_t pk[16];
@@ -695,15 +705,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
           tmem_st16(lanes | (tmem + kTmemP + (kT / 2) * wg + 16 * hf), pk);
         }
         tmem_wait_st();
-        if (r < kT) {
-          // rows past the sequence end (or of a skipped page) must not reach P.V as NaN/Inf
-          uint8_t* stage = smem + st * kStageBytes;
-          for (int i = tid; i < (kT - r) * 32; i += 128) {
-            const int row = r + (i >> 5), box = (i >> 3) & 3, chunk = i & 7;
-            *reinterpret_cast<uint4*>(stage + box * kBoxC + row * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
-          }
-          fence_proxy_async_smem();
-        }
+        if (r < kT) zero_tail(smem + st * kStageBytes, r, tid);   // rows past the end must not reach P.V
         tc_fence_before();
         mbar_arrive(bar(kBarPFull + wg));
       }

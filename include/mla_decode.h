@@ -35,6 +35,14 @@
 
 #include <stdint.h>
 
+/* Only the functions below are exported from libmla_decode.so (it is built with hidden
+ * visibility for everything else). */
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -92,17 +100,17 @@ typedef struct {
  * Check a configuration without touching any GPU: MLA_OK if mla_decode_create would accept
  * it, else the status it would return (MLA_ERR_INVALID_ARG / MLA_ERR_UNSUPPORTED).
  */
-int mla_check_config(const mla_config_t* cfg);
+MLA_API int mla_check_config(const mla_config_t* cfg);
 
 /*
  * Create a handle on CUDA device `device` and allocate its workspace there (sized from
  * cfg->max_batch, cfg->max_kv_len and n_heads). On success *out is the handle and the
  * return is MLA_OK; on failure *out is NULL. Makes `device` current on the calling thread.
  */
-int mla_decode_create(const mla_config_t* cfg, int device, mla_handle_t* out);
+MLA_API int mla_decode_create(const mla_config_t* cfg, int device, mla_handle_t* out);
 
 /* Free the workspace and the handle. Synchronises the device first. NULL is a no-op. */
-int mla_destroy(mla_handle_t h);
+MLA_API int mla_destroy(mla_handle_t h);
 
 /*
  * Query absorption and RoPE ([V2-walk] §2.3 displayed equation: q^T W_UK c = (W_UK^T q)^T c;
@@ -119,7 +127,7 @@ int mla_destroy(mla_handle_t h);
  * q_abs bf16 [batch, n_h, 576]  output
  * Errors: MLA_ERR_INVALID_ARG for NULL pointers or batch outside 1..max_batch.
  */
-int mla_absorb_q(mla_handle_t h, int32_t batch, const void* q_c, const void* q_r,
+MLA_API int mla_absorb_q(mla_handle_t h, int32_t batch, const void* q_c, const void* q_r,
                  const void* w_uk, const int32_t* kv_lens, void* q_abs, mla_stream_t stream);
 
 /*
@@ -147,7 +155,7 @@ int mla_absorb_q(mla_handle_t h, int32_t batch, const void* q_c, const void* q_r
  * given to a contiguous handle (or missing for a paged one), max_pages too small for
  * max_kv_len.
  */
-int mla_decode_attn(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
+MLA_API int mla_decode_attn(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
                     const void* k_r, int64_t row_stride, int64_t seq_stride,
                     const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
                     int32_t num_pages, void* out_latent, float* lse, mla_stream_t stream);
@@ -162,7 +170,7 @@ int mla_decode_attn(mla_handle_t h, int32_t batch, const void* q_abs, const void
  * are exact in bf16). kv_exp int8, one per row; row_stride a multiple of 16, >= 576. Outputs,
  * kv_lens, page table and errors as for mla_decode_attn.
  */
-int mla_decode_attn_fp8(mla_handle_t h, int32_t batch, const void* q_abs, const void* kv_codes,
+MLA_API int mla_decode_attn_fp8(mla_handle_t h, int32_t batch, const void* q_abs, const void* kv_codes,
                         const int8_t* kv_exp, int64_t row_stride, int64_t seq_stride,
                         const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
                         int32_t num_pages, void* out_latent, float* lse, mla_stream_t stream);
@@ -177,7 +185,7 @@ int mla_decode_attn_fp8(mla_handle_t h, int32_t batch, const void* q_abs, const 
  * log-sum-exp merge across GPUs is this library's. MLA_ERR_UNSUPPORTED with q_len > 1 (the
  * causal limits of several new tokens follow their global positions).
  */
-int mla_decode_attn_partial(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
+MLA_API int mla_decode_attn_partial(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
                             const void* k_r, int64_t row_stride, int64_t seq_stride,
                             const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
                             int32_t num_pages, float* out_latent, float* lse, mla_stream_t stream);
@@ -194,7 +202,7 @@ int mla_decode_attn_partial(mla_handle_t h, int32_t batch, const void* q_abs, co
  * Errors: MLA_ERR_INVALID_ARG for NULL pointers, batch outside 1..max_batch, n_parts < 1,
  * misalignment.
  */
-int mla_merge_partials(mla_handle_t h, int32_t batch, int32_t n_parts, const float* latent_parts,
+MLA_API int mla_merge_partials(mla_handle_t h, int32_t batch, int32_t n_parts, const float* latent_parts,
                        const float* lse_parts, void* out_latent, float* lse, mla_stream_t stream);
 
 /*
@@ -202,7 +210,7 @@ int mla_merge_partials(mla_handle_t h, int32_t batch, int32_t n_parts, const flo
  *   out[b,i,:] = W_UV,i latent[b,i,:]                               (fp32 accumulation)
  * latent bf16 [batch, n_h, 512]; w_uv bf16 [n_h, 128, 512]; out bf16 [batch, n_h, 128].
  */
-int mla_apply_wuv(mla_handle_t h, int32_t batch, const void* latent, const void* w_uv,
+MLA_API int mla_apply_wuv(mla_handle_t h, int32_t batch, const void* latent, const void* w_uv,
                   void* out, mla_stream_t stream);
 
 /*
@@ -230,7 +238,7 @@ int mla_apply_wuv(mla_handle_t h, int32_t batch, const void* latent, const void*
  * positive multiple of 64, a bad rms_eps, strides or alignment, a page table given to a
  * contiguous handle (or missing for a paged one); MLA_ERR_UNSUPPORTED for d_model > 8192.
  */
-int mla_append_kv(mla_handle_t h, int32_t batch, int32_t d_model, const void* hidden,
+MLA_API int mla_append_kv(mla_handle_t h, int32_t batch, int32_t d_model, const void* hidden,
                   const void* w_dkv, const void* w_kr, const void* gamma, float rms_eps,
                   void* c_kv, void* k_r, int64_t row_stride, int64_t seq_stride,
                   const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
@@ -244,7 +252,7 @@ int mla_append_kv(mla_handle_t h, int32_t batch, int32_t d_model, const void* hi
  * kv_codes + r*row_stride (bytes; a multiple of 16, >= 576), e to kv_exp[r]. Other arguments
  * and errors as for mla_append_kv.
  */
-int mla_append_kv_fp8(mla_handle_t h, int32_t batch, int32_t d_model, const void* hidden,
+MLA_API int mla_append_kv_fp8(mla_handle_t h, int32_t batch, int32_t d_model, const void* hidden,
                       const void* w_dkv, const void* w_kr, const void* gamma, float rms_eps,
                       void* kv_codes, int8_t* kv_exp, int64_t row_stride, int64_t seq_stride,
                       const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
@@ -274,7 +282,7 @@ int mla_append_kv_fp8(mla_handle_t h, int32_t batch, int32_t d_model, const void
  * The first call on a device looks up the array's device address; make it before any
  * stream capture.
  */
-int mla_decode_attn_noalloc(int32_t n_heads, float softmax_scale, int32_t page_size,
+MLA_API int mla_decode_attn_noalloc(int32_t n_heads, float softmax_scale, int32_t page_size,
                             int64_t max_kv_len, int32_t batch, const void* q_abs,
                             const void* c_kv, const void* k_r, int64_t row_stride,
                             int64_t seq_stride, const int32_t* kv_lens,
@@ -289,13 +297,13 @@ int mla_decode_attn_noalloc(int32_t n_heads, float softmax_scale, int32_t page_s
  * kv_len outside 0..max_kv_len, clamped, or outside 1..max_kv_len in mla_append_kv), or
  * MLA_ERR_CUDA if the synchronisation itself failed.
  */
-int mla_check_device_errors(mla_handle_t h, mla_stream_t stream, uint32_t* detail);
+MLA_API int mla_check_device_errors(mla_handle_t h, mla_stream_t stream, uint32_t* detail);
 
 /* Bytes of device workspace the handle holds. */
-int64_t mla_workspace_bytes(mla_handle_t h);
+MLA_API int64_t mla_workspace_bytes(mla_handle_t h);
 
 /* A static, human-readable name for a status code. */
-const char* mla_status_string(int status);
+MLA_API const char* mla_status_string(int status);
 
 #ifdef __cplusplus
 }

@@ -24,6 +24,7 @@ LIB = os.path.join(PKG, "libmla_decode.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
+                     "-Xcompiler", "-fvisibility=hidden",
                      "-I" + INCLUDE, "-I" + CSRC, "--expt-relaxed-constexpr",
                      "-Xptxas", "-warn-spills"]
 

@@ -94,3 +94,16 @@ def test_null_handle_and_null_out_are_rejected(lib):
                                None) == binding.MLA_ERR_INVALID_ARG
     assert lib.mla_apply_wuv(None, 1, None, None, None, None) == binding.MLA_ERR_INVALID_ARG
     assert lib.mla_workspace_bytes(None) == -1
+
+
+def test_library_exports_nothing_but_the_c_abi(lib):
+    """Everything but the declared C functions is built with hidden visibility."""
+    import shutil
+    import subprocess
+    nm = shutil.which("nm")
+    if nm is None:
+        pytest.skip("nm not available")
+    out = subprocess.run([nm, "-D", "--defined-only", binding.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if len(line.split()) == 3 and line.split()[1] == "T"}
+    assert exported == set(_declared_functions())

@@ -6,16 +6,18 @@
 // written as row kv_len[b]-1 of sequence b, in the cache layout the decode kernel reads
 // (DeepSeek-V2 architecture page eq. 9 c^KV = W^DKV h; the paper notes' RMSNorm after the
 // compressed latent; DeepSeek-V3 walkthrough section 2.2 k^R = RoPE(W^KR h), the two parts
-// that are cached).
+// that are cached). With q_len new tokens per sequence, h is [B, q_len, d] and token t's row
+// is kv_len[b] - q_len + t, rotated at that position. A quantised cache gets the row as E4M3
+// codes with the smallest power-of-two scale that fits (its exponent stored beside).
 //
 // Kernel 1, kv_down_tc: the projection is bound by reading the weights (576 x d bf16, 5.9 MB
 // at d = 5120), so it is cut into many CTAs: one per (128-feature block, slice of d, batch
 // chunk). The weights are the M = 128 operand (four blocks of W_DKV, one of W_KR whose rows
 // past 64 read as zero), the hidden states the N operand; four warps issue a quarter of the
 // slice's K steps each into their own accumulator, and the slice's partial sums go to the
-// handle's workspace. Kernel 2, kv_finalize: one CTA per sequence adds the slices' partials
-// in a fixed order (so the result does not depend on timing), applies the RMSNorm and the
-// rotation, and writes the row.
+// handle's workspace. Kernel 2, kv_finalize: one CTA per (sequence, new token) row adds the
+// slices' partials in a fixed order (so the result does not depend on timing), applies the
+// RMSNorm and the rotation, and writes the row (bf16, or quantised).
 #include <cudaTypedefs.h>
 
 #include <algorithm>

@@ -42,7 +42,11 @@ def shard_ranges(kv_len: int, world: int, tile: int = TILE) -> List[Tuple[int, i
 
 def local_lengths(kv_lens: Sequence[int], rank: int, world: int) -> List[int]:
     """Rows of each sequence that `rank` holds."""
-    return [shard_ranges(int(L), world)[rank][1] - shard_ranges(int(L), world)[rank][0] for L in kv_lens]
+    out = []
+    for L in kv_lens:
+        start, end = shard_ranges(int(L), world)[rank]
+        out.append(end - start)
+    return out
 
 
 def gather_partials(latent: torch.Tensor, lse: torch.Tensor, group=None) -> Tuple[torch.Tensor, torch.Tensor]:

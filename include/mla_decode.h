@@ -280,7 +280,7 @@ MLA_API int mla_append_kv_fp8(mla_handle_t h, int32_t batch, int32_t d_model, co
  * All calls on a device share the array and it keeps the last call's contents: calls whose
  * kernels overlap on the GPU (different streams or host threads) race, so serialise them.
  * The first call on a device looks up the array's device address; make it before any
- * stream capture.
+ * stream capture. A look-up that fails returns MLA_ERR_CUDA and is retried by the next call.
  */
 MLA_API int mla_decode_attn_noalloc(int32_t n_heads, float softmax_scale, int32_t page_size,
                             int64_t max_kv_len, int32_t batch, const void* q_abs,

@@ -19,7 +19,10 @@
 //   * the array keeps the previous call's contents; each call clears the error word and
 //     rewrites everything else it reads;
 //   * the first call on a device looks up the array's device address (cudaGetSymbolAddress)
-//     and caches it; make that first call before any stream capture.
+//     and caches it; make that first call before any stream capture. Only a successful
+//     look-up is cached: if it fails (for instance inside a capture, or with an unrelated
+//     error pending on the device), the call returns MLA_ERR_CUDA and the next call tries
+//     again.
 // The kernels are the same ones mla_decode_attn runs; only the scratch comes from here.
 #include <algorithm>
 #include <cmath>
@@ -39,32 +42,38 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
 struct DeviceScratch {
-  std::once_flag once;
-  cudaError_t status = cudaSuccess;
+  bool ready = false;             // the look-up below succeeded on this device
   unsigned char* base = nullptr;  // device address of g_scratch on this device
   int num_sms = 0;
   int major = 0;
 };
 DeviceScratch g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-// Once per device, with that device current: find the array and the SM count.
-DeviceScratch* device_scratch(int device) {
-  if (device < 0 || device >= kMaxDevices) return nullptr;
-  DeviceScratch* d = &g_dev[device];
-  std::call_once(d->once, [d, device]() {
+// With the device current: find the array and the SM count, once per device. A failed
+// look-up is not remembered, so a later call retries it.
+cudaError_t device_scratch(int device, DeviceScratch* out) {
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceScratch& d = g_dev[device];
+  if (!d.ready) {
+    DeviceScratch n;
     void* p = nullptr;
-    d->status = cudaGetSymbolAddress(&p, g_scratch);
-    if (d->status == cudaSuccess) {
-      d->base = static_cast<unsigned char*>(p);
-      d->status = cudaDeviceGetAttribute(&d->num_sms, cudaDevAttrMultiProcessorCount, device);
+    cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n.num_sms, cudaDevAttrMultiProcessorCount, device);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n.major, cudaDevAttrComputeCapabilityMajor, device);
+    if (e != cudaSuccess) {
+      cudaGetLastError();   // leave no error of the failed look-up behind for later calls
+      return e;
     }
-    if (d->status == cudaSuccess)
-      d->status = cudaDeviceGetAttribute(&d->major, cudaDevAttrComputeCapabilityMajor, device);
-  });
-  return d;
+    n.base = static_cast<unsigned char*>(p);
+    n.ready = true;
+    d = n;
+  }
+  *out = d;
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -112,19 +121,22 @@ extern "C" int mla_decode_attn_noalloc(int32_t n_heads, float softmax_scale, int
   // ---- the device's scratch (looked up once per device)
   int device = 0;
   if (cudaGetDevice(&device) != cudaSuccess) return MLA_ERR_CUDA;
-  DeviceScratch* d = device_scratch(device);
-  if (d == nullptr) return MLA_ERR_UNSUPPORTED;
-  if (d->status != cudaSuccess) return MLA_ERR_CUDA;
+  if (device < 0 || device >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+  DeviceScratch ds;
+  if (device_scratch(device, &ds) != cudaSuccess) return MLA_ERR_CUDA;
+  const DeviceScratch* d = &ds;
   if (d->major != 10) return MLA_ERR_UNSUPPORTED;
 
   // ---- carve the scratch: plan region first, then the split partials. Fewer heads leave
   // room for more slots; the number of units is what fits after one slot per sequence.
   const size_t slot_bytes = size_t(n_heads) * (kDLatent + 1) * sizeof(float);
   const int max_slots = int((kScratchBytes - kPlanBytes - 1024) / slot_bytes);
-  const int units = std::min(d->num_sms, max_slots - batch);
+  // one unit per 2-CTA cluster of the decode kernel, as the handle path plans it
+  const int units = std::min(d->num_sms / 2, max_slots - batch);
   if (units < 1) return MLA_ERR_UNSUPPORTED;
 
-  mla_decode_s h;  // a handle on the stack: no allocation, scratch pointers into g_scratch
+  mla_decode_s h{};  // a handle on the stack: no allocation, scratch pointers into g_scratch
+  h.cfg = mla_config_t{};
   h.cfg.n_heads = n_heads;
   h.q_len = 1;
   h.n_rows = n_heads;

@@ -37,7 +37,11 @@ def test_shard_partials_merge_to_the_whole_request(world):
     g = w.to(DEV)
     a = workload_np(w)
     full = binding.MlaDecode(128, 2, w.max_kv_len)
-    q_abs = full.absorb_q(g.q_c, g.q_r, g.w_uk, g.kv_lens)       # global positions
+    # the oracle's absorbed query (global positions) in bf16 feeds both sides, so no oracle
+    # input comes from the CUDA path
+    q_ref = oracle.absorb_query(a["q_c"], a["q_r"], a["w_uk"], a["kv_lens"], w.rope_base)
+    q_bf = torch.from_numpy(q_ref).to(torch.float32).to(torch.bfloat16)
+    q_abs = q_bf.to(DEV)
     lat_parts, lse_parts = [], []
     for r in range(world):
         local, lens = _local_cache(g.cache, w.kv_lens.tolist(), r, world)
@@ -48,7 +52,7 @@ def test_shard_partials_merge_to_the_whole_request(world):
         lse_parts.append(lse)
     latent, lse = full.merge_partials(torch.stack(lat_parts), torch.stack(lse_parts))
     full.check_device_errors()
-    ref_lat, ref_lse = oracle.latent_attention(to_np(q_abs), a["cache"], a["kv_lens"],
+    ref_lat, ref_lse = oracle.latent_attention(to_np(q_bf), a["cache"], a["kv_lens"],
                                                oracle.default_scale())
     assert_close(f64(latent), ref_lat, f"{world} shards merged: latent")
     assert_close(lse.cpu().numpy(), ref_lse, f"{world} shards merged: lse")

@@ -212,6 +212,49 @@ def test_zero_query_gives_the_mean_latent():
             np.testing.assert_allclose(out[b, i], t["w_uv"][i] @ mean_c, atol=1e-13)
 
 
+def _latent(t):
+    """The oracle's absorbed stages up to the latent output, on a _tiny case (d_c = 8)."""
+    q_abs = oracle.absorb_query(t["q_c"], t["q_r"], t["w_uk"], t["kv_lens"], t["rope_base"])
+    return oracle.latent_attention(q_abs, t["cache"], t["kv_lens"], t["scale"], d_latent=8)
+
+
+def test_latent_of_one_token_is_its_latent_row():
+    """One cached row takes probability 1, so the latent output is exactly that row's d_c
+    latent values (not its k^R part), whatever the query. This pins latent_attention
+    directly: in _tiny W_UV maps 8 latent values to 4, so an error in its null space would
+    pass the head-output pins."""
+    t = _tiny(L=(1, 1))
+    latent, lse = _latent(t)
+    for b in range(2):
+        for i in range(2):
+            np.testing.assert_array_equal(latent[b, i], t["cache"][b, 0, :8])
+    assert np.all(np.isfinite(lse))
+
+
+def test_latent_of_zero_query_is_the_mean_row_and_lse_is_log_l():
+    """A zero absorbed query gives every row the score 0: p = 1/L, the latent output is the
+    mean of the L latent rows and the log-sum-exp is log L."""
+    t = _tiny(L=(5, 3))
+    t["q_c"][:] = 0.0
+    t["q_r"][:] = 0.0
+    latent, lse = _latent(t)
+    for b, L in enumerate(t["kv_lens"]):
+        for i in range(2):
+            np.testing.assert_allclose(latent[b, i], t["cache"][b, :L, :8].mean(axis=0),
+                                       rtol=0, atol=1e-14)
+            np.testing.assert_allclose(lse[b, i], math.log(L), rtol=0, atol=1e-14)
+
+
+def test_latent_of_identical_rows_is_that_row():
+    """Rows that are all equal give the same latent output for any query and weights."""
+    t = _tiny()
+    t["cache"][:] = t["cache"][:, :1, :]
+    latent, _ = _latent(t)
+    for b in range(2):
+        for i in range(2):
+            np.testing.assert_allclose(latent[b, i], t["cache"][b, 0, :8], rtol=0, atol=1e-13)
+
+
 def test_identical_rows_make_the_query_irrelevant():
     t = _tiny()
     t["cache"][:] = t["cache"][:, :1, :]

@@ -5,16 +5,24 @@
 A step is one pass of the whole hot path over one batch: query absorption + RoPE, the
 split-KV decode attention over the latent cache (plan, split kernel, combine), and the W_UV
 up-projection, through the C ABI. The K timed steps are replayed from a CUDA graph of the
-same calls (`value`); `e2e` runs them eagerly through the public API with the inputs copied
-from pinned host memory and the output copied back every step. Inputs are resident in HBM
-before the timed region;
-every step reads a different one of several cache copies whose total exceeds L2 four times,
-so no step finds its cache in L2. Multi-GPU (torchrun, one process per GPU): every rank runs
-its own replica of the workload (sequences are independent; no data-path collective), the
-timing is the max over ranks, and `value` counts the tokens of all ranks (weak scaling).
+same calls (`value`). `e2e` runs the step through the public API with the inputs copied
+from pinned host memory and the output copied back every step: `value` as a serving loop
+would (per-step CUDA graphs, copies on side branches), `eager_value` as plain calls (the
+host path of every C-ABI call inside the timed region). Inputs are resident in HBM before
+the timed region; every step reads a different one of several cache copies whose total
+exceeds L2 four times, so no step finds its cache in L2.
+
+The headline workload is the largest single-GPU configuration (64 ragged sequences, paged);
+`workloads` reports the other four the same way. Multi-GPU (one process per GPU; started
+under torchrun, or `--gpus N` relaunches itself under torchrun): every rank runs its own
+replica of the workload (sequences are independent; no data-path collective), the timing is
+the max over ranks, and `value` counts the tokens of all ranks (weak scaling).
 
 --impl reference times the fp64 CPU oracle on the host cores (rank 0 only), each step one
-(sequence, head) output of the same workload.
+sample unit of the same workload (8 heads of one sequence, the non-absorbed definition),
+the same unit `cpu_baseline` repeats for about 15 s.
+--profile runs W warm-up steps and then K eager steps of the hot path alone (no graphs, no
+extra measurements, no JSON line): the command the committed ncu summaries were taken on.
 """
 
 from __future__ import annotations
@@ -38,7 +46,7 @@ sys.path.insert(0, ROOT)
 from mla_latent_kv_28_b200 import workloads as wl  # noqa: E402
 
 METRIC = "MLA decode tokens/s & latent-KV GB/s on 1 B200; % of binding roofline"
-DEFAULT_WORKLOAD = "v2_b32_l4096"
+DEFAULT_WORKLOAD = "ragged_paged_b64"
 L2_BYTES = 126 * 2**20
 ROW_BYTES = 576 * 2
 KERNEL_SOURCES = ["decode_split.cu", "sm100.cuh"]
@@ -221,23 +229,62 @@ def workload_np(w):
                 page_size=w.page_size)
 
 
-def oracle_tokens_per_s(w, budget_s: float = 15.0, max_tokens: int = 4):
-    """Time the fp64 oracle (non-absorbed definition) on whole decode tokens: every head of
-    sequence 0, then 1, ... until the budget is spent. Returns (tokens/s, tokens, seconds)."""
-    import oracle
-    a = workload_np(w)
-    scale = oracle.default_scale()
-    done, t0 = 0, time.perf_counter()
-    for b in range(min(max_tokens, w.batch)):
-        pairs = [(b, i) for i in range(w.n_heads)]
-        oracle.mla_decode_nonabsorbed(a["q_c"], a["q_r"], a["w_uk"], a["w_uv"], a["cache"],
-                                      a["kv_lens"], scale, w.rope_base, a["page_table"],
-                                      a["page_size"], pairs=pairs)
-        done += 1
+HEADS_PER_UNIT = 8
+
+
+class OracleSample:
+    """The fp64 oracle as it stands (the non-absorbed definition) on sample units of a
+    workload. A unit is HEADS_PER_UNIT heads of one sequence; unit k is head group
+    k // batch of sequence k % batch, so consecutive units spread over the sequences (and,
+    in the ragged workload, over its length mix). The weights and queries are cut to each
+    unit's heads before any timing, so a call widens only what it reads. The reference arm
+    and `cpu_baseline` both time these units."""
+
+    def __init__(self, w):
+        import numpy as np
+        import oracle
+        self.oracle = oracle
+        self.w = w
+        self.a = workload_np(w)
+        self.scale = oracle.default_scale()
+        self.groups = [list(range(i, min(i + HEADS_PER_UNIT, w.n_heads)))
+                       for i in range(0, w.n_heads, HEADS_PER_UNIT)]
+        a = self.a
+        self.cut = []
+        for hs in self.groups:
+            idx = np.array(hs)
+            self.cut.append((a["q_c"][:, idx], a["q_r"][:, idx], a["w_uk"][idx], a["w_uv"][idx]))
+
+    def describe(self) -> str:
+        return (f"units of {HEADS_PER_UNIT} heads of one sequence (non-absorbed fp64), "
+                f"sequence k mod {self.w.batch}, head group k div {self.w.batch}")
+
+    def run(self, k: int) -> float:
+        """Unit k; returns the decode tokens it is worth (heads / n_heads)."""
+        b = k % self.w.batch
+        gi = (k // self.w.batch) % len(self.groups)
+        q_c, q_r, w_uk, w_uv = self.cut[gi]
+        a = self.a
+        n = len(self.groups[gi])
+        self.oracle.mla_decode_nonabsorbed(q_c, q_r, w_uk, w_uv, a["cache"], a["kv_lens"],
+                                           self.scale, self.w.rope_base, a["page_table"],
+                                           a["page_size"], pairs=[(b, i) for i in range(n)])
+        return n / self.w.n_heads
+
+
+def oracle_tokens_per_s(w, budget_s: float = 15.0):
+    """cpu_baseline: oracle sample units, one after another, until the budget is spent.
+    Returns (tokens/s, units, seconds, sample description)."""
+    s = OracleSample(w)
+    s.run(0)   # warm-up (BLAS threads, page faults)
+    tokens, k, t0 = 0.0, 0, time.perf_counter()
+    while True:
+        tokens += s.run(1 + k)
+        k += 1
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
-    return done / dt, done, dt
+    return tokens / dt, k, dt, s.describe()
 
 
 def blas_threads() -> int:
@@ -256,33 +303,22 @@ def run_reference(args):
     rank, world, local = dist_env()
     if rank != 0:
         return 0
-    import oracle
     w = wl.config_workload(args.workload, seed=0)
-    a = workload_np(w)
-    scale = oracle.default_scale()
-    pairs = [(b, i) for b in range(w.batch) for i in range(w.n_heads)]
-
-    def one(k):
-        b, i = pairs[k % len(pairs)]
-        oracle.mla_decode_nonabsorbed(a["q_c"], a["q_r"], a["w_uk"], a["w_uv"], a["cache"],
-                                      a["kv_lens"], scale, w.rope_base, a["page_table"],
-                                      a["page_size"], pairs=[(b, i)])
+    s = OracleSample(w)
     for k in range(args.warmup):
-        one(k)
-    t0 = time.perf_counter()
+        s.run(k)
+    tokens, t0 = 0.0, time.perf_counter()
     for k in range(args.steps):
-        one(args.warmup + k)
+        tokens += s.run(args.warmup + k)
     dt = time.perf_counter() - t0
-    tokens = args.steps / w.n_heads
     value = tokens / dt
     cores = blas_threads()
-    sample = (f"{args.steps} (sequence, head) outputs of {args.workload}, one per step "
-              f"({w.n_heads} make one decode token)")
+    sample = f"{args.steps} sample units of {args.workload}, one per step: {s.describe()}"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(w, args.workload),
+            "config": workload_config(w, args.workload, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -292,14 +328,25 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------------------- ours
-def workload_config(w, name):
+def cache_copies(w) -> tuple[int, int]:
+    """(copies, bytes per copy): enough copies of the cache that their total exceeds L2 four
+    times, so a step that reads the next copy finds none of it in L2."""
+    alloc = w.cache.numel() * w.cache.element_size()
+    return max(1, math.ceil(4 * L2_BYTES / alloc)), alloc
+
+
+def workload_config(w, name, world: int = 1):
     lens = w.kv_lens
+    copies, alloc = cache_copies(w)
     return {"workload": name, "batch": w.batch, "n_heads": w.n_heads,
             "kv_len": int(lens[0]) if bool((lens == lens[0]).all()) else
             f"ragged {int(lens.min())}..{int(lens.max())}",
             "cached_tokens_per_gpu": w.cached_tokens,
             "layout": f"paged {w.page_size}" if w.page_size else "contiguous",
-            "rope_base": w.rope_base, "d_c": 512, "d_rope": 64, "d_head": 128}
+            "rope_base": w.rope_base, "d_c": 512, "d_rope": 64, "d_head": 128,
+            "l2": f"inputs larger than L2: {copies} rotating cache copies of "
+                  f"{alloc / 1e6:.0f} MB per GPU, one per step",
+            "parallelism": f"replicas x{world} (one per GPU, no data-path collective)"}
 
 
 def append_kv_measure(h, w, g, caches, copies, stream, args, world, local, dev,
@@ -319,29 +366,8 @@ def append_kv_measure(h, w, g, caches, copies, stream, args, world, local, dev,
         h.append_kv(inp["hidden"], wd, wr, inp["gamma"], caches[k % copies], g.kv_lens,
                     g.page_table, stream=stream)
 
-    with torch.cuda.stream(stream):
-        for k in range(args.warmup):
-            call(k)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        for k in range(args.steps):
-            call(k)
-    with torch.cuda.stream(stream):
-        graph.replay()
-    torch.cuda.synchronize(dev)
+    ms = graph_ms(call, stream, args, world, local, dev)
     h.check_device_errors(stream)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world, local, True)
-    torch.cuda.synchronize(dev)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        graph.replay()
-        e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(world, local, True)
-    h.check_device_errors(stream)
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
-    del graph
     # algorithmic bytes: the two weights, the hidden states, gamma, the rows written
     algo = wbytes + w.batch * d_model * 2 + 512 * 2 + w.batch * ROW_BYTES
     hbm_gbs, _, peak_kind = measured_peaks()
@@ -433,6 +459,7 @@ def fp8_cache_measure(h, w, g, stream, args, world, local, dev):
                                               stream=stream),
                   stream, args, world, local, dev)
     h.check_device_errors(stream)
+    del copies8
     algo = w.cached_tokens * (576 + 1)
     hbm_gbs, _, peak_kind = measured_peaks()
     gbs = algo / (ms * 1e-3) / 1e9
@@ -442,6 +469,225 @@ def fp8_cache_measure(h, w, g, stream, args, world, local, dev):
             "gpu_launches": 3 * args.steps}
 
 
+class DecodeBench:
+    """One workload on this GPU: its inputs in HBM, the rotating cache copies, a handle, and
+    the timings of the step, of the attention call alone, and of the step end to end."""
+
+    def __init__(self, name, args, world, local, dev, rank):
+        from mla_latent_kv_28_b200 import binding
+        self.name, self.args, self.world, self.local, self.dev = name, args, world, local, dev
+        self.w = wl.config_workload(name, seed=replica_seed(rank))
+        self.g = self.w.to(dev)
+        self.copies, self.alloc_bytes = cache_copies(self.w)
+        self.caches = [self.g.cache] + [self.g.cache.clone() for _ in range(self.copies - 1)]
+        w = self.w
+        self.h = binding.MlaDecode(w.n_heads, w.batch, w.max_kv_len, page_size=w.page_size,
+                                   rope_base=w.rope_base)
+        B, H = w.batch, w.n_heads
+        self.bufs = {"q_abs": torch.empty((B, H, 576), dtype=torch.bfloat16, device=dev),
+                     "latent": torch.empty((B, H, 512), dtype=torch.bfloat16, device=dev),
+                     "out": torch.empty((B, H, 128), dtype=torch.bfloat16, device=dev)}
+        self.stream = torch.cuda.Stream(dev)   # a capturable stream for the graphs below
+
+    def step(self, k):
+        h, g, b, s = self.h, self.g, self.bufs, self.stream
+        q_abs = h.absorb_q(g.q_c, g.q_r, g.w_uk, g.kv_lens, b["q_abs"], s)
+        h.decode_attn(q_abs, self.caches[k % self.copies], g.kv_lens, g.page_table, b["latent"],
+                      None, want_lse=False, stream=s)
+        h.apply_wuv(b["latent"], g.w_uv, b["out"], s)
+
+    def attn(self, k):
+        h, g, b = self.h, self.g, self.bufs
+        h.decode_attn(b["q_abs"], self.caches[k % self.copies], g.kv_lens, g.page_table,
+                      b["latent"], None, want_lse=False, stream=self.stream)
+
+    def device_times(self, clocks=None):
+        """(step ms, attention ms, wall window of the step's timed region), each from a CUDA
+        graph of K calls (no host launch time between kernels; the kernels are the launches
+        the eager calls make), max over ranks."""
+        args, stream, dev = self.args, self.stream, self.dev
+        with torch.cuda.stream(stream):
+            for k in range(args.warmup):
+                self.step(k)
+        self.h.check_device_errors(stream)
+        step_graph, attn_graph = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(step_graph, stream=stream):
+            for k in range(args.steps):
+                self.step(k)
+        with torch.cuda.graph(attn_graph, stream=stream):
+            for k in range(args.steps):
+                self.attn(k)
+        with torch.cuda.stream(stream):
+            step_graph.replay()
+            attn_graph.replay()
+        torch.cuda.synchronize(dev)
+        self.h.check_device_errors(stream)
+
+        def timed(graph):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            barrier(self.world, self.local, True)
+            torch.cuda.synchronize(dev)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                graph.replay()
+                e1.record(stream)
+            torch.cuda.synchronize(dev)
+            barrier(self.world, self.local, True)
+            return e0.elapsed_time(e1) / args.steps
+
+        w0 = time.perf_counter()
+        ms = timed(step_graph)
+        w1 = time.perf_counter()
+        attn_ms = timed(attn_graph)
+        self.h.check_device_errors(stream)
+        del step_graph, attn_graph
+        return (max_over_ranks(ms, self.world, dev), max_over_ranks(attn_ms, self.world, dev),
+                (w0, w1))
+
+    def e2e_times(self):
+        """(graph ms, eager ms, h2d bytes, d2h bytes) per step, end to end through the public
+        API: every step uploads its inputs (q^C, q^R, kv_len) from pinned host memory and
+        downloads its head outputs to pinned host memory.
+
+        Graph: as a serving loop would, the step runs as a CUDA graph with the copies on their
+        own branches: graph k computes step k from the inputs graph k-1 uploaded, while
+        uploading step k+1's inputs and downloading step k-1's outputs, so the copies overlap
+        the kernels and one graph launch is all the host does per step. The graphs are
+        captured from the public calls (MlaDecode.step and tensor copies); the timed region
+        covers the first upload, K graphs, and the last download.
+        Eager: the same per step as plain calls on one stream (upload, MlaDecode.step,
+        download), so the host path of every C-ABI call (argument checks, tensor-map encodes,
+        launches) is inside the timed region."""
+        args, stream, dev, g, h = self.args, self.stream, self.dev, self.g, self.h
+        B, H = self.w.batch, self.w.n_heads
+        hq_c = g.q_c.cpu().pin_memory()
+        hq_r = g.q_r.cpu().pin_memory()
+        hlens = g.kv_lens.cpu().pin_memory()
+        hout = [torch.empty((B, H, 128), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        din = [(torch.empty_like(g.q_c), torch.empty_like(g.q_r), torch.empty_like(g.kv_lens))
+               for _ in range(2)]
+        dout = [torch.empty((B, H, 128), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        h2d = hq_c.numel() * 2 + hq_r.numel() * 2 + hlens.numel() * 4
+        d2h = hout[0].numel() * 2
+        copy = torch.cuda.Stream(dev)       # uploads
+        copy_out = torch.cuda.Stream(dev)   # downloads, on another copy engine
+        copies = self.copies
+
+        def upload(slot):
+            for d, hsrc in zip(din[slot], (hq_c, hq_r, hlens)):
+                d.copy_(hsrc, non_blocking=True)
+
+        def e2e_step(k):
+            slot = k % 2
+            fork = torch.cuda.Event()
+            fork.record(stream)
+            copy.wait_event(fork)
+            copy_out.wait_event(fork)
+            with torch.cuda.stream(copy):
+                upload(1 - slot)                                        # inputs of step k+1
+                join_in = torch.cuda.Event()
+                join_in.record(copy)
+            with torch.cuda.stream(copy_out):
+                hout[1 - slot].copy_(dout[1 - slot], non_blocking=True)  # outputs of step k-1
+                join_out = torch.cuda.Event()
+                join_out.record(copy_out)
+            dq_c, dq_r, dlens = din[slot]
+            h.step(dq_c, dq_r, g.w_uk, g.w_uv, self.caches[k % copies], dlens, g.page_table,
+                   stream, dict(self.bufs, out=dout[slot]))
+            stream.wait_event(join_in)
+            stream.wait_event(join_out)
+
+        n_graphs = 2 * copies // math.gcd(2, copies)   # input slot and cache copy both cycle
+        with torch.cuda.stream(stream):
+            upload(0)
+            for k in range(max(args.warmup, n_graphs)):
+                e2e_step(k)
+        torch.cuda.synchronize(dev)
+        e2e_graphs = []
+        for k in range(n_graphs):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                e2e_step(k)
+            e2e_graphs.append(gr)
+        with torch.cuda.stream(stream):
+            upload(0)
+            for k in range(n_graphs):
+                e2e_graphs[k].replay()
+        torch.cuda.synchronize(dev)
+        h.check_device_errors(stream)
+        e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(self.world, self.local, True)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            e_start.record(stream)
+            upload(0)
+            for k in range(args.steps):
+                e2e_graphs[k % n_graphs].replay()
+            hout[(args.steps - 1) % 2].copy_(dout[(args.steps - 1) % 2], non_blocking=True)
+            e_end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(self.world, self.local, True)
+        h.check_device_errors(stream)
+        del e2e_graphs
+        graph_ms_ = max_over_ranks(e_start.elapsed_time(e_end) / args.steps, self.world, dev)
+
+        # eager: every call from the host, in order, on one stream
+        def eager_step(k):
+            upload(0)
+            dq_c, dq_r, dlens = din[0]
+            h.step(dq_c, dq_r, g.w_uk, g.w_uv, self.caches[k % copies], dlens, g.page_table,
+                   stream, dict(self.bufs, out=dout[0]))
+            hout[0].copy_(dout[0], non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for k in range(args.warmup):
+                eager_step(k)
+        torch.cuda.synchronize(dev)
+        barrier(self.world, self.local, True)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            e_start.record(stream)
+            for k in range(args.steps):
+                eager_step(k)
+            e_end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(self.world, self.local, True)
+        h.check_device_errors(stream)
+        eager_ms = max_over_ranks(e_start.elapsed_time(e_end) / args.steps, self.world, dev)
+        return graph_ms_, eager_ms, h2d, d2h
+
+    def roofline(self, attn_ms):
+        hbm_gbs, bf16_tf, peak_kind = measured_peaks()
+        cache_bytes = self.w.cached_tokens * ROW_BYTES
+        achieved = cache_bytes / (attn_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                "frac": achieved / hbm_gbs, "traffic": profiled_traffic(self.name),
+                "kernel": "mla_decode_attn (plan + split-KV + combine)",
+                "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes": cache_bytes,
+                "tensor_frac_of_measured": (self.w.cached_tokens * 2 * 1088 * self.w.n_heads)
+                / (attn_ms * 1e-3) / (bf16_tf * 1e12)}
+
+    def close(self):
+        self.h.close()
+        del self.caches, self.g
+
+
+def run_profile(args):
+    """W warm-up steps, then K eager steps of the hot path of one workload: nothing else
+    runs, so an ncu capture of this command sees only the step's kernels."""
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    bench = DecodeBench(args.workload, args, 1, local, dev, rank)
+    with torch.cuda.stream(bench.stream):
+        for k in range(args.warmup + args.steps):
+            bench.step(k)
+    torch.cuda.synchronize(dev)
+    bench.h.check_device_errors(bench.stream)
+    bench.close()
+    return 0
+
+
 def run_ours(args):
     rank, world, local = dist_env()
     if not torch.cuda.is_available():
@@ -449,196 +695,78 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     init_dist(world, local, "nccl")
-    from mla_latent_kv_28_b200 import binding
 
-    w = wl.config_workload(args.workload, seed=replica_seed(rank))
-    g = w.to(dev)
-    cache_bytes = w.cached_tokens * ROW_BYTES              # algorithmic bytes per step
-    alloc_bytes = g.cache.numel() * g.cache.element_size()
-    copies = max(1, math.ceil(4 * L2_BYTES / alloc_bytes))
-    caches = [g.cache] + [g.cache.clone() for _ in range(copies - 1)]
-
-    h = binding.MlaDecode(w.n_heads, w.batch, w.max_kv_len, page_size=w.page_size,
-                          rope_base=w.rope_base)
-    B, H = w.batch, w.n_heads
-    bufs = {"q_abs": torch.empty((B, H, 576), dtype=torch.bfloat16, device=dev),
-            "latent": torch.empty((B, H, 512), dtype=torch.bfloat16, device=dev),
-            "out": torch.empty((B, H, 128), dtype=torch.bfloat16, device=dev)}
-    stream = torch.cuda.Stream(dev)   # a capturable stream for the graphs below
-
-    def step(k):
-        q_abs = h.absorb_q(g.q_c, g.q_r, g.w_uk, g.kv_lens, bufs["q_abs"], stream)
-        h.decode_attn(q_abs, caches[k % copies], g.kv_lens, g.page_table, bufs["latent"],
-                      None, want_lse=False, stream=stream)
-        h.apply_wuv(bufs["latent"], g.w_uv, bufs["out"], stream)
-
-    def attn(k):
-        h.decode_attn(bufs["q_abs"], caches[k % copies], g.kv_lens, g.page_table, bufs["latent"],
-                      None, want_lse=False, stream=stream)
-
-    with torch.cuda.stream(stream):
-        for k in range(args.warmup):
-            step(k)
-    h.check_device_errors(stream)
-    # The K timed steps are replayed from one CUDA graph, so no host launch time sits between
-    # kernels (the kernels are the same launches the eager calls make); the attention call
-    # alone, K times, is a second graph timed the same way for the kernel's roofline.
-    step_graph, attn_graph = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(step_graph, stream=stream):
-        for k in range(args.steps):
-            step(k)
-    with torch.cuda.graph(attn_graph, stream=stream):
-        for k in range(args.steps):
-            attn(k)
-    with torch.cuda.stream(stream):
-        step_graph.replay()
-        attn_graph.replay()
-    torch.cuda.synchronize(dev)
-    h.check_device_errors(stream)
-
-    def timed(graph):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier(world, local, True)
-        torch.cuda.synchronize(dev)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            graph.replay()
-            e1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier(world, local, True)
-        return e0.elapsed_time(e1) / args.steps
-
+    main = DecodeBench(args.workload, args, world, local, dev, rank)
+    w = main.w
     clocks = ClockSampler(local)
     clocks.start()
-    w0 = time.perf_counter()
-    ms = timed(step_graph)
-    w1 = time.perf_counter()
-    attn_ms = timed(attn_graph)
-    h.check_device_errors(stream)
-    ms_max = max_over_ranks(ms, world, dev)
-    del step_graph, attn_graph
-
-    # End to end through the public API: every step uploads its inputs from pinned host
-    # memory and downloads its head outputs to pinned host memory. A serving loop would run
-    # the step as a CUDA graph with the copies on their own branch: graph k computes step k
-    # from the inputs uploaded by graph k-1, while uploading step k+1's inputs and downloading
-    # step k-1's outputs, so the copies overlap the kernels and one graph launch is all the
-    # host does per step. The graphs are captured from the public calls (MlaDecode.step and
-    # tensor copies); the timed region covers the first upload, K graphs, and the last
-    # download.
-    hq_c = g.q_c.cpu().pin_memory()
-    hq_r = g.q_r.cpu().pin_memory()
-    hlens = g.kv_lens.cpu().pin_memory()
-    hout = [torch.empty((B, H, 128), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    din = [(torch.empty_like(g.q_c), torch.empty_like(g.q_r), torch.empty_like(g.kv_lens))
-           for _ in range(2)]
-    dout = [torch.empty((B, H, 128), dtype=torch.bfloat16, device=dev) for _ in range(2)]
-    h2d = hq_c.numel() * 2 + hq_r.numel() * 2 + hlens.numel() * 4
-    d2h = hout[0].numel() * 2
-    copy = torch.cuda.Stream(dev)       # uploads
-    copy_out = torch.cuda.Stream(dev)   # downloads, on another copy engine
-
-    def upload(slot):
-        for d, hsrc in zip(din[slot], (hq_c, hq_r, hlens)):
-            d.copy_(hsrc, non_blocking=True)
-
-    def e2e_step(k):
-        slot = k % 2
-        fork = torch.cuda.Event()
-        fork.record(stream)
-        copy.wait_event(fork)
-        copy_out.wait_event(fork)
-        with torch.cuda.stream(copy):
-            upload(1 - slot)                                        # inputs of step k+1
-            join_in = torch.cuda.Event()
-            join_in.record(copy)
-        with torch.cuda.stream(copy_out):
-            hout[1 - slot].copy_(dout[1 - slot], non_blocking=True)  # outputs of step k-1
-            join_out = torch.cuda.Event()
-            join_out.record(copy_out)
-        dq_c, dq_r, dlens = din[slot]
-        h.step(dq_c, dq_r, g.w_uk, g.w_uv, caches[k % copies], dlens, g.page_table, stream,
-               dict(bufs, out=dout[slot]))
-        stream.wait_event(join_in)
-        stream.wait_event(join_out)
-
-    n_graphs = 2 * copies // math.gcd(2, copies)   # input slot and cache copy both cycle
-    with torch.cuda.stream(stream):
-        upload(0)
-        for k in range(max(args.warmup, n_graphs)):
-            e2e_step(k)
-    torch.cuda.synchronize(dev)
-    e2e_graphs = []
-    for k in range(n_graphs):
-        gr = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gr, stream=stream):
-            e2e_step(k)
-        e2e_graphs.append(gr)
-    with torch.cuda.stream(stream):
-        upload(0)
-        for k in range(n_graphs):
-            e2e_graphs[k].replay()
-    torch.cuda.synchronize(dev)
-    h.check_device_errors(stream)
-    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world, local, True)
-    torch.cuda.synchronize(dev)
-    with torch.cuda.stream(stream):
-        e_start.record(stream)
-        upload(0)
-        for k in range(args.steps):
-            e2e_graphs[k % n_graphs].replay()
-        hout[(args.steps - 1) % 2].copy_(dout[(args.steps - 1) % 2], non_blocking=True)
-        e_end.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(world, local, True)
-    h.check_device_errors(stream)
-    del e2e_graphs
-    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / args.steps, world, dev)
+    ms_max, attn_ms, (w0, w1) = main.device_times()
+    e2e_ms, eager_ms, h2d, d2h = main.e2e_times()
     clocks.stop()
 
-    append = append_kv_measure(h, w, g, caches, copies, stream, args, world, local, dev)
-    tokens = multi_token_measure(w, g, caches, copies, stream, args, world, local, dev)
-    fp8 = fp8_cache_measure(h, w, g, stream, args, world, local, dev)
+    append = append_kv_measure(main.h, w, main.g, main.caches, main.copies, main.stream, args,
+                               world, local, dev)
+    tokens = multi_token_measure(w, main.g, main.caches, main.copies, main.stream, args, world,
+                                 local, dev)
+    fp8 = fp8_cache_measure(main.h, w, main.g, main.stream, args, world, local, dev)
+    roof = main.roofline(attn_ms)
+    main.close()
+    del main
+    torch.cuda.empty_cache()
+
+    # the other workloads, timed the same way (one at a time, each with its own cache copies)
+    others = {}
+    for name in sorted(wl.CONFIGS):
+        if name == args.workload or args.headline_only:
+            continue
+        o = DecodeBench(name, args, world, local, dev, rank)
+        o_ms, o_attn, _ = o.device_times()
+        o_e2e, o_eager, _, _ = o.e2e_times()
+        others[name] = {"tokens_per_s": job_tokens_per_s(world, o.w.batch, o_ms),
+                        "ms_per_step": o_ms, "attn_us": o_attn * 1e3,
+                        "cached_tokens_per_gpu": o.w.cached_tokens,
+                        "roofline": o.roofline(o_attn),
+                        "e2e": {"value": job_tokens_per_s(world, o.w.batch, o_e2e),
+                                "eager_value": job_tokens_per_s(world, o.w.batch, o_eager),
+                                "unit": "tokens/s"},
+                        "config": workload_config(o.w, name, world),
+                        "gpu_launches": 5 * args.steps}
+        o.close()
+        del o
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, toks, secs = oracle_tokens_per_s(w)
+        tps, units, secs, desc = oracle_tokens_per_s(w)
         cpu = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{toks} decode token(s) of {args.workload} (all {H} heads of sequences "
-                         f"0..{toks - 1}, non-absorbed fp64), {secs:.1f} s"}
+               "sample": f"{units} sample units of {args.workload} in {secs:.1f} s: {desc}"}
 
-    hbm_gbs, bf16_tf, peak_kind = measured_peaks()
-    achieved = cache_bytes / (attn_ms * 1e-3) / 1e9
-    value = job_tokens_per_s(world, B, ms_max)
+    cache_bytes = w.cached_tokens * ROW_BYTES
+    B = w.batch
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "metric": METRIC, "value": job_tokens_per_s(world, B, ms_max), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; workload shapes of the DeepSeek-V2 MLA layer)",
-        "config": dict(workload_config(w, args.workload),
-                       l2=f"inputs larger than L2: {copies} rotating cache copies of "
-                          f"{alloc_bytes / 1e6:.0f} MB per GPU, one per step",
-                       parallelism=f"replicas x{world} (one per GPU, no data-path collective)"),
+        "config": workload_config(w, args.workload, world),
         "kv_gbs": world * cache_bytes / (ms_max * 1e-3) / 1e9,
         "attn_us": attn_ms * 1e3,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
-                     "frac": achieved / hbm_gbs, "traffic": profiled_traffic(args.workload),
-                     "kernel": "mla_decode_attn (plan + split-KV + combine)",
-                     "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes": cache_bytes,
-                     "tensor_frac_of_measured": (cache_bytes / ROW_BYTES * 2 * 1088 * H)
-                     / (attn_ms * 1e-3) / (bf16_tf * 1e12)},
+        "roofline": roof,
         "e2e": {"value": job_tokens_per_s(world, B, e2e_ms), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "eager_value": job_tokens_per_s(world, B, eager_ms),
+                "how": "value: per-step CUDA graphs of MlaDecode.step with the copies on side "
+                       "branches; eager_value: plain calls (upload, step, download) per step"},
         "gpu_launches": 5 * args.steps,
         "clocks": clocks.summary(w0, w1),
     }
     line["append_kv"] = append
     line["multi_token"] = tokens
     line["fp8_cache"] = fp8
+    if others:
+        line["workloads"] = others
     if cpu is not None:
         line["cpu_baseline"] = cpu
-    h.close()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -647,20 +775,47 @@ def run_ours(args):
     return 0
 
 
+def relaunch_under_torchrun(argv, gpus: int) -> int:
+    """`--gpus N` (N > 1) started without torchrun: start N ranks through torchrun on this
+    node (rendezvous on 127.0.0.1) and return its exit status."""
+    import socket
+    import subprocess
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={gpus}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__)] + list(argv)
+    return subprocess.call(cmd)
+
+
 def main(argv=None):
+    argv = sys.argv[1:] if argv is None else list(argv)
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wl.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time only --workload (no `workloads` key)")
+    ap.add_argument("--profile", action="store_true",
+                    help="run W + K eager steps of --workload and nothing else (for ncu)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
     rank, world, _ = dist_env()
-    if world != args.gpus and not (world == 1 and args.gpus == 1):
-        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return relaunch_under_torchrun(argv, args.gpus)
+    if world != args.gpus:
+        print(f"error: --gpus {args.gpus} but WORLD_SIZE {world}: launch one process per GPU "
+              f"(torchrun --nproc-per-node {args.gpus}) or drop torchrun", file=sys.stderr)
+        return 2
+    if args.profile:
+        return run_profile(args)
     return run_reference(args) if args.impl == "reference" else run_ours(args)
 
 

@@ -80,3 +80,50 @@ def test_committed_decode_profile_parses():
     # while the kernel sources are the profiled ones, bench reports the traffic
     if vals["kernel_sources_sha"] == bench.kernel_sources_sha():
         assert bench.profiled_traffic("v2_b32_l4096") == float(vals["dram_bytes_per_launch"])
+
+
+def _run_bench(*args, timeout=600):
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    env["CUDA_VISIBLE_DEVICES"] = ""
+    return subprocess.run([sys.executable, os.path.join(root, "bench.py"), *args],
+                          capture_output=True, text=True, timeout=timeout, cwd=root, env=env)
+
+
+def test_gpus_n_without_torchrun_starts_n_ranks():
+    """`--gpus 2` outside torchrun relaunches itself as two ranks: the reference arm then runs
+    on rank 0 alone (the other rank exits 0 without work) and reports n_gpus 2."""
+    import json
+    r = _run_bench("--gpus", "2", "--impl", "reference", "--workload", "tiny_h16_l256",
+                   "--steps", "2", "--warmup", "3")
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1 and lines[0]["n_gpus"] == 2 and lines[0]["impl"] == "reference"
+
+
+def test_gpus_n_never_measures_fewer_gpus():
+    """Without GPUs, `--gpus 2` fails loudly (each rank needs a GPU) instead of printing a
+    one-GPU line; a WORLD_SIZE that disagrees with --gpus is refused."""
+    r = _run_bench("--gpus", "2", "--workload", "tiny_h16_l256", "--steps", "2", "--warmup", "3",
+                   "--no-cpu-baseline")
+    assert r.returncode != 0
+    assert '"n_gpus": 1' not in r.stdout
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0", CUDA_VISIBLE_DEVICES="")
+    r2 = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2"],
+                        capture_output=True, text=True, timeout=300, cwd=root, env=env)
+    assert r2.returncode == 2 and "WORLD_SIZE" in r2.stderr
+
+
+def test_reference_arm_and_cpu_baseline_time_the_same_units():
+    """Both CPU figures come from OracleSample: the same units, cut per head group."""
+    w = wl.config_workload("tiny_h16_l256")
+    s = bench.OracleSample(w)
+    assert abs(s.run(0) - bench.HEADS_PER_UNIT / w.n_heads) < 1e-12
+    tps, units, secs, desc = bench.oracle_tokens_per_s(w, budget_s=0.5)
+    assert tps > 0 and units >= 1 and "heads of one sequence" in desc

@@ -18,11 +18,19 @@ def test_bench_json_line():
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
         assert key in line, key
-    assert line["value"] > 0 and line["e2e"]["value"] > 0
+    assert line["value"] > 0 and line["e2e"]["value"] > 0 and line["e2e"]["eager_value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] > 0 and line["e2e"]["d2h_bytes_per_step"] > 0
     roof = line["roofline"]
     assert roof["bound"] == "hbm" and 0 < roof["frac"] < 1.5
-    assert line["config"]["workload"] == "v2_b32_l4096"
+    # the headline is the largest single-GPU workload; the other four sit under `workloads`
+    assert line["config"]["workload"] == "ragged_paged_b64"
+    others = line["workloads"]
+    assert sorted(others) == ["long_b4_l32768", "single_l131072_lognormal", "tiny_h16_l256",
+                              "v2_b32_l4096"]
+    for name, o in others.items():
+        assert o["tokens_per_s"] > 0 and o["attn_us"] > 0, name
+        assert 0 < o["roofline"]["frac"] < 1.5 and o["e2e"]["value"] > 0, name
+        assert o["config"]["workload"] == name
     assert line["gpu_launches"] == 5 * 5
     app = line["append_kv"]
     assert app["us"] > 0 and 0 < app["frac_of_hbm"] < 1.5 and app["gpu_launches"] == 2 * 5

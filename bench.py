@@ -469,6 +469,82 @@ def fp8_cache_measure(h, w, g, stream, args, world, local, dev):
             "gpu_launches": 3 * args.steps}
 
 
+def quantise_weight_e4m3(w: torch.Tensor):
+    """Input preparation for the FP8-weight measurement: a bf16 weight [n_h, 128, 512] as E4M3
+    codes [n_h * 128, 512] and one power-of-two exponent per 1 x 128 tile [n_h * 128, 4] (the
+    smallest e with max|tile| / 2^e <= 448; codes by torch's float8_e4m3fn cast)."""
+    rows = w.detach().double().reshape(-1, 4, 128)
+    amax = rows.abs().amax(dim=2)
+    e = torch.where(amax > 0, torch.ceil(torch.log2(amax / 448.0)), torch.zeros_like(amax))
+    e = e + (amax / torch.exp2(e) > 448.0).double()
+    e = e - ((amax > 0) & (amax / torch.exp2(e - 1) <= 448.0)).double()
+    codes = (rows / torch.exp2(e)[:, :, None]).float().to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.reshape(-1, 512).contiguous(), e.to(torch.int8).contiguous()
+
+
+def head_gemm_measure(b, args, world, local, dev):
+    """The two head projections alone (absorb + RoPE, and W_UV), bf16 and FP8 weights, each
+    timed from a graph of K calls over rotating weight copies (4x L2 in total, so every call
+    reads its weights from HBM). Algorithmic bytes: the weights (bf16: 2 B per element; FP8:
+    1 B + one exponent byte per 128) plus the call's inputs and outputs."""
+    w, g, h, stream = b.w, b.g, b.h, b.stream
+    B, H = w.batch, w.n_heads
+    hbm_gbs, _, peak_kind = measured_peaks()
+    q_abs = torch.empty((B, H, 576), dtype=torch.bfloat16, device=dev)
+    latent = wl.draw_latent(B, H, seed=12).to(dev)
+    out = torch.empty((B, H, 128), dtype=torch.bfloat16, device=dev)
+    res = {}
+    for kind in ("bf16", "fp8"):
+        if kind == "bf16":
+            wk, wv = g.w_uk, g.w_uv
+            wbytes = wk.numel() * 2
+        else:
+            wk, wv = quantise_weight_e4m3(g.w_uk), quantise_weight_e4m3(g.w_uv)
+            wbytes = wk[0].numel() + wk[1].numel()
+        n = max(1, math.ceil(4 * L2_BYTES / wbytes))
+        clone = (lambda t: t.clone()) if kind == "bf16" else (lambda t: (t[0].clone(), t[1].clone()))
+        wks = [wk] + [clone(wk) for _ in range(n - 1)]
+        wvs = [wv] + [clone(wv) for _ in range(n - 1)]
+        if kind == "bf16":
+            fa = lambda k: h.absorb_q(g.q_c, g.q_r, wks[k % n], g.kv_lens, q_abs, stream)
+            fv = lambda k: h.apply_wuv(latent, wvs[k % n], out, stream)
+        else:
+            fa = lambda k: h.absorb_q_fp8(g.q_c, g.q_r, wks[k % n][0], wks[k % n][1], g.kv_lens, q_abs, stream)
+            fv = lambda k: h.apply_wuv_fp8(latent, wvs[k % n][0], wvs[k % n][1], out, stream)
+        ms_a = graph_ms(fa, stream, args, world, local, dev)
+        ms_v = graph_ms(fv, stream, args, world, local, dev)
+        h.check_device_errors(stream)
+        io_a = B * H * (128 + 64 + 576) * 2
+        io_v = B * H * (512 + 128) * 2
+        for name, ms, io in (("absorb", ms_a, io_a), ("wuv", ms_v, io_v)):
+            algo = wbytes + io
+            gbs = algo / (ms * 1e-3) / 1e9
+            res[f"{name}_{kind}"] = {"us": ms * 1e3, "algorithmic_bytes": algo, "achieved_gbs": gbs,
+                                     "frac_of_hbm": gbs / hbm_gbs}
+        del wks, wvs
+    res["peak_source"] = f"{peak_kind} hbm_gbs"
+    res["l2"] = "rotating weight copies, 4x L2 in total"
+    res["gpu_launches"] = 8 * args.steps
+    return res
+
+
+def fp8_weight_step_ms(b, args, world, local, dev):
+    """The whole step (absorb, attention, W_UV) with FP8 W_UK / W_UV, timed like the step."""
+    g, h, stream, bufs = b.g, b.h, b.stream, b.bufs
+    uk, uv = quantise_weight_e4m3(g.w_uk), quantise_weight_e4m3(g.w_uv)
+
+    def step(k):
+        q_abs = h.absorb_q_fp8(g.q_c, g.q_r, uk[0], uk[1], g.kv_lens, bufs["q_abs"], stream)
+        h.decode_attn(q_abs, b.caches[k % b.copies], g.kv_lens, g.page_table, bufs["latent"],
+                      None, want_lse=False, stream=stream)
+        h.apply_wuv_fp8(bufs["latent"], uv[0], uv[1], bufs["out"], stream)
+
+    ms = graph_ms(step, stream, args, world, local, dev)
+    h.check_device_errors(stream)
+    return {"ms_per_step": ms, "tokens_per_s": job_tokens_per_s(world, b.w.batch, ms),
+            "weights": "E4M3 codes + one power-of-two scale per 1 x 128 tile", "gpu_launches": 5 * args.steps}
+
+
 class DecodeBench:
     """One workload on this GPU: its inputs in HBM, the rotating cache copies, a handle, and
     the timings of the step, of the attention call alone, and of the step end to end."""
@@ -709,6 +785,8 @@ def run_ours(args):
     tokens = multi_token_measure(w, main.g, main.caches, main.copies, main.stream, args, world,
                                  local, dev)
     fp8 = fp8_cache_measure(main.h, w, main.g, main.stream, args, world, local, dev)
+    heads = head_gemm_measure(main, args, world, local, dev)
+    fp8w = fp8_weight_step_ms(main, args, world, local, dev)
     roof = main.roofline(attn_ms)
     main.close()
     del main
@@ -763,6 +841,8 @@ def run_ours(args):
     line["append_kv"] = append
     line["multi_token"] = tokens
     line["fp8_cache"] = fp8
+    line["head_gemms"] = heads
+    line["fp8_weights"] = fp8w
     if others:
         line["workloads"] = others
     if cpu is not None:

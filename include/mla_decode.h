@@ -214,6 +214,27 @@ MLA_API int mla_apply_wuv(mla_handle_t h, int32_t batch, const void* latent, con
                   void* out, mla_stream_t stream);
 
 /*
+ * FP8 weights for the two head projections ([V3-walk] section 4.4: weights quantised in
+ * 1 x 128 tiles with high-precision accumulation; section 5.5: FP8 for storage with the
+ * arithmetic in BF16 is the safe first step; [V2-notes] "Inference cost": the deployed model
+ * converts its parameters to FP8). A weight W [n_h * 128, 512] (W_UK or W_UV as nn.Linear
+ * weights, the [n_h, 128, 512] arrays above) is given as
+ *   w_codes  uint8 [n_h * 128, 512]: E4M3 codes (OCP FP8 E4M3: bias 7, no infinities, code
+ *            0x7F/0xFF NaN), 16-byte aligned;
+ *   w_exp    int8  [n_h * 128, 4]:   one exponent e per 1 x 128 tile, the tile of row r
+ *            covering latent columns [128 t, 128 t + 128); e in -126..127;
+ * and stands for W[r, c] = value(w_codes[r, c]) * 2^w_exp[r, c / 128]. Each such value is a
+ * bf16 number, so the results are those of mla_absorb_q / mla_apply_wuv on the dequantised
+ * weights (the same products, accumulated in fp32). Other arguments and errors as there.
+ */
+MLA_API int mla_absorb_q_fp8(mla_handle_t h, int32_t batch, const void* q_c, const void* q_r,
+                     const void* w_uk_codes, const int8_t* w_uk_exp, const int32_t* kv_lens,
+                     void* q_abs, mla_stream_t stream);
+
+MLA_API int mla_apply_wuv_fp8(mla_handle_t h, int32_t batch, const void* latent, const void* w_uv_codes,
+                      const int8_t* w_uv_exp, void* out, mla_stream_t stream);
+
+/*
  * Cache write of the step's new token ([V2-arch] eq. 9 c^KV = W^DKV h; [V2-notes]
  * architecture: an RMSNorm follows the compressed latent; [V3-walk] §2.2 k^R = RoPE(W^KR h)
  * and only c^KV and k^R are cached):

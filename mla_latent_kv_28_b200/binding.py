@@ -63,6 +63,8 @@ SIGNATURES = {
     "mla_absorb_q": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P, _P, _P]),
     "mla_decode_attn": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32, _P, _P, _P]),
     "mla_apply_wuv": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P]),
+    "mla_absorb_q_fp8": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P, _P, _P, _P]),
+    "mla_apply_wuv_fp8": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P, _P]),
     "mla_append_kv_fp8": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _P, _P, ctypes.c_float, _P, _P,
                                          _I64, _I64, _P, _P, _I32, _I32, _P]),
     "mla_decode_attn_fp8": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32, _P, _P, _P]),
@@ -369,6 +371,46 @@ class MlaDecode:
         _need(out, torch.bfloat16, "out")
         _check(self._lib.mla_apply_wuv(self._h, B, _ptr(latent), _ptr(w_uv), _ptr(out),
                                        _stream(stream)), "mla_apply_wuv")
+        return out
+
+    @staticmethod
+    def _fp8_weight(codes: torch.Tensor, exps: torch.Tensor, n_heads: int, what: str):
+        if not codes.is_cuda or codes.dtype != torch.uint8 or not codes.is_contiguous() or \
+                codes.numel() != n_heads * 128 * D_LATENT:
+            raise ValueError(f"{what} codes: expected a contiguous CUDA uint8 [n_h * 128, 512] tensor")
+        if not exps.is_cuda or exps.dtype != torch.int8 or not exps.is_contiguous() or \
+                exps.numel() != n_heads * 128 * (D_LATENT // 128):
+            raise ValueError(f"{what} exponents: expected a contiguous CUDA int8 [n_h * 128, 4] tensor")
+
+    def absorb_q_fp8(self, q_c: torch.Tensor, q_r: torch.Tensor, w_uk_codes: torch.Tensor,
+                     w_uk_exp: torch.Tensor, kv_lens: torch.Tensor,
+                     q_abs: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """absorb_q with W_UK as E4M3 codes [n_h * 128, 512] and one int8 exponent per 1 x 128
+        tile [n_h * 128, 4] (W = value(code) * 2^exp)."""
+        B = q_c.shape[0]
+        for t, n in ((q_c, "q_c"), (q_r, "q_r")):
+            _need(t, torch.bfloat16, n)
+        _need(kv_lens, torch.int32, "kv_lens")
+        self._fp8_weight(w_uk_codes, w_uk_exp, self.cfg.n_heads, "w_uk")
+        if q_abs is None:
+            q_abs = torch.empty(tuple(q_c.shape[:-1]) + (ROW,), dtype=torch.bfloat16, device=q_c.device)
+        _need(q_abs, torch.bfloat16, "q_abs")
+        _check(self._lib.mla_absorb_q_fp8(self._h, B, _ptr(q_c), _ptr(q_r), _ptr(w_uk_codes),
+                                          _ptr(w_uk_exp), _ptr(kv_lens), _ptr(q_abs), _stream(stream)),
+               "mla_absorb_q_fp8")
+        return q_abs
+
+    def apply_wuv_fp8(self, latent: torch.Tensor, w_uv_codes: torch.Tensor, w_uv_exp: torch.Tensor,
+                      out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """apply_wuv with W_UV as E4M3 codes and per-tile exponents (as absorb_q_fp8)."""
+        B = latent.shape[0]
+        _need(latent, torch.bfloat16, "latent")
+        self._fp8_weight(w_uv_codes, w_uv_exp, self.cfg.n_heads, "w_uv")
+        if out is None:
+            out = torch.empty(tuple(latent.shape[:-1]) + (128,), dtype=torch.bfloat16, device=latent.device)
+        _need(out, torch.bfloat16, "out")
+        _check(self._lib.mla_apply_wuv_fp8(self._h, B, _ptr(latent), _ptr(w_uv_codes), _ptr(w_uv_exp),
+                                           _ptr(out), _stream(stream)), "mla_apply_wuv_fp8")
         return out
 
     def step(self, q_c, q_r, w_uk, w_uv, cache, kv_lens, page_table=None, stream=None,

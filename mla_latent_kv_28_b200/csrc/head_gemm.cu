@@ -12,7 +12,15 @@
 // into separate accumulators: one 128-feature block each for the absorption, one quarter of
 // the 512-long reduction each for W_UV (the epilogue adds the four). The tile leaves tensor
 // memory through shared memory and TMA stores.
+//
+// FP8 weights: E4M3 codes with one power-of-two scale 2^e per 1 x 128 tile of a weight row
+// (row r of the [n_h * 128, 512] matrix, latent columns [128 t, 128 t + 128)). The codes of each
+// 64-column box land by TMA in the upper half of that box's bf16 slot and all threads expand
+// them in place, four boxes at a time (every thread reads its codes of the four boxes, the CTA
+// meets, then the threads write the bf16 rows): E4M3 values times a power of two are exact in
+// bf16, so the MMAs see exactly the dequantised weights and accumulate in fp32 as with bf16.
 #include <cudaTypedefs.h>
+#include <cuda_fp16.h>
 
 #include <algorithm>
 #include <cmath>
@@ -30,6 +38,7 @@ constexpr int kThreads = 256;   // 8 warps: 4 MMA issuers, all 8 in the epilogue
 constexpr int kIssuers = 4;
 constexpr uint32_t kWeightBox = 128 * 128;      // 128 rows x 64 columns bf16 = 16 KB
 constexpr uint32_t kWeightBytes = 8 * kWeightBox;  // one head's 128 x 512 matrix
+constexpr uint32_t kCodeBox = kWeightBox / 2;      // FP8: 128 rows x 64 codes of one box
 
 enum Mode { kAbsorb = 0, kUpProject = 1 };
 
@@ -38,6 +47,7 @@ struct GemmParams {
   int q_len;                      // one (sequence, new token): row = sequence * q_len + token
   uint32_t idesc;
   __nv_bfloat16* out;             // q_abs [B, n_h, 576] or out [B, n_h, 128]
+  const int8_t* w_exp;            // FP8: exponents [n_h * 128, 4]
   const __nv_bfloat16* q_r;       // absorb only
   const int32_t* kv_lens;         // absorb only
   double theta[kDRope / 2];       // absorb only: RoPE frequencies base^(-2m/d_R), 0 when off
@@ -57,9 +67,10 @@ __device__ __forceinline__ bool wait_simple(uint32_t bar, uint32_t parity, const
 }
 
 // RoPE of the decoupled query of this head for the CTA's rows, rotated to the row's token
-// position max(kv_len - q_len + token, 0) (kv_len - 1 for one new token). The angle pos * theta_m reaches ~1.3e5 rad at 128K tokens, so it is formed in
-// double and brought into [-pi, pi] by Cody-Waite reduction with a two-term 2*pi before the
-// sine and cosine are taken; the result is exact to far below bf16 resolution.
+// position max(kv_len - q_len + token, 0) (kv_len - 1 for one new token). The angle
+// pos * theta_m reaches ~1.3e5 rad at 128K tokens, so it is formed in double and brought into
+// [-pi, pi] by Cody-Waite reduction with a two-term 2*pi; the sine and cosine of the reduced
+// angle are taken in single precision (about 1e-7 off, far below bf16 resolution).
 __device__ __forceinline__ void rope_rows(const GemmParams& p, int h, int b0) {
   constexpr double kTwoPiHi = 6.283185307179586;            // nearest double to 2*pi
   constexpr double kTwoPiLo = 2.4492935982947064e-16;       // 2*pi - kTwoPiHi
@@ -76,8 +87,8 @@ __device__ __forceinline__ void rope_rows(const GemmParams& p, int h, int b0) {
       const double a = (double)pos * p.theta[m];
       const double k = rint(a * kInvTwoPi);
       const double r = fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, a));
-      double sn, cs;
-      sincos(r, &sn, &cs);
+      float sn, cs;
+      sincosf((float)r, &sn, &cs);
       y0 = (double)x0 * cs - (double)x1 * sn;
       y1 = (double)x0 * sn + (double)x1 * cs;
     }
@@ -88,7 +99,54 @@ __device__ __forceinline__ void rope_rows(const GemmParams& p, int h, int b0) {
   }
 }
 
-template <int MODE>
+// Two E4M3 codes (low byte first) -> their values times 2^e as a bf16 pair: E4M3 -> f16 by the
+// hardware conversion (exact), f16 -> f32 (exact), times the power-of-two scale (exact), and
+// bf16 of that (exact: 4 significant bits).
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t codes2, float scale) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((unsigned short)(codes2 & 0xFFFFu)));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+  __nv_bfloat162 b = __floats2bfloat162_rn(f.x * scale, f.y * scale);
+  return *reinterpret_cast<uint32_t*>(&b);
+}
+
+// FP8: the head's codes (box i's 128 rows x 64 codes in the upper half of bf16 box i) -> the
+// bf16 boxes (128-byte swizzle), in two rounds of four boxes. Thread t takes row t / 2 and the
+// half t % 2 of its 64 columns (32 codes) in each box.
+__device__ __forceinline__ void expand_weights(uint8_t* smem, const GemmParams& p, int h) {
+  const int t = threadIdx.x, row = t >> 1, half = t & 1;
+#pragma unroll 1
+  for (int round = 0; round < 2; ++round) {
+    uint4 c[4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+        c[i][k] = *reinterpret_cast<const uint4*>(smem + (4 * round + i) * kWeightBox + kCodeBox + row * 64 + half * 32 + 16 * k);
+    float scale[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {   // the two 128-column tiles of this round's boxes
+      const int e = p.w_exp[((int64_t)h * kDHead + row) * (kDLatent / 128) + 2 * round + q];
+      scale[q] = __uint_as_float((uint32_t)(min(max(e, -126), 127) + 127) << 23);
+    }
+    __syncthreads();   // every code of these boxes is read before any of them is overwritten
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {   // 16-byte chunk half * 4 + k of the row: 8 columns
+        const uint4 w = c[i][k >> 1];
+        const uint32_t lo = (k & 1) ? w.z : w.x, hi = (k & 1) ? w.w : w.y;
+        const float sc = scale[i >> 1];
+        const int chunk = half * 4 + k;
+        *reinterpret_cast<uint4*>(smem + (4 * round + i) * kWeightBox + row * 128 + ((chunk ^ (row & 7)) << 4)) =
+            make_uint4(e4m3x2_to_bf16x2(lo, sc), e4m3x2_to_bf16x2(lo >> 16, sc),
+                       e4m3x2_to_bf16x2(hi, sc), e4m3x2_to_bf16x2(hi >> 16, sc));
+      }
+  }
+  fence_proxy_async_smem();   // read by the MMAs (async proxy)
+}
+
+template <int MODE, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
 head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
              const __grid_constant__ CUtensorMap tmap_o, const GemmParams p) {
@@ -121,7 +179,7 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
     prefetch_tmap(&tmap_o);
     // the head's weights into L2 while the previous kernel finishes (a hint only: L2 is
     // where writes land, so it cannot return stale data)
-    for (int i = 0; i < 8; ++i) tma_prefetch_2d(&tmap_w, 64 * i, 128 * h);
+    for (int i = 0; i < 8; ++i) tma_prefetch_2d(&tmap_w, 64 * i, 128 * h);   // FP8: 64 codes per box
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), tmem_cols);
@@ -136,16 +194,27 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
 
   bool ok = true;
   if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(bars, kWeightBytes + kXBoxes * xbox);
-    for (int i = 0; i < 8; ++i) tma_load_2d(sbase + i * kWeightBox, &tmap_w, 64 * i, 128 * h, bars);
+    mbar_arrive_expect_tx(bars, (FP8 ? 8 * kCodeBox : kWeightBytes) + kXBoxes * xbox);
+    for (int i = 0; i < 8; ++i)
+      tma_load_2d(sbase + i * kWeightBox + (FP8 ? kCodeBox : 0), &tmap_w, 64 * i, 128 * h, bars);
     const int xcol = h * (MODE == kAbsorb ? kDHead : kDLatent);
     for (int i = 0; i < kXBoxes; ++i) tma_load_2d(xbase + i * xbox, &tmap_x, xcol + 64 * i, b0, bars);
   }
   if (MODE == kAbsorb) rope_rows(p, h, b0);   // needs no weights: runs while they load
   volatile int* ok_flags = reinterpret_cast<volatile int*>(smem + (bars - sbase) + 8 * (1 + kIssuers) + 4);
+  bool landed = true;   // FP8: every thread waits for the codes and expands its share
+  if (FP8) {
+    landed = wait_simple(bars, 0, p);
+    if (__syncthreads_and(landed ? 1 : 0)) {
+      expand_weights(smem, p, h);
+    } else {
+      landed = false;
+    }
+    __syncthreads();
+  }
   if (warp < kIssuers && lane == 0) {
     const int q = warp;
-    ok = wait_simple(bars, 0, p);
+    ok = FP8 ? landed : wait_simple(bars, 0, p);
     tc_fence_after();
     if (ok) {
       // absorb: accumulator q = output features [128q, 128q+128), K = 128 (8 steps);
@@ -166,7 +235,7 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
       }
       mma_commit(bars + 8 * (1 + q));
       ok = wait_simple(bars + 8 * (1 + q), 0, p);
-    } else {
+    } else if (!FP8) {
       wait_simple(bars, 0, p);  // never leave with copies in flight
     }
     ok_flags[q] = ok ? 1 : 0;
@@ -251,17 +320,32 @@ bool encode(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE>
-cudaError_t launch(const mla_decode_s& h, int batch, const __nv_bfloat16* w, const __nv_bfloat16* x,
-                   __nv_bfloat16* out, const __nv_bfloat16* q_r, const int32_t* kv_lens,
-                   cudaStream_t s) {
+// The FP8 weight codes [rows, 512] bytes as a TMA source with {64, 128} boxes (no swizzle).
+bool encode_codes(CUtensorMap* m, const void* base, uint64_t rows) {
+  const PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)kDLatent, rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kDLatent};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE, bool FP8>
+cudaError_t launch(const mla_decode_s& h, int batch, const void* w, const int8_t* w_exp,
+                   const __nv_bfloat16* x, __nv_bfloat16* out, const __nv_bfloat16* q_r,
+                   const int32_t* kv_lens, cudaStream_t s) {
   constexpr int kXBoxes = MODE == kAbsorb ? 2 : 8;
   constexpr int kCap = MODE == kAbsorb ? 128 : 64;  // weights + x boxes fit in shared memory
   const int n_tile = std::min(kCap, (batch + 15) / 16 * 16);
   const int kx = MODE == kAbsorb ? kDHead : kDLatent;
   const int ko = MODE == kAbsorb ? kRow : kDHead;   // output row of one head
   CUtensorMap tw, tx, to;
-  if (!encode(&tw, w, (uint64_t)h.cfg.n_heads * kDHead, kDLatent, 128) ||
+  const bool w_ok = FP8 ? encode_codes(&tw, w, (uint64_t)h.cfg.n_heads * kDHead)
+                        : encode(&tw, w, (uint64_t)h.cfg.n_heads * kDHead, kDLatent, 128);
+  if (!w_ok ||
       !encode(&tx, x, (uint64_t)batch, (uint64_t)h.cfg.n_heads * kx, (uint32_t)n_tile) ||
       !encode(&to, out, (uint64_t)batch, (uint64_t)h.cfg.n_heads * ko, (uint32_t)n_tile,
               CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -270,7 +354,7 @@ cudaError_t launch(const mla_decode_s& h, int batch, const __nv_bfloat16* w, con
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(head_gemm_tc<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr = cudaFuncSetAttribute(head_gemm_tc<MODE, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kSmemMax);
   });
   if (attr != cudaSuccess) return attr;
@@ -281,6 +365,7 @@ cudaError_t launch(const mla_decode_s& h, int batch, const __nv_bfloat16* w, con
   p.q_len = h.q_len;
   p.idesc = idesc_bf16_f32(128, n_tile, MODE == kAbsorb, false);
   p.out = out;
+  p.w_exp = w_exp;
   p.q_r = q_r;
   p.kv_lens = kv_lens;
   for (int m = 0; m < kDRope / 2; ++m)
@@ -289,7 +374,7 @@ cudaError_t launch(const mla_decode_s& h, int batch, const __nv_bfloat16* w, con
   p.wait_limit = 2000000000LL;
   const uint32_t smem = kWeightBytes + kXBoxes * n_tile * 128 + 64 + 1024;
   dim3 grid(h.cfg.n_heads, (batch + n_tile - 1) / n_tile);
-  return launch_pdl(head_gemm_tc<MODE>, grid, dim3(kThreads), smem, s, tw, tx, to, p);
+  return launch_pdl(head_gemm_tc<MODE, FP8>, grid, dim3(kThreads), smem, s, tw, tx, to, p);
 }
 
 }  // namespace
@@ -297,12 +382,25 @@ cudaError_t launch(const mla_decode_s& h, int batch, const __nv_bfloat16* w, con
 cudaError_t launch_absorb_q(const mla_decode_s& h, int batch, const __nv_bfloat16* q_c,
                             const __nv_bfloat16* q_r, const __nv_bfloat16* w_uk,
                             const int32_t* kv_lens, __nv_bfloat16* q_abs, cudaStream_t s) {
-  return launch<kAbsorb>(h, batch, w_uk, q_c, q_abs, q_r, kv_lens, s);
+  return launch<kAbsorb, false>(h, batch, w_uk, nullptr, q_c, q_abs, q_r, kv_lens, s);
 }
 
 cudaError_t launch_apply_wuv(const mla_decode_s& h, int batch, const __nv_bfloat16* latent,
                              const __nv_bfloat16* w_uv, __nv_bfloat16* out, cudaStream_t s) {
-  return launch<kUpProject>(h, batch, w_uv, latent, out, nullptr, nullptr, s);
+  return launch<kUpProject, false>(h, batch, w_uv, nullptr, latent, out, nullptr, nullptr, s);
+}
+
+cudaError_t launch_absorb_q_fp8(const mla_decode_s& h, int batch, const __nv_bfloat16* q_c,
+                                const __nv_bfloat16* q_r, const uint8_t* w_uk_codes,
+                                const int8_t* w_uk_exp, const int32_t* kv_lens,
+                                __nv_bfloat16* q_abs, cudaStream_t s) {
+  return launch<kAbsorb, true>(h, batch, w_uk_codes, w_uk_exp, q_c, q_abs, q_r, kv_lens, s);
+}
+
+cudaError_t launch_apply_wuv_fp8(const mla_decode_s& h, int batch, const __nv_bfloat16* latent,
+                                 const uint8_t* w_uv_codes, const int8_t* w_uv_exp,
+                                 __nv_bfloat16* out, cudaStream_t s) {
+  return launch<kUpProject, true>(h, batch, w_uv_codes, w_uv_exp, latent, out, nullptr, nullptr, s);
 }
 
 }  // namespace mla

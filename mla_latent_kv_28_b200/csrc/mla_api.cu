@@ -382,6 +382,34 @@ int mla_apply_wuv(mla_handle_t h, int32_t batch, const void* latent, const void*
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+int mla_absorb_q_fp8(mla_handle_t h, int32_t batch, const void* q_c, const void* q_r,
+                     const void* w_uk_codes, const int8_t* w_uk_exp, const int32_t* kv_lens,
+                     void* q_abs, mla_stream_t stream) {
+  if (h == nullptr || q_c == nullptr || q_r == nullptr || w_uk_codes == nullptr ||
+      w_uk_exp == nullptr || kv_lens == nullptr || q_abs == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > h->cfg.max_batch) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_c) || !aligned16(q_r) || !aligned16(w_uk_codes) || !aligned16(q_abs))
+    return MLA_ERR_INVALID_ARG;
+  const cudaError_t e = mla::launch_absorb_q_fp8(
+      *h, batch * h->q_len, static_cast<const __nv_bfloat16*>(q_c), static_cast<const __nv_bfloat16*>(q_r),
+      static_cast<const uint8_t*>(w_uk_codes), w_uk_exp, kv_lens, static_cast<__nv_bfloat16*>(q_abs), stream);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_apply_wuv_fp8(mla_handle_t h, int32_t batch, const void* latent, const void* w_uv_codes,
+                      const int8_t* w_uv_exp, void* out, mla_stream_t stream) {
+  if (h == nullptr || latent == nullptr || w_uv_codes == nullptr || w_uv_exp == nullptr ||
+      out == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > h->cfg.max_batch) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(latent) || !aligned16(w_uv_codes) || !aligned16(out)) return MLA_ERR_INVALID_ARG;
+  const cudaError_t e = mla::launch_apply_wuv_fp8(
+      *h, batch * h->q_len, static_cast<const __nv_bfloat16*>(latent),
+      static_cast<const uint8_t*>(w_uv_codes), w_uv_exp, static_cast<__nv_bfloat16*>(out), stream);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 int mla_check_device_errors(mla_handle_t h, mla_stream_t stream, uint32_t* detail) {
   if (h == nullptr) return MLA_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return MLA_ERR_CUDA;

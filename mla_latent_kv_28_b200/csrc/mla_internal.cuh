@@ -147,4 +147,15 @@ cudaError_t launch_append_kv(const mla_decode_s& h, int batch, int d_model,
 cudaError_t launch_apply_wuv(const mla_decode_s& h, int batch, const __nv_bfloat16* latent,
                              const __nv_bfloat16* w_uv, __nv_bfloat16* out, cudaStream_t s);
 
+// FP8 weights: E4M3 codes [n_h * 128, 512] and one power-of-two exponent per 1 x 128 tile
+// [n_h * 128, 4] (the tile of row r covering latent columns [128 t, 128 t + 128)).
+cudaError_t launch_absorb_q_fp8(const mla_decode_s& h, int batch, const __nv_bfloat16* q_c,
+                                const __nv_bfloat16* q_r, const uint8_t* w_uk_codes,
+                                const int8_t* w_uk_exp, const int32_t* kv_lens,
+                                __nv_bfloat16* q_abs, cudaStream_t s);
+
+cudaError_t launch_apply_wuv_fp8(const mla_decode_s& h, int batch, const __nv_bfloat16* latent,
+                                 const uint8_t* w_uv_codes, const int8_t* w_uv_exp,
+                                 __nv_bfloat16* out, cudaStream_t s);
+
 }  // namespace mla

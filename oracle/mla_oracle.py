@@ -306,6 +306,31 @@ def dequantize_rows_fp8(codes, exps) -> np.ndarray:
     return e4m3_decode(codes) * np.exp2(np.asarray(exps, dtype=np.float64))[..., None]
 
 
+def quantize_weight_fp8(w, tile: int = 128):
+    """A projection weight (an nn.Linear weight [rows, d_c], e.g. W_UK or W_UV as
+    [n_h * d_h, d_c]; an [n_h, d_h, d_c] array is taken row by row) as E4M3 codes with one
+    power-of-two scale per 1 x `tile` tile of a row ([V3-walk] section 4.4: weights quantised in
+    1 x 128 tiles): (codes uint8 [rows, d_c], exponents int [rows, d_c / tile]). Each tile's
+    exponent is the smallest e with max|tile| / 2^e <= 448 and its codes the nearest E4M3
+    codes of tile / 2^e (quantize_rows_fp8 applied to the tiles)."""
+    w = widen(w)
+    d_c = w.shape[-1]
+    rows = w.reshape(-1, d_c)
+    codes, exps = quantize_rows_fp8(rows.reshape(-1, tile))
+    return codes.reshape(rows.shape).astype(np.uint8), exps.reshape(rows.shape[0], d_c // tile)
+
+
+def dequantize_weight_fp8(codes, exps, d_head: int = D_HEAD) -> np.ndarray:
+    """The weight in float64 [rows / d_head, d_head, d_c] from its E4M3 codes [rows, d_c] and
+    tile exponents [rows, d_c / tile]: W[r, c] = value(code[r, c]) * 2^exp[r, c // tile]."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    exps = np.asarray(exps, dtype=np.float64)
+    rows, d_c = codes.shape
+    tile = d_c // exps.shape[1]
+    w = e4m3_decode(codes).reshape(rows, d_c // tile, tile) * np.exp2(exps)[:, :, None]
+    return w.reshape(rows // d_head, d_head, d_c)
+
+
 def default_scale(d_head: int = D_HEAD, d_rope: int = D_ROPE, yarn: Optional[Yarn] = None) -> float:
     """1/sqrt(d_h + d_h^R) (the reading of the softmax scale, module doc), times the YaRN
     score factor t when YaRN is on."""

@@ -52,3 +52,17 @@ def workload_np(w):
                 cache=to_np(w.cache), kv_lens=w.kv_lens.cpu().numpy(),
                 page_table=None if w.page_table is None else w.page_table.cpu().numpy(),
                 page_size=w.page_size)
+
+
+def quantise_weight_e4m3(w: torch.Tensor):
+    """Test input preparation: a bf16 weight [n_h, 128, 512] as E4M3 codes [n_h * 128, 512]
+    and one power-of-two exponent per 1 x 128 tile [n_h * 128, 4] (the smallest e with
+    max|tile| / 2^e <= 448; codes by torch's float8_e4m3fn cast, round to nearest even).
+    tests/test_gpu_fp8_weights.py checks both against the oracle's quantiser on samples."""
+    rows = w.detach().cpu().double().reshape(-1, 4, 128)
+    amax = rows.abs().amax(dim=2)
+    e = torch.where(amax > 0, torch.ceil(torch.log2(amax / 448.0)), torch.zeros_like(amax))
+    e = e + (amax / torch.exp2(e) > 448.0).double()
+    e = e - ((amax > 0) & (amax / torch.exp2(e - 1) <= 448.0)).double()
+    codes = (rows / torch.exp2(e)[:, :, None]).float().to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.reshape(-1, 512).contiguous(), e.to(torch.int8).contiguous()

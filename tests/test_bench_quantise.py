@@ -20,3 +20,13 @@ def test_bench_quantiser_matches_the_oracle():
         assert np.array_equal(oracle.e4m3_encode(r / 2.0 ** e), codes.view(-1, 576)[i].numpy())
         checked += 1
     assert checked == 70 + 5 + 130
+
+
+def test_bench_weight_quantiser_matches_the_oracle():
+    """The FP8-weight input preparation (1 x 128 tiles) gives the oracle's tile exponents and
+    codes: oracle.quantize_weight_fp8 on a small weight, element by element."""
+    w = wl.make_workload(1, 2, [4], seed=3).w_uk          # [2, 128, 512] bf16
+    codes, exps = bench.quantise_weight_e4m3(w)
+    ref_codes, ref_exps = oracle.quantize_weight_fp8(w.float().numpy())
+    assert np.array_equal(exps.numpy().astype(np.int64), ref_exps)
+    assert np.array_equal(codes.numpy(), ref_codes)

@@ -36,5 +36,9 @@ def test_bench_json_line():
     assert app["us"] > 0 and 0 < app["frac_of_hbm"] < 1.5 and app["gpu_launches"] == 2 * 5
     mt = line["multi_token"]
     assert mt["q_len"] == 8 and mt["attn_us"] > 0 and mt["query_tokens_per_s"] > 0
+    hg = line["head_gemms"]
+    for k in ("absorb_bf16", "wuv_bf16", "absorb_fp8", "wuv_fp8"):
+        assert hg[k]["us"] > 0 and 0 < hg[k]["frac_of_hbm"] < 1.5, k
+    assert line["fp8_weights"]["tokens_per_s"] > 0
     q8 = line["fp8_cache"]
     assert q8["attn_us"] > 0 and 0 < q8["frac_of_hbm"] < 1.5

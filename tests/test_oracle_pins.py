@@ -642,3 +642,32 @@ def test_fp8_rows_quantise_within_half_a_step():
         assert 224.0 < amax / 2.0 ** e <= 448.0          # the smallest exponent that fits
         step = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(r) / 2.0 ** e, 2.0 ** -6))) - 3) * 2.0 ** e
         assert np.all(np.abs(d - r) <= step / 2 * (1 + 1e-12))
+
+
+def test_fp8_weight_tiles_have_their_own_scale_and_dequantise_within_half_a_step():
+    """FP8 weights: one power-of-two scale per 1 x 128 tile of a weight row (DeepSeek-V3
+    walkthrough, section 4.4). A tile's exponent depends on its own 128 values only (a row
+    with one large tile keeps its small tiles' resolution), and the dequantised weight is
+    within half an E4M3 step of the original everywhere."""
+    rng = np.random.default_rng(92)
+    w = rng.standard_normal((2, 4, 512)) / math.sqrt(512)      # 2 heads of d_h = 4 rows
+    w[0, 1, 128:256] *= 1000.0                                   # one large tile in row 1
+    codes, exps = oracle.quantize_weight_fp8(w)
+    assert codes.shape == (8, 512) and exps.shape == (8, 4)
+    rows = w.reshape(8, 512)
+    for r in range(8):
+        for t in range(4):
+            tile = rows[r, 128 * t:128 * (t + 1)]
+            assert exps[r, t] == oracle.fp8_row_exponent(tile)
+    assert exps[1, 1] - exps[1, 0] >= 9                          # the large tile's own scale
+    deq = oracle.dequantize_weight_fp8(codes, exps, d_head=4)
+    assert deq.shape == (2, 4, 512)
+    full = deq.reshape(8, 512)
+    for r in range(8):
+        for t in range(4):
+            e = exps[r, t]
+            x = rows[r, 128 * t:128 * (t + 1)]
+            step = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(x) / 2.0 ** e, 2.0 ** -6))) - 3) * 2.0 ** e
+            assert np.all(np.abs(full[r, 128 * t:128 * (t + 1)] - x) <= step / 2 * (1 + 1e-12))
+    # the codes decode to exactly value(code) * 2^e: a table lookup of the E4M3 definition
+    assert full[0, 0] == oracle.e4m3_value(int(codes[0, 0])) * 2.0 ** exps[0, 0]

@@ -181,6 +181,16 @@ def measured_peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+def sustained_tensor_peak():
+    """bf16 dense TFLOP/s for a kernel timed inside a long loop: the measured sustained figure,
+    else the fallback (about 1.4 PFLOP/s under the power cap)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured bf16_tflops_sustained"
+    return 1400.0, "fallback 1400 TFLOP/s"
+
+
 def kernel_sources_sha() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mla_latent_kv_28_b200", "csrc")
@@ -545,6 +555,31 @@ def fp8_weight_step_ms(b, args, world, local, dev):
             "weights": "E4M3 codes + one power-of-two scale per 1 x 128 tile", "gpu_launches": 5 * args.steps}
 
 
+def prefill_measure(args, world, local, dev, T: int = 2048, n_heads: int = 128):
+    """Prefill: one prompt of T new tokens (the whole cache: kv_len = T) through
+    mla_prefill_attn, timed from a graph of K calls. Its work is a contraction (each cache row
+    is read by 128 rows of one head at once and stays in L2), so it is reported against the
+    tensor peak: FLOPs = sum over tokens of visible rows x n_h x 2 x (576 + 512)."""
+    from mla_latent_kv_28_b200 import binding
+    w = wl.make_workload(1, n_heads, [T], seed=13)
+    g = w.to(dev)
+    q = wl.draw_q_abs(T, n_heads, seed=14).view(1, T, n_heads, 576).to(dev)
+    h = binding.MlaDecode(n_heads, 1, T, q_len=T)
+    lat = torch.empty((1, T, n_heads, 512), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.Stream(dev)
+    ms = graph_ms(lambda k: h.prefill_attn(q, g.cache, g.kv_lens, None, lat, None, want_lse=False,
+                                           stream=stream), stream, args, world, local, dev)
+    h.check_device_errors(stream)
+    h.close()
+    flops = sum(t + 1 for t in range(T)) * n_heads * 2 * (576 + 512)
+    peak_s, kind = sustained_tensor_peak()
+    tflops = flops / (ms * 1e-3) / 1e12
+    return {"prompt_tokens": T, "n_heads": n_heads, "us": ms * 1e3,
+            "tokens_per_s": world * T / (ms * 1e-3), "tflops": tflops,
+            "tensor_frac": tflops / peak_s, "peak_source": kind,
+            "flops": flops, "gpu_launches": args.steps}
+
+
 class DecodeBench:
     """One workload on this GPU: its inputs in HBM, the rotating cache copies, a handle, and
     the timings of the step, of the attention call alone, and of the step end to end."""
@@ -786,6 +821,7 @@ def run_ours(args):
                                  local, dev)
     fp8 = fp8_cache_measure(main.h, w, main.g, main.stream, args, world, local, dev)
     heads = head_gemm_measure(main, args, world, local, dev)
+    prefill = prefill_measure(args, world, local, dev)
     fp8w = fp8_weight_step_ms(main, args, world, local, dev)
     roof = main.roofline(attn_ms)
     main.close()
@@ -842,6 +878,7 @@ def run_ours(args):
     line["multi_token"] = tokens
     line["fp8_cache"] = fp8
     line["head_gemms"] = heads
+    line["prefill"] = prefill
     line["fp8_weights"] = fp8w
     if others:
         line["workloads"] = others

@@ -90,9 +90,11 @@ typedef struct {
    * lse [batch, T, n_h], latent/out of mla_apply_wuv, hidden [batch, T, d] of
    * mla_append_kv); kv_lens counts the T new tokens, which sit at positions kv_len - T + t;
    * token t attends to rows 0 .. kv_len - T + t (a token with none: latent 0, lse -inf) and
-   * its q^R is rotated at max(kv_len - T + t, 0). Limits: n_heads * T <= 1024 and
-   * max_batch * T <= 1024; mla_decode_attn runs more than 128 attention rows per sequence in
-   * groups of 128, each reading the cache. */
+   * its q^R is rotated at max(kv_len - T + t, 0). Limits: n_heads * T <= 2^20 and
+   * max_batch * T <= 8192 (the cache write's workspace holds max_batch * T rows of 2.3 KB
+   * each); mla_decode_attn runs more than 128 attention rows per sequence in groups of 128,
+   * each reading the cache, which suits a few draft tokens; a long prompt (prefill) goes
+   * through mla_prefill_attn. */
   int32_t q_len;
 } mla_config_t;
 
@@ -159,6 +161,25 @@ MLA_API int mla_decode_attn(mla_handle_t h, int32_t batch, const void* q_abs, co
                     const void* k_r, int64_t row_stride, int64_t seq_stride,
                     const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
                     int32_t num_pages, void* out_latent, float* lse, mla_stream_t stream);
+
+/*
+ * Prefill: the attention of a prompt's T = q_len new tokens over the latent cache, the same
+ * results as mla_decode_attn with this handle (token t of sequence b attends to cache rows
+ * 0 .. kv_len[b] - T + t, the causal mask of [V2-arch]'s MHA equations, softmax over j = 1..t)
+ * for long prompts ([V2-notes] "Inference cost": prompt input throughput is a headline figure
+ * of the deployed model). One kernel: each work item is one head and 128 consecutive new tokens
+ * of one sequence (128 attention rows sharing every cache row they read), taken whole by one
+ * 2-CTA cluster over the rows its last token sees, with the normalised latent written directly
+ * (no split partials, no merge).
+ *   q_abs      bf16 [batch, T, n_h, 576] (mla_absorb_q with this handle)
+ *   cache      as for mla_decode_attn (bf16 only)
+ *   out_latent bf16 [batch, T, n_h, 512]; lse fp32 [batch, T, n_h] or NULL
+ * A token that sees no row gets latent 0 and lse -inf. Errors as for mla_decode_attn.
+ */
+MLA_API int mla_prefill_attn(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
+                     const void* k_r, int64_t row_stride, int64_t seq_stride,
+                     const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                     int32_t num_pages, void* out_latent, float* lse, mla_stream_t stream);
 
 /*
  * mla_decode_attn over a quantised cache ([V2-notes] Inference cost: the deployed KV cache is

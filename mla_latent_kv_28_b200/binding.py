@@ -63,6 +63,7 @@ SIGNATURES = {
     "mla_absorb_q": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P, _P, _P]),
     "mla_decode_attn": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32, _P, _P, _P]),
     "mla_apply_wuv": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P]),
+    "mla_prefill_attn": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32, _P, _P, _P]),
     "mla_absorb_q_fp8": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P, _P, _P, _P]),
     "mla_apply_wuv_fp8": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P, _P]),
     "mla_append_kv_fp8": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _P, _P, ctypes.c_float, _P, _P,
@@ -282,6 +283,28 @@ class MlaDecode:
             self._h, B, _ptr(q_abs), ctypes.c_void_p(c_kv), ctypes.c_void_p(k_r), row_stride,
             seq_stride, _ptr(kv_lens), _ptr(page_table), max_pages, num_pages, _ptr(out_latent),
             _ptr(lse), _stream(stream)), "mla_decode_attn")
+        return out_latent, lse
+
+    def prefill_attn(self, q_abs: torch.Tensor, cache: torch.Tensor, kv_lens: torch.Tensor,
+                     page_table: Optional[torch.Tensor] = None,
+                     out_latent: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                     want_lse: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+        """Prefill: the handle's q_len new tokens of every sequence, q_abs [B, T, n_h, 576], over
+        the cache (as decode_attn), in one kernel. Returns (out_latent [B, T, n_h, 512] bf16,
+        lse [B, T, n_h] fp32 or None); the same results as decode_attn with this handle."""
+        B = q_abs.shape[0]
+        _need(q_abs, torch.bfloat16, "q_abs")
+        _need(kv_lens, torch.int32, "kv_lens")
+        row_stride, seq_stride, c_kv, k_r, max_pages, num_pages = self._cache_view(cache, page_table)
+        if out_latent is None:
+            out_latent = torch.empty(tuple(q_abs.shape[:-1]) + (D_LATENT,), dtype=torch.bfloat16,
+                                     device=q_abs.device)
+        if lse is None and want_lse:
+            lse = torch.empty(tuple(q_abs.shape[:-1]), dtype=torch.float32, device=q_abs.device)
+        _check(self._lib.mla_prefill_attn(
+            self._h, B, _ptr(q_abs), ctypes.c_void_p(c_kv), ctypes.c_void_p(k_r), row_stride,
+            seq_stride, _ptr(kv_lens), _ptr(page_table), max_pages, num_pages, _ptr(out_latent),
+            _ptr(lse), _stream(stream)), "mla_prefill_attn")
         return out_latent, lse
 
     def decode_attn_fp8(self, q_abs: torch.Tensor, codes: torch.Tensor, exps: torch.Tensor,

@@ -49,6 +49,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include "mla_internal.cuh"
 #include "sm100.cuh"
@@ -144,6 +145,15 @@ struct Params {
   // quantised cache (E4M3 codes + one power-of-two scale per row), else kv_exp == nullptr
   const int8_t* kv_exp;
   int64_t kv_rows;          // rows of the cache, for the bounds of the exponent loads
+  // prefill (the kPrefill instantiation): a work item is one head and 128 consecutive new
+  // tokens of one sequence, taken whole by one cluster, whose latent rows go to the output
+  int q_tokens;             // T, new tokens per sequence
+  int n_blocks;             // 128-token blocks per head: ceil(T / 128)
+  int n_items;              // batch * heads * n_blocks
+  const int32_t* kv_lens;
+  int64_t max_kv_len;
+  __nv_bfloat16* out_latent;   // [B, T, n_h, 512]
+  float* out_lse;              // [B, T, n_h] or nullptr
 };
 
 // Walks this cluster's work tile by tile: units in turn, the segments (one sequence's
@@ -201,6 +211,70 @@ struct TileCursor {
   __device__ __forceinline__ int rows() const { return min(kT, j1 - j()); }
   __device__ __forceinline__ bool first() const { return k == 0; }
   __device__ __forceinline__ bool last() const { return k == nk - 1; }
+  // cache rows attention row `row` sees: new token t of q_len sits at len - q_len + t and does
+  // not see the new tokens after it
+  __device__ __forceinline__ int visible(const Params& p, int row) const {
+    return len - (p.q_len - 1 - (p.row_base + row) / p.heads_per_token);
+  }
+  // the query row of attention row `row` (576 values), or nullptr past the launch's rows
+  __device__ __forceinline__ const __nv_bfloat16* q_row(const Params& p, int row) const {
+    return row < p.n_heads ? p.q_abs + ((int64_t)b * p.q_row_stride + p.row_base + row) * kRow : nullptr;
+  }
+};
+
+// Prefill: this cluster's work items (item u: sequence b, head, token block tb; items
+// cluster_id, cluster_id + clusters, ...), each one segment over the cache rows its block's
+// last token sees. Attention row r of an item is new token t = 128 tb + r of the head.
+struct PrefillCursor {
+  int u, b, head, tb;
+  int slot, len, j0, j1;   // slot: the item; len: the sequence's kv_len
+  int k, nk;
+  uint32_t g, seg;
+  bool valid;
+
+  __device__ __forceinline__ void find(const Params& p) {
+    if (u < p.n_items) {
+      tb = u % p.n_blocks;
+      head = (u / p.n_blocks) % p.heads_per_token;
+      b = u / (p.n_blocks * p.heads_per_token);
+      len = (int)min(max((int64_t)p.kv_lens[b], (int64_t)0), p.max_kv_len);
+      slot = u;
+      j0 = 0;
+      j1 = max(0, min(len, len - p.q_tokens + 128 * (tb + 1)));
+      // an item whose rows see nothing still takes one (empty) tile: its rows get latent 0 and
+      // lse -inf from the same code as every other row
+      nk = max(1, (j1 + kT - 1) / kT);
+      k = 0;
+      valid = true;
+    } else {
+      valid = false;
+    }
+  }
+  __device__ __forceinline__ void init(const Params& p) {
+    u = (int)cluster_id_x();
+    g = 0;
+    seg = 0;
+    find(p);
+  }
+  __device__ __forceinline__ void next(const Params& p) {
+    ++g;
+    if (++k < nk) return;
+    ++seg;
+    u += (int)num_clusters_x();
+    find(p);
+  }
+  __device__ __forceinline__ int j() const { return j0 + kT * k; }
+  __device__ __forceinline__ int rows() const { return min(kT, j1 - j()); }
+  __device__ __forceinline__ bool first() const { return k == 0; }
+  __device__ __forceinline__ bool last() const { return k == nk - 1; }
+  __device__ __forceinline__ int visible(const Params& p, int row) const {
+    const int t = 128 * tb + row;
+    return t < p.q_tokens ? len - p.q_tokens + t + 1 : 0;
+  }
+  __device__ __forceinline__ const __nv_bfloat16* q_row(const Params& p, int row) const {
+    const int t = 128 * tb + row;
+    return t < p.q_tokens ? p.q_abs + (((int64_t)b * p.q_tokens + t) * p.heads_per_token + head) * kRow : nullptr;
+  }
 };
 
 __device__ __forceinline__ bool wait_teardown(uint32_t bar, uint32_t parity, long long limit) {
@@ -233,18 +307,16 @@ __device__ __forceinline__ void q_chunks_out(const uint4 (&v)[12], uint8_t* smem
   }
 }
 
-// One third (12 of the 36 16-byte chunks) of this CTA's 288 query columns of head h of
-// sequence b, to TMEM / shared memory as above.
-__device__ __forceinline__ void load_q_part(const Params& p, uint8_t* smem, uint32_t tmem, uint32_t lanes,
-                                            int h, int b, int part, uint32_t rank) {
-  const bool head_ok = h < p.n_heads;
-  const __nv_bfloat16* qrow = p.q_abs + ((int64_t)b * p.q_row_stride + p.row_base + (head_ok ? h : 0)) * kRow;
+// One third (12 of the 36 16-byte chunks) of this CTA's 288 query columns of attention row h
+// (query row qrow, or zeros when it is nullptr), to TMEM / shared memory as above.
+__device__ __forceinline__ void load_q_part(const __nv_bfloat16* qrow, uint8_t* smem, uint32_t tmem,
+                                            uint32_t lanes, int h, int part, uint32_t rank) {
   uint4 v[12];
 #pragma unroll
   for (int i = 0; i < 12; ++i) {
     const int ci = part * 12 + i;  // 16-byte chunk 0..35 of this CTA's 288 columns
     const int col = ci < 32 ? 256 * (int)rank + 8 * ci : kDLatent + 32 * (int)rank + 8 * (ci - 32);
-    v[i] = head_ok ? *reinterpret_cast<const uint4*>(qrow + col) : make_uint4(0, 0, 0, 0);
+    v[i] = qrow != nullptr ? *reinterpret_cast<const uint4*>(qrow + col) : make_uint4(0, 0, 0, 0);
   }
   q_chunks_out(v, smem, tmem, lanes, h, part);
 }
@@ -291,7 +363,9 @@ __device__ __noinline__ void zero_tail(uint8_t* stage, int r, int tid) {
 
 // kQ8: the cache is quantised (E4M3 codes expanded in shared memory); a separate
 // instantiation, so that the bf16 kernel carries none of that code.
-template <bool kQ8>
+// kPrefill: the work is prefill items (PrefillCursor) instead of the split plan's segments,
+// and each item's latent rows go straight to the output.
+template <bool kQ8, bool kPrefill>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constant__ CUtensorMap tmap_r,
                 const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_qr,
@@ -306,6 +380,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
   volatile int* tile_valid = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);  // [kStages]
   volatile long long* tile_row_s = reinterpret_cast<volatile long long*>(smem + kOffMisc + 24);  // [kStages]
   constexpr bool q8 = kQ8;   // quantised cache
+  using Cursor = std::conditional_t<kPrefill, PrefillCursor, TileCursor>;
   float2* ml = reinterpret_cast<float2*>(smem + kOffMl);                             // [2][2][128]
   volatile float* mh = reinterpret_cast<volatile float*>(smem + kOffMh);             // [128]
   volatile int* epi_seg = reinterpret_cast<volatile int*>(smem + kOffEpi);           // [128]
@@ -370,22 +445,29 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       // first row of a tile in the cache, or -1 for a page-table entry out of range
-      auto tile_row = [&](const TileCursor& t) -> int64_t {
+      auto tile_row = [&](const Cursor& t) -> int64_t {
         const int j = t.j();
         if (p.page_table == nullptr) return (int64_t)t.b * p.seq_stride + j;
         const int32_t page = p.page_table[(int64_t)t.b * p.max_pages + j / kTileTokens];
         if (page < 0 || page >= p.num_pages) return -1;
         return (int64_t)page * kTileTokens + (j % kTileTokens);
       };
-      TileCursor c;
+      Cursor c;
       c.init(p);
       if (c.valid) {   // the first segment's query columns: one request, ahead of the tiles
-        const int qrow = c.b * p.q_row_stride + p.row_base;
         const uint32_t qdst = sbase + kStageBytes;
         mbar_arrive_expect_tx(bar(kBarQLanded), kQBytes);
-        for (int i = 0; i < 4; ++i)
-          tma_load_2d(qdst + i * kQBoxC, &tmap_q, 256 * (int)rank + 64 * i, qrow, bar(kBarQLanded));
-        tma_load_2d(qdst + 4 * kQBoxC, &tmap_qr, kDLatent + 32 * (int)rank, qrow, bar(kBarQLanded));
+        if constexpr (kPrefill) {   // 128 tokens of one head: (column, head, token) maps
+          const int tok = c.b * p.q_tokens + 128 * c.tb;
+          for (int i = 0; i < 4; ++i)
+            tma_load_3d(qdst + i * kQBoxC, &tmap_q, 256 * (int)rank + 64 * i, c.head, tok, bar(kBarQLanded));
+          tma_load_3d(qdst + 4 * kQBoxC, &tmap_qr, kDLatent + 32 * (int)rank, c.head, tok, bar(kBarQLanded));
+        } else {
+          const int qrow = c.b * p.q_row_stride + p.row_base;
+          for (int i = 0; i < 4; ++i)
+            tma_load_2d(qdst + i * kQBoxC, &tmap_q, 256 * (int)rank + 64 * i, qrow, bar(kBarQLanded));
+          tma_load_2d(qdst + 4 * kQBoxC, &tmap_qr, kDLatent + 32 * (int)rank, qrow, bar(kBarQLanded));
+        }
       }
       for (; c.valid; c.next(p)) {
         const uint32_t g = c.g, st = g % kStages;
@@ -427,7 +509,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     // S(g) = Q . K(g)^T once the tile landed, the softmax has copied S(g-1) out of TMEM
     // and (first tile of a segment) the segment's query columns are in TMEM.
     if (lane == 0) {
-      TileCursor c;
+      Cursor c;
       c.init(p);
       for (; c.valid; c.next(p)) {
         const uint32_t g = c.g, st = g % kStages;
@@ -467,7 +549,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     // O += P(g) . V(g) once P(g) is in TMEM and (first tile of a segment) the previous
     // segment's O has been read out. Its completion frees the stage, P, and O.
     if (lane == 0) {
-      TileCursor c;
+      Cursor c;
       c.init(p);
       for (; c.valid; c.next(p)) {
         const uint32_t g = c.g, st = g % kStages;
@@ -561,7 +643,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
 
     uint32_t total = 0;   // tiles of this cluster's work
     {
-      TileCursor t;
+      Cursor t;
       t.init(p);
       if (t.valid) {   // two thirds of the first segment's query columns (the rest: transitions)
         if (wait_bounded(bar(kBarQLanded), 0, guard)) {
@@ -573,7 +655,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       }
       for (; t.valid; t.next(p)) ++total;
     }
-    TileCursor c;
+    Cursor c;
     c.init(p);
     float m_own = -INFINITY, l_own = 0.f;   // this warpgroup's max and normaliser share
     int my_seg = -1;                        // segment of the last tile this warpgroup took
@@ -585,9 +667,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
         const uint32_t st = g % kStages, u = g >> 1, xb = u & 1u;
         if (!wait_spin(bar(kBarKvFull + st), (g / kStages) & 1u, guard)) break;
         const int r = tile_valid[st] ? c.rows() : 0;   // valid tokens of the tile
-        // ... of which this row sees those up to its own token's position: new token t of
-        // q_len sits at len - q_len + t and does not see the new tokens after it
-        const int rr = max(0, min(r, c.len - (p.q_len - 1 - (p.row_base + h) / p.heads_per_token) - c.j()));
+        // ... of which this row sees those up to its own token's position
+        const int rr = max(0, min(r, c.visible(p, h) - c.j()));
         // own partial S out of TMEM (S is free for the next QK once we have it)
         float sv[kT];
         {
@@ -745,7 +826,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
     const int h = 32 * quarter + lane;
     const uint32_t lanes = (uint32_t)(32 * quarter) << 16;
     const bool head_ok = h < p.n_heads;
-    TileCursor c;
+    Cursor c;
     c.init(p);
     int prev_slot = -1;
     auto epilogue = [&](uint32_t seg, int slot) -> bool {
@@ -763,6 +844,39 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       const float l1 = m1.y > 0.f ? m1.y * exp2f(m1.x - mlast) : 0.f;
       const float2 mls = make_float2(mlast, l0 + l1);
       const float inv = mls.y > 0.f ? 1.f / mls.y : 0.f;
+      const float lse_e = mls.y > 0.f ? (mls.x + log2f(mls.y)) * 0.69314718055994531f : -INFINITY;
+      if constexpr (kPrefill) {
+        // the item's row h is new token t of the head: its normalised latent (this CTA's 256
+        // columns) and lse go straight to the output
+        const int tb = slot % p.n_blocks, head = (slot / p.n_blocks) % p.heads_per_token;
+        const int b = slot / (p.n_blocks * p.heads_per_token);
+        const int t = 128 * tb + h;
+        const bool row_ok = t < p.q_tokens;
+        const int64_t orow = ((int64_t)b * p.q_tokens + (row_ok ? t : 0)) * p.heads_per_token + head;
+        __nv_bfloat16* dst = p.out_latent + orow * kDLatent + 256 * rank;
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t o[32];
+          tmem_ld32_sync(lanes | (tmem + kTmemO + 32 * cc), o);
+          if (row_ok) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t w[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[8 * q + 2 * i]) * inv,
+                                                          __uint_as_float(o[8 * q + 2 * i + 1]) * inv);
+                w[i] = *reinterpret_cast<uint32_t*>(&b2);
+              }
+              *reinterpret_cast<uint4*>(dst + 32 * cc + 8 * q) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        }
+        if (row_ok && rank == 0 && p.out_lse != nullptr) p.out_lse[orow] = lse_e;
+        tc_fence_before();
+        mbar_arrive(bar(kBarOFree));
+        return true;
+      }
       // partial O as [slot][column quad][head][4 floats]: the 32 heads of a warp write 512
       // contiguous bytes per store
       const int64_t quad_stride = (int64_t)p.n_heads * 4;
@@ -780,9 +894,7 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
                             __uint_as_float(o[4 * q + 2]) * inv, __uint_as_float(o[4 * q + 3]) * inv);
         }
       }
-      if (head_ok && rank == 0)
-        p.part_lse[(int64_t)slot * p.n_heads + h] =
-            mls.y > 0.f ? (mls.x + log2f(mls.y)) * 0.69314718055994531f : -INFINITY;
+      if (head_ok && rank == 0) p.part_lse[(int64_t)slot * p.n_heads + h] = lse_e;
       tc_fence_before();
       mbar_arrive(bar(kBarOFree));
       return true;
@@ -827,7 +939,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
           mbar_arrive(bar(kBarQReady0));
         } else {
 #pragma unroll 1
-          for (int part = 0; part < 3; ++part) load_q_part(p, smem, tmem, lanes, h, c.b, part, rank);
+          const __nv_bfloat16* qrow = c.q_row(p, h);
+          for (int part = 0; part < 3; ++part) load_q_part(qrow, smem, tmem, lanes, h, part, rank);
           tmem_wait_st();
           fence_proxy_async_smem();   // the k^R query columns are read by the MMA (async proxy)
           tc_fence_before();
@@ -851,8 +964,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       }
       prev_slot = seg_slot;
       if (!ok) break;
-      if (c.valid && head_ok) {
-        const __nv_bfloat16* qrow = p.q_abs + ((int64_t)c.b * p.q_row_stride + p.row_base + h) * kRow;
+      const __nv_bfloat16* qrow = c.valid ? c.q_row(p, h) : nullptr;
+      if (qrow != nullptr) {
         asm volatile("prefetch.global.L2 [%0];" :: "l"(qrow + 256 * (int)rank) : "memory");
         asm volatile("prefetch.global.L2 [%0];" :: "l"(qrow + 256 * (int)rank + 64) : "memory");
         asm volatile("prefetch.global.L2 [%0];" :: "l"(qrow + 256 * (int)rank + 128) : "memory");
@@ -926,19 +1039,88 @@ bool encode_codes(CUtensorMap* m, const void* base, uint64_t rows, int64_t row_s
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
+// q_abs [B, T, n_h, 576] as a 3-D tensor (columns, heads, tokens): a {box_cols, 1, 128} box is
+// 128 consecutive tokens of one head and lands as 128 rows of box_cols columns.
+bool encode_tokens(CUtensorMap* m, const void* base, uint64_t heads, uint64_t tokens, uint32_t box_cols,
+                   CUtensorMapSwizzle swz) {
+  const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)kRow, heads, tokens};
+  const cuuint64_t strides[2] = {(cuuint64_t)kRow * 2, (cuuint64_t)heads * kRow * 2};
+  const cuuint32_t box[3] = {box_cols, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
-cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfloat16* q_abs,
-                                const CacheView& cv, int row_base, cudaStream_t s) {
+cudaError_t set_smem_attributes() {
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(decode_split_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr_err = cudaFuncSetAttribute(decode_split_tc<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)kSmemAlloc);
     if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(decode_split_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      attr_err = cudaFuncSetAttribute(decode_split_tc<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kSmemAlloc);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(decode_split_tc<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kSmemAlloc);
   });
+  return attr_err;
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const mla_decode_s& h, int batch, const __nv_bfloat16* q_abs,
+                           const CacheView& cv, __nv_bfloat16* out_latent, float* lse, cudaStream_t s) {
+  const cudaError_t attr = set_smem_attributes();
+  if (attr != cudaSuccess) return attr;
+  if (cv.kv_exp != nullptr) return cudaErrorInvalidValue;
+  const int64_t rows = cv.page_table != nullptr ? (int64_t)cv.num_pages * cv.page_size
+                                                : (int64_t)batch * cv.seq_stride;
+  if (rows <= 0 || rows >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+  const int T = h.q_len, n_h = h.cfg.n_heads;
+  CUtensorMap tc, tr, tq, tqr;
+  if (!encode_latent_groups(&tc, cv.c_kv, (uint64_t)rows, cv.row_stride) ||
+      !encode_rows(&tr, cv.k_r, kDRope, (uint64_t)rows, cv.row_stride, 32, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !encode_tokens(&tq, q_abs, (uint64_t)n_h, (uint64_t)batch * T, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tokens(&tqr, q_abs, (uint64_t)n_h, (uint64_t)batch * T, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  Params p{};
+  p.q_abs = q_abs;
+  p.batch = batch;
+  p.n_heads = 128;           // attention rows per item: 128 tokens of one head
+  p.q_len = T;
+  p.heads_per_token = n_h;
+  p.row_base = 0;
+  p.q_row_stride = T * n_h;
+  p.seq_stride = cv.seq_stride;
+  p.page_table = cv.page_table;
+  p.max_pages = cv.max_pages;
+  p.num_pages = cv.num_pages;
+  p.scale_log2 = h.scale * 1.4426950408889634f;
+  p.part_o = h.ws.part_o;
+  p.part_lse = h.ws.part_lse;
+  p.err = h.ws.err;
+  p.wait_limit = 2000000000LL;  // SM cycles, about a second
+  p.kv_exp = nullptr;
+  p.kv_rows = rows;
+  p.q_tokens = T;
+  p.n_blocks = (T + 127) / 128;
+  p.n_items = batch * n_h * p.n_blocks;
+  p.kv_lens = cv.kv_lens;
+  p.max_kv_len = h.cfg.max_kv_len;
+  p.out_latent = out_latent;
+  p.out_lse = lse;
+  const int pairs = std::max(1, std::min(p.n_items, h.num_sms / 2));
+  return launch_pdl(decode_split_tc<false, true>, dim3(2 * pairs), dim3(kThreads), kSmemAlloc, s, tc, tr, tq,
+                    tqr, p);
+}
+
+cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfloat16* q_abs,
+                                const CacheView& cv, int row_base, cudaStream_t s) {
+  const cudaError_t attr_err = set_smem_attributes();
   if (attr_err != cudaSuccess) return attr_err;
 
   const int64_t rows = cv.page_table != nullptr ? (int64_t)cv.num_pages * cv.page_size
@@ -981,8 +1163,8 @@ cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfl
   const int pairs = std::max(1, std::min(h.units, h.num_sms / 2));
   // the 2-CTA cluster shape is compiled into the kernel
   return cv.kv_exp != nullptr
-             ? launch_pdl(decode_split_tc<true>, dim3(2 * pairs), dim3(kThreads), kSmemAlloc, s, tc, tr, tq, tqr, p)
-             : launch_pdl(decode_split_tc<false>, dim3(2 * pairs), dim3(kThreads), kSmemAlloc, s, tc, tr, tq, tqr, p);
+             ? launch_pdl(decode_split_tc<true, false>, dim3(2 * pairs), dim3(kThreads), kSmemAlloc, s, tc, tr, tq, tqr, p)
+             : launch_pdl(decode_split_tc<false, false>, dim3(2 * pairs), dim3(kThreads), kSmemAlloc, s, tc, tr, tq, tqr, p);
 }
 
 }  // namespace mla

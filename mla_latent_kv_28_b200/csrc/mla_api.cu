@@ -35,7 +35,7 @@ int config_status(const mla_config_t* c) {
   if (c->q_len < 0) return MLA_ERR_INVALID_ARG;
   {
     const int64_t T = c->q_len > 1 ? c->q_len : 1;
-    if ((int64_t)c->n_heads * T > mla::kMaxRows || (int64_t)c->max_batch * T > mla::kMaxBatch)
+    if ((int64_t)c->n_heads * T > mla::kMaxRows || (int64_t)c->max_batch * T > mla::kMaxTokenRows)
       return MLA_ERR_UNSUPPORTED;
   }
   if (!(c->yarn_factor >= 0.f) || !std::isfinite(c->yarn_factor) ||
@@ -188,6 +188,30 @@ int mla_absorb_q(mla_handle_t h, int32_t batch, const void* q_c, const void* q_r
 
 namespace {
 
+// The cache arguments of the attention calls, checked against the handle.
+int cache_view(const mla_decode_s* h, const void* c_kv, const void* k_r, int64_t row_stride,
+               int64_t seq_stride, const int32_t* page_table, int32_t max_pages, int32_t num_pages,
+               mla::CacheView* cv) {
+  if (!aligned16(c_kv) || !aligned16(k_r)) return MLA_ERR_INVALID_ARG;
+  if (row_stride < kDLatent || row_stride % 8 != 0) return MLA_ERR_INVALID_ARG;
+  *cv = mla::CacheView{};
+  cv->c_kv = static_cast<const __nv_bfloat16*>(c_kv);
+  cv->k_r = static_cast<const __nv_bfloat16*>(k_r);
+  cv->row_stride = row_stride;
+  cv->page_size = h->cfg.page_size;
+  if (h->cfg.page_size == 0) {
+    if (page_table != nullptr || seq_stride < h->cfg.max_kv_len) return MLA_ERR_INVALID_ARG;
+    cv->seq_stride = seq_stride;
+  } else {
+    const int64_t need = (h->cfg.max_kv_len + h->cfg.page_size - 1) / h->cfg.page_size;
+    if (page_table == nullptr || max_pages < need || num_pages < 1) return MLA_ERR_INVALID_ARG;
+    cv->page_table = page_table;
+    cv->max_pages = max_pages;
+    cv->num_pages = num_pages;
+  }
+  return MLA_OK;
+}
+
 // The shared body of mla_decode_attn (bf16 latent) and mla_decode_attn_partial (fp32).
 int decode_attn_common(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
                        const void* k_r, int64_t row_stride, int64_t seq_stride,
@@ -230,6 +254,26 @@ int decode_attn_common(mla_handle_t h, int32_t batch, const void* q_abs, const v
 }
 
 }  // namespace
+
+int mla_prefill_attn(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
+                     const void* k_r, int64_t row_stride, int64_t seq_stride,
+                     const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                     int32_t num_pages, void* out_latent, float* lse, mla_stream_t stream) {
+  if (h == nullptr || q_abs == nullptr || c_kv == nullptr || k_r == nullptr ||
+      kv_lens == nullptr || out_latent == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > h->cfg.max_batch) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_abs) || !aligned16(out_latent) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3) != 0))
+    return MLA_ERR_INVALID_ARG;
+  mla::CacheView cv;
+  const int st = cache_view(h, c_kv, k_r, row_stride, seq_stride, page_table, max_pages, num_pages, &cv);
+  if (st != MLA_OK) return st;
+  cv.kv_lens = kv_lens;
+  const cudaError_t e = mla::launch_prefill(*h, batch, static_cast<const __nv_bfloat16*>(q_abs), cv,
+                                            static_cast<__nv_bfloat16*>(out_latent), lse, stream);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
 
 int mla_decode_attn(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
                     const void* k_r, int64_t row_stride, int64_t seq_stride,

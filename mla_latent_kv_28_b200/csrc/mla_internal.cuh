@@ -16,7 +16,8 @@ constexpr int kDLatent = 512;  // d_c
 constexpr int kDRope = 64;     // d_h^R
 constexpr int kRow = kDLatent + kDRope;  // one cache row: [c^KV ; k^R]
 constexpr int kMaxHeads = 128;
-constexpr int kMaxRows = 1024;   // attention rows per sequence (heads x new tokens), in groups of 128
+constexpr int kMaxRows = 1 << 20;   // attention rows per sequence (heads x new tokens)
+constexpr int kMaxTokenRows = 8192;  // (sequence, new token) rows per call: max_batch x new tokens
 constexpr int kMaxBatch = 1024;
 constexpr int kTileTokens = 64;  // tokens per KV tile: the unit of the work plan
 constexpr int kAppendSlices = 16;  // the cache write's projection is split over at most 16 slices of d
@@ -121,12 +122,19 @@ struct CacheView {
   // quantised cache: c_kv / k_r point at E4M3 codes (row_stride in bytes), and row r's values
   // are 2^kv_exp[r] times its codes' values
   const int8_t* kv_exp = nullptr;
+  const int32_t* kv_lens = nullptr;   // prefill: read by the kernel itself (no split plan)
 };
 
 // row_base: the first of the (at most group_rows) attention rows of each sequence this launch
 // takes; the partials it writes hold just those rows.
 cudaError_t launch_decode_split(const mla_decode_s& h, int batch, const __nv_bfloat16* q_abs,
                                 const CacheView& cache, int row_base, cudaStream_t s);
+
+// Prefill: attention of the handle's q_len new tokens of every sequence over its cache rows,
+// one work item (one head, 128 consecutive tokens) per cluster at a time; the normalised latent
+// rows [B, T, n_h, 512] and lse [B, T, n_h] (or nullptr) are written directly.
+cudaError_t launch_prefill(const mla_decode_s& h, int batch, const __nv_bfloat16* q_abs,
+                           const CacheView& cv, __nv_bfloat16* out_latent, float* lse, cudaStream_t s);
 
 cudaError_t launch_combine(const mla_decode_s& h, int batch, __nv_bfloat16* out_latent,
                            float* lse, int row_base, cudaStream_t s);

@@ -69,12 +69,13 @@ def test_config_checks(lib):
          binding.MLA_ERR_INVALID_ARG),
         (binding.make_config(8, 1, 1, yarn_factor=40.0, yarn_mscale_coef=-0.1), binding.MLA_ERR_INVALID_ARG),
         (binding.make_config(8, 1, 1, yarn_factor=40.0, yarn_original_len=0), binding.MLA_ERR_INVALID_ARG),
-        # several new tokens: at most 1024 attention rows and 1024 (sequence, token) rows
-        (binding.make_config(128, 1, 16, q_len=9), binding.MLA_ERR_UNSUPPORTED),
-        (binding.make_config(16, 512, 16, q_len=4), binding.MLA_ERR_UNSUPPORTED),
+        # several new tokens: at most 2^20 attention rows and 8192 (sequence, token) rows
+        (binding.make_config(128, 1, 16, q_len=8193), binding.MLA_ERR_UNSUPPORTED),
+        (binding.make_config(16, 512, 16, q_len=17), binding.MLA_ERR_UNSUPPORTED),
         (binding.make_config(16, 1, 16, q_len=-1), binding.MLA_ERR_INVALID_ARG),
     ]
     assert binding.check_config(binding.make_config(16, 128, 4096, q_len=8)) == binding.MLA_OK
+    assert binding.check_config(binding.make_config(128, 1, 4096, q_len=4096)) == binding.MLA_OK   # a prefill
     assert binding.check_config(binding.make_config(128, 64, 131072, yarn_factor=40.0)) == binding.MLA_OK
     assert binding.check_config(binding.make_config(8, 1, 1, yarn_factor=1.0)) == binding.MLA_OK
     for cfg, want in bad:
@@ -93,6 +94,10 @@ def test_null_handle_and_null_out_are_rejected(lib):
     assert lib.mla_decode_attn(None, 1, None, None, None, 576, 1, None, None, 0, 0, None, None,
                                None) == binding.MLA_ERR_INVALID_ARG
     assert lib.mla_apply_wuv(None, 1, None, None, None, None) == binding.MLA_ERR_INVALID_ARG
+    assert lib.mla_prefill_attn(None, 1, None, None, None, 576, 1, None, None, 0, 0, None, None,
+                                None) == binding.MLA_ERR_INVALID_ARG
+    assert lib.mla_absorb_q_fp8(None, 1, None, None, None, None, None, None, None) == binding.MLA_ERR_INVALID_ARG
+    assert lib.mla_apply_wuv_fp8(None, 1, None, None, None, None, None) == binding.MLA_ERR_INVALID_ARG
     assert lib.mla_workspace_bytes(None) == -1
 
 

@@ -40,5 +40,7 @@ def test_bench_json_line():
     for k in ("absorb_bf16", "wuv_bf16", "absorb_fp8", "wuv_fp8"):
         assert hg[k]["us"] > 0 and 0 < hg[k]["frac_of_hbm"] < 1.5, k
     assert line["fp8_weights"]["tokens_per_s"] > 0
+    pf = line["prefill"]
+    assert pf["tokens_per_s"] > 0 and 0 < pf["tensor_frac"] < 1.5
     q8 = line["fp8_cache"]
     assert q8["attn_us"] > 0 and 0 < q8["frac_of_hbm"] < 1.5

@@ -64,11 +64,13 @@ def test_single_rank_needs_no_process_group():
     bench.barrier(1, 0, cuda=False)  # a no-op without a process group
 
 
-def test_committed_decode_profile_parses():
-    """The ncu summary bench.py reads roofline.traffic from has its hash and byte count lines."""
+@pytest.mark.parametrize("workload", ["ragged_paged_b64", "v2_b32_l4096"])
+def test_committed_decode_profile_parses(workload):
+    """The ncu summaries bench.py reads roofline.traffic from have their hash and byte count
+    lines (the headline workload's is taken on the current kernel sources)."""
     import bench
     path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "profiles",
-                        "decode_attn_v2_b32_l4096.txt")
+                        f"decode_attn_{workload}.txt")
     vals = {}
     with open(path) as f:
         for line in f:
@@ -79,7 +81,9 @@ def test_committed_decode_profile_parses():
     assert float(vals["dram_bytes_per_launch"]) > float(vals["algorithmic_bytes_per_launch"]) * 0.9
     # while the kernel sources are the profiled ones, bench reports the traffic
     if vals["kernel_sources_sha"] == bench.kernel_sources_sha():
-        assert bench.profiled_traffic("v2_b32_l4096") == float(vals["dram_bytes_per_launch"])
+        assert bench.profiled_traffic(workload) == float(vals["dram_bytes_per_launch"])
+    if workload == bench.DEFAULT_WORKLOAD:
+        assert vals["kernel_sources_sha"] == bench.kernel_sources_sha()
 
 
 def _run_bench(*args, timeout=600):

@@ -69,8 +69,9 @@ __device__ __forceinline__ bool wait_simple(uint32_t bar, uint32_t parity, const
 // RoPE of the decoupled query of this head for the CTA's rows, rotated to the row's token
 // position max(kv_len - q_len + token, 0) (kv_len - 1 for one new token). The angle
 // pos * theta_m reaches ~1.3e5 rad at 128K tokens, so it is formed in double and brought into
-// [-pi, pi] by Cody-Waite reduction with a two-term 2*pi; the sine and cosine of the reduced
-// angle are taken in single precision (about 1e-7 off, far below bf16 resolution).
+// [-pi, pi] by Cody-Waite reduction with a two-term 2*pi; everything after that is single
+// precision: the sine and cosine of the reduced angle (MUFU, absolute error about 2^-21) and
+// the rotation by two fused multiply-adds, far below the bf16 rounding of the result.
 __device__ __forceinline__ void rope_rows(const GemmParams& p, int h, int b0) {
   constexpr double kTwoPiHi = 6.283185307179586;            // nearest double to 2*pi
   constexpr double kTwoPiLo = 2.4492935982947064e-16;       // 2*pi - kTwoPiHi
@@ -80,22 +81,21 @@ __device__ __forceinline__ void rope_rows(const GemmParams& p, int h, int b0) {
     if (b >= p.batch) continue;
     const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(
         p.q_r + ((int64_t)b * p.n_heads + h) * kDRope + 2 * m);
-    const float x0 = __low2float(x), x1 = __high2float(x);
-    double y0 = x0, y1 = x1;
+    float y0 = __low2float(x), y1 = __high2float(x);
     if (p.theta[m] != 0.0) {
-      const int pos = max(p.kv_lens[b / p.q_len] - p.q_len + b % p.q_len, 0);
+      const int pos = p.q_len == 1 ? max(p.kv_lens[b] - 1, 0)
+                                   : max(p.kv_lens[b / p.q_len] - p.q_len + b % p.q_len, 0);
       const double a = (double)pos * p.theta[m];
       const double k = rint(a * kInvTwoPi);
-      const double r = fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, a));
+      const float r = (float)fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, a));
       float sn, cs;
-      sincosf((float)r, &sn, &cs);
-      y0 = (double)x0 * cs - (double)x1 * sn;
-      y1 = (double)x0 * sn + (double)x1 * cs;
+      __sincosf(r, &sn, &cs);
+      const float x0 = y0, x1 = y1;
+      y0 = fmaf(x0, cs, -x1 * sn);
+      y1 = fmaf(x0, sn, x1 * cs);
     }
-    __nv_bfloat162 y;
-    y.x = __double2bfloat16(y0);   // one rounding, from double
-    y.y = __double2bfloat16(y1);
-    *reinterpret_cast<__nv_bfloat162*>(p.out + ((int64_t)b * p.n_heads + h) * kRow + kDLatent + 2 * m) = y;
+    *reinterpret_cast<__nv_bfloat162*>(p.out + ((int64_t)b * p.n_heads + h) * kRow + kDLatent + 2 * m) =
+        __floats2bfloat162_rn(y0, y1);
   }
 }
 

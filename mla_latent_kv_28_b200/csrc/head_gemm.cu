@@ -235,7 +235,7 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
       }
       mma_commit(bars + 8 * (1 + q));
       ok = wait_simple(bars + 8 * (1 + q), 0, p);
-    } else if (!FP8) {
+    } else {
       wait_simple(bars, 0, p);  // never leave with copies in flight
     }
     ok_flags[q] = ok ? 1 : 0;

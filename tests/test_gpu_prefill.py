@@ -106,3 +106,30 @@ def test_prefill_step_stage_by_stage():
                                             pairs=[(0, i)])
         assert_close(got[0, t, i], ref[0, i], f"whole prefill step, token {t} head {i}")
     h.close()
+
+
+def test_prefill_t4096_two_sequences_sampled_tokens():
+    """T = 4096 new tokens in each of two sequences (one with 2000 earlier rows), 128 heads:
+    sampled tokens, every head, against the oracle's one-token attention over the rows the token
+    sees (token t of T over L rows is a one-token decode over the first L - T + t + 1 rows, an
+    equivalence the oracle pins fix), plus the first and last token of each 128-token block."""
+    T, H = 4096, 128
+    w = wl.make_workload(2, H, [4096, 6096], seed=130)
+    a = workload_np(w)
+    g = w.to(DEV)
+    q = _queries(2, T, H, seed=131)
+    h = binding.MlaDecode(H, 2, w.max_kv_len, q_len=T)
+    lat, lse = h.prefill_attn(q.to(DEV), g.cache, g.kv_lens)
+    h.check_device_errors()
+    got_lat, got_lse = f64(lat), lse.cpu().numpy()
+    qn = to_np(q)
+    scale = oracle.default_scale()
+    for b, t in [(0, 0), (0, 127), (0, 128), (0, 2047), (0, 4095), (1, 0), (1, 1000), (1, 3968),
+                 (1, 4095)]:
+        L = int(a["kv_lens"][b])
+        n = L - T + t + 1
+        rows = a["cache"][b:b + 1]
+        ref_lat, ref_lse = oracle.latent_attention(qn[b:b + 1, t], rows, np.array([n]), scale)
+        assert_close(got_lat[b, t], ref_lat[0], f"T=4096: sequence {b} token {t}, latent")
+        assert_close(got_lse[b, t], ref_lse[0], f"T=4096: sequence {b} token {t}, lse")
+    h.close()

@@ -19,6 +19,8 @@
 // them in place, four boxes at a time (every thread reads its codes of the four boxes, the CTA
 // meets, then the threads write the bf16 rows): E4M3 values times a power of two are exact in
 // bf16, so the MMAs see exactly the dequantised weights and accumulate in fp32 as with bf16.
+// The two halves land on separate barriers: the first four boxes are expanded, and the two
+// issuers that need only them start their MMAs, while the other four are still landing.
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 
@@ -110,13 +112,12 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t codes2, float scal
   return *reinterpret_cast<uint32_t*>(&b);
 }
 
-// FP8: the head's codes (box i's 128 rows x 64 codes in the upper half of bf16 box i) -> the
-// bf16 boxes (128-byte swizzle), in two rounds of four boxes. Thread t takes row t / 2 and the
-// half t % 2 of its 64 columns (32 codes) in each box.
-__device__ __forceinline__ void expand_weights(uint8_t* smem, const GemmParams& p, int h) {
+// FP8: the codes of boxes 4 round .. 4 round + 3 (box i's 128 rows x 64 codes in the upper
+// half of bf16 box i) -> those bf16 boxes (128-byte swizzle). Thread t takes row t / 2 and the
+// half t % 2 of its 64 columns (32 codes) in each box. Every thread of the CTA calls it.
+__device__ __forceinline__ void expand_round(uint8_t* smem, const GemmParams& p, int h, int round) {
   const int t = threadIdx.x, row = t >> 1, half = t & 1;
-#pragma unroll 1
-  for (int round = 0; round < 2; ++round) {
+  {
     uint4 c[4][2];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -160,8 +161,10 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
   const uint32_t xbase = sbase + kWeightBytes;
   const uint32_t xbox = (uint32_t)p.n_tile * 128;        // bytes of one x box
   const uint32_t bars = xbase + kXBoxes * xbox;
-  // barriers: [0] operands landed, [1..4] the MMAs of issuer q done; then the TMEM slot
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (bars - sbase) + 8 * (1 + kIssuers));
+  // barriers: [0] operands landed (FP8: x and the first four code boxes), [1..4] the MMAs of
+  // issuer q done, [5] FP8: the last four code boxes landed; then the TMEM slot
+  const uint32_t bar_hi = bars + 8 * (1 + kIssuers);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (bars - sbase) + 8 * (2 + kIssuers));
   const int h = blockIdx.x, b0 = blockIdx.y * p.n_tile;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // accumulator block mb sits at column mb * col_stride; the epilogue reads 32 columns at a
@@ -173,6 +176,7 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
   if (threadIdx.x == 0) {
     mbar_init(bars, 1);                                             // operands landed
     for (int q = 0; q < kIssuers; ++q) mbar_init(bars + 8 * (1 + q), 1);  // issuer q's MMAs done
+    mbar_init(bar_hi, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&tmap_w);
     prefetch_tmap(&tmap_x);
@@ -194,33 +198,23 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
 
   bool ok = true;
   if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(bars, (FP8 ? 8 * kCodeBox : kWeightBytes) + kXBoxes * xbox);
+    mbar_arrive_expect_tx(bars, (FP8 ? 4 * kCodeBox : kWeightBytes) + kXBoxes * xbox);
+    if (FP8) mbar_arrive_expect_tx(bar_hi, 4 * kCodeBox);
     for (int i = 0; i < 8; ++i)
-      tma_load_2d(sbase + i * kWeightBox + (FP8 ? kCodeBox : 0), &tmap_w, 64 * i, 128 * h, bars);
+      tma_load_2d(sbase + i * kWeightBox + (FP8 ? kCodeBox : 0), &tmap_w, 64 * i, 128 * h,
+                  FP8 && i >= 4 ? bar_hi : bars);
     const int xcol = h * (MODE == kAbsorb ? kDHead : kDLatent);
     for (int i = 0; i < kXBoxes; ++i) tma_load_2d(xbase + i * xbox, &tmap_x, xcol + 64 * i, b0, bars);
   }
   if (MODE == kAbsorb) rope_rows(p, h, b0);   // needs no weights: runs while they load
-  volatile int* ok_flags = reinterpret_cast<volatile int*>(smem + (bars - sbase) + 8 * (1 + kIssuers) + 4);
-  bool landed = true;   // FP8: every thread waits for the codes and expands its share
-  if (FP8) {
-    landed = wait_simple(bars, 0, p);
-    if (__syncthreads_and(landed ? 1 : 0)) {
-      expand_weights(smem, p, h);
-    } else {
-      landed = false;
-    }
-    __syncthreads();
-  }
-  if (warp < kIssuers && lane == 0) {
-    const int q = warp;
-    ok = FP8 ? landed : wait_simple(bars, 0, p);
+  volatile int* ok_flags = reinterpret_cast<volatile int*>(smem + (bars - sbase) + 8 * (2 + kIssuers) + 4);
+  // issuer q's MMAs: absorb: accumulator q = output features [128q, 128q+128), K = 128 (8
+  // steps); W_UV: accumulator q = the partial sum over latent columns [128q, 128q+128). Either
+  // way they read weight boxes 2q and 2q+1 only.
+  auto issue = [&](int q) {
     tc_fence_after();
-    if (ok) {
-      // absorb: accumulator q = output features [128q, 128q+128), K = 128 (8 steps);
-      // W_UV: accumulator q = the partial sum over latent columns [128q, 128q+128)
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
+    for (int kk = 0; kk < 8; ++kk) {
         uint64_t ad, bd;
         if (MODE == kAbsorb) {
           // A[c, d]: W_UK box (2q) holds d rows x 64 c; 16 d rows per K step
@@ -232,12 +226,43 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
           bd = smem_desc(xbase + (k >> 2) * xbox + (k & 3) * 32, 16, 1024, 2);
         }
         mma_ss(tmem + q * col_stride, ad, bd, p.idesc, kk > 0 ? 1u : 0u);
-      }
-      mma_commit(bars + 8 * (1 + q));
-      ok = wait_simple(bars + 8 * (1 + q), 0, p);
-    } else {
-      wait_simple(bars, 0, p);  // never leave with copies in flight
     }
+    mma_commit(bars + 8 * (1 + q));
+  };
+  bool issued = false;   // issuer threads: this thread's MMAs are in flight
+  if (FP8) {
+    // every thread expands its share of boxes 0..3 once they land, then issuers 0 and 1 (which
+    // read only those) start while boxes 4..7 are expanded, then issuers 2 and 3
+    bool good = true;
+    for (int round = 0; round < 2; ++round) {
+      const bool landed = wait_simple(round == 0 ? bars : bar_hi, 0, p);
+      good = __syncthreads_and(good && landed ? 1 : 0) != 0;
+      if (!good) continue;
+      expand_round(smem, p, h, round);
+      __syncthreads();
+      if (warp < kIssuers && lane == 0 && (warp >> 1) == round) {
+        issue(warp);
+        issued = true;
+      }
+    }
+    if (!good && threadIdx.x == 0) {   // never leave with copies in flight
+      wait_simple(bars, 0, p);
+      wait_simple(bar_hi, 0, p);
+    }
+  }
+  if (warp < kIssuers && lane == 0) {
+    const int q = warp;
+    if (FP8) {
+      ok = issued;
+    } else {
+      ok = wait_simple(bars, 0, p);
+      if (ok) {
+        issue(q);
+      } else {
+        wait_simple(bars, 0, p);  // never leave with copies in flight
+      }
+    }
+    if (ok) ok = wait_simple(bars + 8 * (1 + q), 0, p);
     ok_flags[q] = ok ? 1 : 0;
   }
   __syncthreads();
@@ -350,7 +375,7 @@ cudaError_t launch(const mla_decode_s& h, int batch, const void* w, const int8_t
       !encode(&to, out, (uint64_t)batch, (uint64_t)h.cfg.n_heads * ko, (uint32_t)n_tile,
               CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
-  constexpr uint32_t kSmemMax = kWeightBytes + kXBoxes * kCap * 128 + 64 + 1024;
+  constexpr uint32_t kSmemMax = kWeightBytes + kXBoxes * kCap * 128 + 128 + 1024;
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
@@ -372,7 +397,7 @@ cudaError_t launch(const mla_decode_s& h, int batch, const void* w, const int8_t
     p.theta[m] = h.theta[m];
   p.err = h.ws.err;
   p.wait_limit = 2000000000LL;
-  const uint32_t smem = kWeightBytes + kXBoxes * n_tile * 128 + 64 + 1024;
+  const uint32_t smem = kWeightBytes + kXBoxes * n_tile * 128 + 128 + 1024;
   dim3 grid(h.cfg.n_heads, (batch + n_tile - 1) / n_tile);
   return launch_pdl(head_gemm_tc<MODE, FP8>, grid, dim3(kThreads), smem, s, tw, tx, to, p);
 }

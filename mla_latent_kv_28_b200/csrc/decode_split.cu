@@ -51,6 +51,7 @@
 #include <mutex>
 #include <type_traits>
 
+#include "e4m3_bf16.cuh"
 #include "mla_internal.cuh"
 #include "sm100.cuh"
 
@@ -907,15 +908,14 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       const int t = (int)threadIdx.x - 384;   // 0..127 within this warpgroup
       const int64_t row0 = tile_row_s[st];
       const int64_t row = row0 + (t >> 1);
-      const int e = (row0 >= 0 && row < p.kv_rows) ? (int)p.kv_exp[row] : 0;
-      const float scale = __uint_as_float((uint32_t)(min(max(e, -126), 127) + 127) << 23);   // 2^e
+      const int e = (row0 >= 0 && row < p.kv_rows) ? min(max((int)p.kv_exp[row], -126), 127) : 0;
       uint8_t* stage = smem + st * kStageBytes;
       TileCodes v;
       read_codes(stage, t, v);
       mbar_arrive(bar(kBarConvSync));
       if (!wait_bounded(bar(kBarConvSync), n_expanded & 1u, guard)) return false;
       ++n_expanded;
-      write_bf16(stage, t, v, scale);
+      write_bf16(stage, t, v, e);
       fence_proxy_async_smem();   // read by the MMAs (async proxy)
       mbar_arrive(bar(kBarKvConv + st));
       return true;
@@ -938,8 +938,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
           tc_fence_before();
           mbar_arrive(bar(kBarQReady0));
         } else {
-#pragma unroll 1
           const __nv_bfloat16* qrow = c.q_row(p, h);
+#pragma unroll 1
           for (int part = 0; part < 3; ++part) load_q_part(qrow, smem, tmem, lanes, h, part, rank);
           tmem_wait_st();
           fence_proxy_async_smem();   // the k^R query columns are read by the MMA (async proxy)

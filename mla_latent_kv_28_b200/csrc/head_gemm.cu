@@ -28,6 +28,7 @@
 #include <cmath>
 #include <mutex>
 
+#include "e4m3_bf16.cuh"
 #include "mla_internal.cuh"
 #include "sm100.cuh"
 
@@ -101,15 +102,24 @@ __device__ __forceinline__ void rope_rows(const GemmParams& p, int h, int b0) {
   }
 }
 
-// Two E4M3 codes (low byte first) -> their values times 2^e as a bf16 pair: E4M3 -> f16 by the
-// hardware conversion (exact), f16 -> f32 (exact), times the power-of-two scale (exact), and
-// bf16 of that (exact: 4 significant bits).
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t codes2, float scale) {
-  uint32_t h2;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((unsigned short)(codes2 & 0xFFFFu)));
-  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
-  __nv_bfloat162 b = __floats2bfloat162_rn(f.x * scale, f.y * scale);
-  return *reinterpret_cast<uint32_t*>(&b);
+// FP8: bf16 boxes 4 round .. 4 round + 3 from the codes c[i] of this thread's 32 columns of box
+// 4 round + i (row t / 2, half t % 2), tile scales 2^e[0] (boxes 0-1 of the round) and 2^e[1];
+// kWide: an exponent above kE4m3OneMulMaxExp (two multiplies per pair, same bits).
+template <bool kWide>
+__device__ __forceinline__ void write_round(uint8_t* smem, const uint4 (&c)[4][2], int round, const int (&e)[2]) {
+  const int t = threadIdx.x, row = t >> 1, half = t & 1;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const E4m3Scale s = e4m3_scale<kWide>(e[i >> 1]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {   // 16-byte chunk half * 4 + k of the row: 8 columns
+      const uint4 w = c[i][k >> 1];
+      const uint32_t lo = (k & 1) ? w.z : w.x, hi = (k & 1) ? w.w : w.y;
+      const int chunk = half * 4 + k;
+      *reinterpret_cast<uint4*>(smem + (4 * round + i) * kWeightBox + row * 128 + ((chunk ^ (row & 7)) << 4)) =
+          e4m3x8_bf16x8<kWide>(lo, hi, s);
+    }
+  }
 }
 
 // FP8: the codes of boxes 4 round .. 4 round + 3 (box i's 128 rows x 64 codes in the upper
@@ -117,33 +127,19 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t codes2, float scal
 // half t % 2 of its 64 columns (32 codes) in each box. Every thread of the CTA calls it.
 __device__ __forceinline__ void expand_round(uint8_t* smem, const GemmParams& p, int h, int round) {
   const int t = threadIdx.x, row = t >> 1, half = t & 1;
-  {
-    uint4 c[4][2];
+  uint4 c[4][2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int k = 0; k < 2; ++k)
-        c[i][k] = *reinterpret_cast<const uint4*>(smem + (4 * round + i) * kWeightBox + kCodeBox + row * 64 + half * 32 + 16 * k);
-    float scale[2];
+    for (int k = 0; k < 2; ++k)
+      c[i][k] = *reinterpret_cast<const uint4*>(smem + (4 * round + i) * kWeightBox + kCodeBox + row * 64 + half * 32 + 16 * k);
+  int e[2];
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {   // the two 128-column tiles of this round's boxes
-      const int e = p.w_exp[((int64_t)h * kDHead + row) * (kDLatent / 128) + 2 * round + q];
-      scale[q] = __uint_as_float((uint32_t)(min(max(e, -126), 127) + 127) << 23);
-    }
-    __syncthreads();   // every code of these boxes is read before any of them is overwritten
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {   // 16-byte chunk half * 4 + k of the row: 8 columns
-        const uint4 w = c[i][k >> 1];
-        const uint32_t lo = (k & 1) ? w.z : w.x, hi = (k & 1) ? w.w : w.y;
-        const float sc = scale[i >> 1];
-        const int chunk = half * 4 + k;
-        *reinterpret_cast<uint4*>(smem + (4 * round + i) * kWeightBox + row * 128 + ((chunk ^ (row & 7)) << 4)) =
-            make_uint4(e4m3x2_to_bf16x2(lo, sc), e4m3x2_to_bf16x2(lo >> 16, sc),
-                       e4m3x2_to_bf16x2(hi, sc), e4m3x2_to_bf16x2(hi >> 16, sc));
-      }
-  }
+  for (int q = 0; q < 2; ++q)   // the two 128-column tiles of this round's boxes
+    e[q] = min(max((int)p.w_exp[((int64_t)h * kDHead + row) * (kDLatent / 128) + 2 * round + q], -126), 127);
+  __syncthreads();   // every code of these boxes is read before any of them is overwritten
+  if (e[0] <= kE4m3OneMulMaxExp && e[1] <= kE4m3OneMulMaxExp) write_round<false>(smem, c, round, e);
+  else write_round<true>(smem, c, round, e);
   fence_proxy_async_smem();   // read by the MMAs (async proxy)
 }
 

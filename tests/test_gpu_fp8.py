@@ -83,6 +83,18 @@ def test_rows_spanning_decades_one_long_sequence():
     _check(w, wl.draw_q_abs(1, 128, seed=99), "decades of row magnitude")
 
 
+@pytest.mark.parametrize("lo,hi", [(-118, -110), (14, 22), (-20, 20)])
+def test_row_exponent_ranges(lo, hi):
+    """Row magnitudes 2^U(lo, hi): rows whose expanded values fall below bf16's normal range
+    (exponents down to -126), rows past the single-multiply range of the expansion (exponents
+    above 7), and both kinds mixed inside every tile."""
+    w = wl.make_workload(2, 64, [1000, 333], seed=300 + lo)
+    gen = torch.Generator().manual_seed(301 + lo)
+    mag = torch.exp2(lo + torch.rand((2, w.cache.shape[1], 1), generator=gen) * (hi - lo))
+    w.cache = (w.cache.float() * mag).to(torch.bfloat16)
+    _check(w, wl.draw_q_abs(2, 64, seed=102), f"row magnitudes 2^[{lo}, {hi}]")
+
+
 def test_argument_errors():
     h = binding.MlaDecode(16, 1, 64)
     qa = torch.zeros((1, 16, 576), dtype=torch.bfloat16, device=DEV)

@@ -73,6 +73,31 @@ def test_fp8_head_projections_every_output(batch, n_heads, q_len):
     h.close()
 
 
+@pytest.mark.parametrize("log2_scale", [-110, 20])
+def test_fp8_weight_exponent_ranges(log2_scale):
+    """Weights scaled by 2^-110 (tile exponents near the bottom of the range, expanded values
+    partly below bf16's normal range) and by 2^20 (exponents above 7: two multiplies per pair
+    in the expansion): still bit for bit the bf16 calls on the dequantised weights."""
+    batch, n_heads = 9, 32
+    w = wl.make_workload(batch, n_heads, [40] * batch, seed=75)
+    g = w.to(DEV)
+    c_uk, e_uk = quantise_weight_e4m3((w.w_uk.double() * 2.0 ** log2_scale).to(torch.bfloat16))
+    c_uv, e_uv = quantise_weight_e4m3((w.w_uv.double() * 2.0 ** log2_scale).to(torch.bfloat16))
+    assert (e_uk.min() < -117 and e_uv.min() < -117) if log2_scale < 0 else (e_uk.max() > 7 and e_uv.max() > 7)
+    h = binding.MlaDecode(n_heads, batch, w.max_kv_len, rope_base=w.rope_base)
+    q8 = h.absorb_q_fp8(g.q_c, g.q_r, c_uk.to(DEV), e_uk.to(DEV), g.kv_lens)
+    latent = wl.draw_latent(batch, n_heads, seed=76).to(DEV)
+    o8 = h.apply_wuv_fp8(latent, c_uv.to(DEV), e_uv.to(DEV))
+    wb_uk = torch.from_numpy(_deq(c_uk, e_uk)).float().to(torch.bfloat16).to(DEV)
+    wb_uv = torch.from_numpy(_deq(c_uv, e_uv)).float().to(torch.bfloat16).to(DEV)
+    qb = h.absorb_q(g.q_c, g.q_r, wb_uk, g.kv_lens)
+    ob = h.apply_wuv(latent, wb_uv)
+    h.check_device_errors()
+    assert torch.equal(q8.view(torch.int16), qb.view(torch.int16))
+    assert torch.equal(o8.view(torch.int16), ob.view(torch.int16))
+    h.close()
+
+
 def test_fp8_weights_whole_step_against_the_nonabsorbed_definition():
     w = wl.make_workload(3, 128, [700, 64, 1500], seed=74)
     a = workload_np(w)

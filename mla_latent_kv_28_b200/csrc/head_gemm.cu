@@ -69,30 +69,51 @@ __device__ __forceinline__ bool wait_simple(uint32_t bar, uint32_t parity, const
   return true;
 }
 
-// RoPE of the decoupled query of this head for the CTA's rows, rotated to the row's token
-// position max(kv_len - q_len + token, 0) (kv_len - 1 for one new token). The angle
-// pos * theta_m reaches ~1.3e5 rad at 128K tokens, so it is formed in double and brought into
-// [-pi, pi] by Cody-Waite reduction with a two-term 2*pi; everything after that is single
-// precision: the sine and cosine of the reduced angle (MUFU, absolute error about 2^-21) and
-// the rotation by two fused multiply-adds, far below the bf16 rounding of the result.
-__device__ __forceinline__ void rope_rows(const GemmParams& p, int h, int b0) {
+constexpr int kRopeRows = 128 / (kThreads / 32);   // rows of a tile per warp (n_tile <= 128)
+
+// The kv_len behind each of this thread's RoPE rows (rows w, w + 8, ... of the tile for warp w),
+// loaded before any wait and not used until the rotation, so that the loads are in flight
+// while the weights land instead of holding the thread.
+__device__ __forceinline__ void rope_lens(const GemmParams& p, int b0, int (&len)[kRopeRows]) {
+  const int w = threadIdx.x >> 5;
+#pragma unroll
+  for (int k = 0; k < kRopeRows; ++k) {
+    const int r = w + 8 * k, b = b0 + r;
+    len[k] = 0;
+    if (r < p.n_tile && b < p.batch) len[k] = p.kv_lens[p.q_len == 1 ? b : b / p.q_len];
+  }
+}
+
+// RoPE of the decoupled query of this head for the CTA's rows, from the tile of q^R that landed
+// in shared memory (row r: 64 values, 128 bytes at qr + 128 r), rotated to the row's token
+// position max(kv_len - q_len + token, 0) (kv_len - 1 for one new token).
+// The angle pos * theta_m reaches ~1.3e5 rad at 128K tokens, so it is formed in double and
+// brought into [-pi, pi] by Cody-Waite reduction with a two-term 2*pi; everything after that is
+// single precision: the sine and cosine of the reduced angle (MUFU, absolute error about
+// 2^-21) and the rotation by two fused multiply-adds, far below the bf16 rounding of the
+// result. Lane m of warp w takes the pair (2m, 2m+1) of rows w, w + 8, ... (a warp covers one
+// 128-byte row per step).
+__device__ __forceinline__ void rope_rows(const GemmParams& p, int h, int b0, const uint8_t* qr,
+                                          const int (&len)[kRopeRows]) {
   constexpr double kTwoPiHi = 6.283185307179586;            // nearest double to 2*pi
   constexpr double kTwoPiLo = 2.4492935982947064e-16;       // 2*pi - kTwoPiHi
   constexpr double kInvTwoPi = 0.15915494309189535;
-  for (int i = threadIdx.x; i < p.n_tile * (kDRope / 2); i += kThreads) {
-    const int b = b0 + i / (kDRope / 2), m = i % (kDRope / 2);
-    if (b >= p.batch) continue;
-    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(
-        p.q_r + ((int64_t)b * p.n_heads + h) * kDRope + 2 * m);
+  static_assert(kDRope / 2 == 32, "one lane per rotated pair");
+  const int m = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const double theta = p.theta[m];
+#pragma unroll
+  for (int k = 0; k < kRopeRows; ++k) {
+    const int r = w + 8 * k, b = b0 + r;
+    if (r >= p.n_tile || b >= p.batch) break;
+    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(qr + r * 128 + 4 * m);
     float y0 = __low2float(x), y1 = __high2float(x);
-    if (p.theta[m] != 0.0) {
-      const int pos = p.q_len == 1 ? max(p.kv_lens[b] - 1, 0)
-                                   : max(p.kv_lens[b / p.q_len] - p.q_len + b % p.q_len, 0);
-      const double a = (double)pos * p.theta[m];
-      const double k = rint(a * kInvTwoPi);
-      const float r = (float)fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, a));
+    if (theta != 0.0) {
+      const int pos = max(len[k] - p.q_len + (p.q_len == 1 ? 0 : b % p.q_len), 0);   // row b: token b % q_len
+      const double a = (double)pos * theta;
+      const double kq = rint(a * kInvTwoPi);
+      const float rr = (float)fma(-kq, kTwoPiLo, fma(-kq, kTwoPiHi, a));
       float sn, cs;
-      __sincosf(r, &sn, &cs);
+      __sincosf(rr, &sn, &cs);
       const float x0 = y0, x1 = y1;
       y0 = fmaf(x0, cs, -x1 * sn);
       y1 = fmaf(x0, sn, x1 * cs);
@@ -146,7 +167,8 @@ __device__ __forceinline__ void expand_round(uint8_t* smem, const GemmParams& p,
 template <int MODE, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
 head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
-             const __grid_constant__ CUtensorMap tmap_o, const GemmParams p) {
+             const __grid_constant__ CUtensorMap tmap_o, const __grid_constant__ CUtensorMap tmap_r,
+             const GemmParams p) {
   // MODE kAbsorb:    D[c, b] = sum_d W_UK[h][d][c] x[b][d]   (A = W_UK, M-major; 4 M blocks, K = 128)
   // MODE kUpProject: D[d, b] = sum_c W_UV[h][d][c] x[b][c]   (A = W_UV, K-major; 1 M block,  K = 512)
   constexpr int kMBlocks = MODE == kAbsorb ? 4 : 1;
@@ -156,11 +178,15 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
   const uint32_t sbase = smem_u32(smem);
   const uint32_t xbase = sbase + kWeightBytes;
   const uint32_t xbox = (uint32_t)p.n_tile * 128;        // bytes of one x box
-  const uint32_t bars = xbase + kXBoxes * xbox;
+  // absorb: the tile's q^R rows (n_tile x 64 bf16, unswizzled) after the x boxes
+  const uint32_t qrbase = xbase + kXBoxes * xbox;
+  const uint32_t bars = qrbase + (MODE == kAbsorb ? xbox : 0u);
   // barriers: [0] operands landed (FP8: x and the first four code boxes), [1..4] the MMAs of
-  // issuer q done, [5] FP8: the last four code boxes landed; then the TMEM slot
+  // issuer q done, [5] FP8: the last four code boxes landed, [6] absorb: q^R landed; then the
+  // TMEM slot and the issuers' flags
   const uint32_t bar_hi = bars + 8 * (1 + kIssuers);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (bars - sbase) + 8 * (2 + kIssuers));
+  const uint32_t bar_qr = bars + 8 * (2 + kIssuers);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (bars - sbase) + 8 * (3 + kIssuers));
   const int h = blockIdx.x, b0 = blockIdx.y * p.n_tile;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // accumulator block mb sits at column mb * col_stride; the epilogue reads 32 columns at a
@@ -173,10 +199,12 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
     mbar_init(bars, 1);                                             // operands landed
     for (int q = 0; q < kIssuers; ++q) mbar_init(bars + 8 * (1 + q), 1);  // issuer q's MMAs done
     mbar_init(bar_hi, 1);
+    mbar_init(bar_qr, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&tmap_w);
     prefetch_tmap(&tmap_x);
     prefetch_tmap(&tmap_o);
+    if (MODE == kAbsorb) prefetch_tmap(&tmap_r);
     // the head's weights into L2 while the previous kernel finishes (a hint only: L2 is
     // where writes land, so it cannot return stale data)
     for (int i = 0; i < 8; ++i) tma_prefetch_2d(&tmap_w, 64 * i, 128 * h);   // FP8: 64 codes per box
@@ -193,17 +221,32 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
   allow_dependent_launch();
 
   bool ok = true;
+  // absorb: the rows' kv_lens are requested before the weights, so that they do not queue
+  // behind this SM's 128 KB of weight copies; q^R comes first on a barrier of its own, and the
+  // rotation runs while the weights are landing
+  int lens[kRopeRows];
+  if (MODE == kAbsorb) {
+    rope_lens(p, b0, lens);
+    __syncthreads();
+  }
   if (threadIdx.x == 0) {
+    if (MODE == kAbsorb) {
+      mbar_arrive_expect_tx(bar_qr, xbox);
+      tma_load_2d(qrbase, &tmap_r, h * kDRope, b0, bar_qr);
+    }
     mbar_arrive_expect_tx(bars, (FP8 ? 4 * kCodeBox : kWeightBytes) + kXBoxes * xbox);
     if (FP8) mbar_arrive_expect_tx(bar_hi, 4 * kCodeBox);
+    const int xcol = h * (MODE == kAbsorb ? kDHead : kDLatent);
+    for (int i = 0; i < kXBoxes; ++i) tma_load_2d(xbase + i * xbox, &tmap_x, xcol + 64 * i, b0, bars);
     for (int i = 0; i < 8; ++i)
       tma_load_2d(sbase + i * kWeightBox + (FP8 ? kCodeBox : 0), &tmap_w, 64 * i, 128 * h,
                   FP8 && i >= 4 ? bar_hi : bars);
-    const int xcol = h * (MODE == kAbsorb ? kDHead : kDLatent);
-    for (int i = 0; i < kXBoxes; ++i) tma_load_2d(xbase + i * xbox, &tmap_x, xcol + 64 * i, b0, bars);
   }
-  if (MODE == kAbsorb) rope_rows(p, h, b0);   // needs no weights: runs while they load
-  volatile int* ok_flags = reinterpret_cast<volatile int*>(smem + (bars - sbase) + 8 * (2 + kIssuers) + 4);
+  if (MODE == kAbsorb) {
+    if (wait_simple(bar_qr, 0, p)) rope_rows(p, h, b0, smem + (qrbase - sbase), lens);
+    else if (threadIdx.x == 0) wait_simple(bar_qr, 0, p);   // never leave with the copy in flight
+  }
+  volatile int* ok_flags = reinterpret_cast<volatile int*>(smem + (bars - sbase) + 8 * (3 + kIssuers) + 4);
   // issuer q's MMAs: absorb: accumulator q = output features [128q, 128q+128), K = 128 (8
   // steps); W_UV: accumulator q = the partial sum over latent columns [128q, 128q+128). Either
   // way they read weight boxes 2q and 2q+1 only.
@@ -246,20 +289,14 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
       wait_simple(bar_hi, 0, p);
     }
   }
+  if (!FP8 && warp < kIssuers && lane == 0) {
+    issued = wait_simple(bars, 0, p);
+    if (issued) issue(warp);
+    else wait_simple(bars, 0, p);   // never leave with copies in flight
+  }
   if (warp < kIssuers && lane == 0) {
-    const int q = warp;
-    if (FP8) {
-      ok = issued;
-    } else {
-      ok = wait_simple(bars, 0, p);
-      if (ok) {
-        issue(q);
-      } else {
-        wait_simple(bars, 0, p);  // never leave with copies in flight
-      }
-    }
-    if (ok) ok = wait_simple(bars + 8 * (1 + q), 0, p);
-    ok_flags[q] = ok ? 1 : 0;
+    ok = issued && wait_simple(bars + 8 * (1 + warp), 0, p);
+    ok_flags[warp] = ok ? 1 : 0;
   }
   __syncthreads();
   tc_fence_after();
@@ -273,41 +310,41 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
   const uint32_t lanes = (uint32_t)(32 * (warp & 3)) << 16;
   const int chalf = 16 * (warp >> 2);
   const uint32_t obox = (uint32_t)p.n_tile * 128;   // bytes of one 64-feature output box
-  if (ok) {
-    for (int mb = 0; mb < kMBlocks; ++mb) {
-      const int feat = 128 * mb + 32 * (warp & 3) + lane;
-      uint8_t* col = smem + (feat >> 6) * obox + (feat & 63) * 2;
-      for (int c0 = chalf; c0 < p.n_tile; c0 += 32) {
-        float v[16];
-        uint32_t r[16];
-        if (MODE == kAbsorb) {
-          tmem_ld16_sync(lanes | (tmem + mb * col_stride + c0), r);
+  // (ok is the same for the whole CTA.) Each block of 128 features is stored as soon as it is
+  // written, so its TMA stores overlap the next block's reads of tensor memory.
+  const int x0 = h * (MODE == kAbsorb ? kRow : kDHead);
+  for (int mb = 0; mb < kMBlocks && ok; ++mb) {
+    const int feat = 128 * mb + 32 * (warp & 3) + lane;
+    uint8_t* col = smem + (feat >> 6) * obox + (feat & 63) * 2;
+    for (int c0 = chalf; c0 < p.n_tile; c0 += 32) {
+      float v[16];
+      uint32_t r[16];
+      if (MODE == kAbsorb) {
+        tmem_ld16_sync(lanes | (tmem + mb * col_stride + c0), r);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
-        } else {
+        for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+      } else {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = 0.f;
-          for (int q = 0; q < kIssuers; ++q) {   // the four partial sums over the latent columns
-            tmem_ld16_sync(lanes | (tmem + q * col_stride + c0), r);
+        for (int j = 0; j < 16; ++j) v[j] = 0.f;
+        for (int q = 0; q < kIssuers; ++q) {   // the four partial sums over the latent columns
+          tmem_ld16_sync(lanes | (tmem + q * col_stride + c0), r);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] += __uint_as_float(r[j]);
-          }
+          for (int j = 0; j < 16; ++j) v[j] += __uint_as_float(r[j]);
         }
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (c0 + j < p.n_tile)
-            *reinterpret_cast<__nv_bfloat16*>(col + (c0 + j) * 128) = __float2bfloat16_rn(v[j]);
       }
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (c0 + j < p.n_tile)
+          *reinterpret_cast<__nv_bfloat16*>(col + (c0 + j) * 128) = __float2bfloat16_rn(v[j]);
     }
     fence_proxy_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int k = 2 * mb; k < 2 * mb + 2; ++k) tma_store_2d(&tmap_o, sbase + k * obox, x0 + 64 * k, b0);
+      bulk_commit_group();
+    }
   }
-  __syncthreads();
-  if (ok && threadIdx.x == 0) {
-    const int x0 = h * (MODE == kAbsorb ? kRow : kDHead);
-    for (int k = 0; k < kMBlocks * 2; ++k) tma_store_2d(&tmap_o, sbase + k * obox, x0 + 64 * k, b0);
-    bulk_commit_group();
-    bulk_wait_group0();
-  }
+  if (ok && threadIdx.x == 0) bulk_wait_group0();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -363,7 +400,7 @@ cudaError_t launch(const mla_decode_s& h, int batch, const void* w, const int8_t
   const int n_tile = std::min(kCap, (batch + 15) / 16 * 16);
   const int kx = MODE == kAbsorb ? kDHead : kDLatent;
   const int ko = MODE == kAbsorb ? kRow : kDHead;   // output row of one head
-  CUtensorMap tw, tx, to;
+  CUtensorMap tw, tx, to, tr;
   const bool w_ok = FP8 ? encode_codes(&tw, w, (uint64_t)h.cfg.n_heads * kDHead)
                         : encode(&tw, w, (uint64_t)h.cfg.n_heads * kDHead, kDLatent, 128);
   if (!w_ok ||
@@ -371,7 +408,13 @@ cudaError_t launch(const mla_decode_s& h, int batch, const void* w, const int8_t
       !encode(&to, out, (uint64_t)batch, (uint64_t)h.cfg.n_heads * ko, (uint32_t)n_tile,
               CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
-  constexpr uint32_t kSmemMax = kWeightBytes + kXBoxes * kCap * 128 + 128 + 1024;
+  // absorb: q^R [rows, n_h * 64] in boxes of 64 values x n_tile rows (W_UV: unused)
+  tr = tx;
+  if (MODE == kAbsorb && !encode(&tr, q_r, (uint64_t)batch, (uint64_t)h.cfg.n_heads * kDRope,
+                                 (uint32_t)n_tile, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  constexpr int kBoxes = kXBoxes + (MODE == kAbsorb ? 1 : 0);   // x boxes, and absorb's q^R box
+  constexpr uint32_t kSmemMax = kWeightBytes + kBoxes * kCap * 128 + 128 + 1024;
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
@@ -393,9 +436,9 @@ cudaError_t launch(const mla_decode_s& h, int batch, const void* w, const int8_t
     p.theta[m] = h.theta[m];
   p.err = h.ws.err;
   p.wait_limit = 2000000000LL;
-  const uint32_t smem = kWeightBytes + kXBoxes * n_tile * 128 + 128 + 1024;
+  const uint32_t smem = kWeightBytes + kBoxes * n_tile * 128 + 128 + 1024;
   dim3 grid(h.cfg.n_heads, (batch + n_tile - 1) / n_tile);
-  return launch_pdl(head_gemm_tc<MODE, FP8>, grid, dim3(kThreads), smem, s, tw, tx, to, p);
+  return launch_pdl(head_gemm_tc<MODE, FP8>, grid, dim3(kThreads), smem, s, tw, tx, to, tr, p);
 }
 
 }  // namespace

@@ -96,21 +96,28 @@ split_plan_kernel(const int32_t* __restrict__ kv_lens, int batch, int64_t max_kv
   const int total = s_tstart[batch];
   for (int b = tid; b <= batch; b += kPlanThreads) plan.seq_tile[b] = s_tstart[b];
 
-  int n_units = 0;
+  int n_units = 0, per = 0;
   if (total > 0) {
     if (max_splits == 0) {
-      const int per = (total + units_target - 1) / units_target;
+      per = (total + units_target - 1) / units_target;
       n_units = (total + per - 1) / per;
-      for (int u = tid; u < n_units; u += kPlanThreads) plan.unit_begin[u] = u * per;
+      for (int u = tid; u < n_units; u += kPlanThreads) {
+        plan.unit_begin[u] = u * per;
+        // first sequence of the unit: the one whose tile range holds its first tile
+        plan.unit_seq[u] = upper_index(s_tstart, batch, u * per);
+      }
     } else {
-      // sequence b is cut into min(max_splits, tiles) near-equal ranges
+      // sequence b is cut into min(max_splits, tiles) near-equal ranges, units s_aux[b] on
       for (int b = tid; b < batch; b += kPlanThreads) s_aux[b] = min(s_a[b], max_splits);
       __syncthreads();
       block_exclusive_scan(s_aux, batch, s_aux, s_warp);
       n_units = s_aux[batch];
       for (int b = tid; b < batch; b += kPlanThreads) {
         const int t = s_a[b], n = min(t, max_splits);
-        for (int k = 0; k < n; ++k) plan.unit_begin[s_aux[b] + k] = s_tstart[b] + (k * t) / n;
+        for (int k = 0; k < n; ++k) {
+          plan.unit_begin[s_aux[b] + k] = s_tstart[b] + (k * t) / n;
+          plan.unit_seq[s_aux[b] + k] = b;
+        }
       }
     }
   }
@@ -119,19 +126,20 @@ split_plan_kernel(const int32_t* __restrict__ kv_lens, int batch, int64_t max_kv
     plan.header[0] = total;
     plan.header[1] = n_units;
   }
-  __threadfence_block();
-  __syncthreads();   // unit_begin is read back below
 
-  // first sequence of each unit: the one whose tile range holds the unit's first tile
-  for (int u = tid; u < n_units; u += kPlanThreads)
-    plan.unit_seq[u] = upper_index(s_tstart, batch, plan.unit_begin[u]);
-  // first unit of each sequence, and how many units (slots) it spans
+  // first unit of each sequence and how many units (slots) it spans, from the cut itself
+  // (no search of unit_begin in global memory): balanced units are per tiles long; capped
+  // units never cross a sequence
   for (int b = tid; b < batch; b += kPlanThreads) {
     int n = 0, first = 0;
     if (s_a[b] > 0) {
-      first = upper_index(plan.unit_begin, n_units, s_tstart[b]);
-      const int last = upper_index(plan.unit_begin, n_units, s_tstart[b] + s_a[b] - 1);
-      n = last - first + 1;
+      if (max_splits == 0) {
+        first = s_tstart[b] / per;
+        n = (s_tstart[b] + s_a[b] - 1) / per - first + 1;
+      } else {
+        first = s_aux[b];
+        n = min(s_a[b], max_splits);
+      }
     }
     plan.seq_unit[b] = first;
     s_aux[b] = n;   // slots of sequence b

@@ -455,6 +455,9 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
       };
       Cursor c;
       c.init(p);
+      // decode reads each cache tile once: its lines may leave L2 first, ahead of the split
+      // partials the combine reads next (prefill items of other heads re-read the same rows)
+      const uint64_t pol = kPrefill ? l2_policy_evict_normal() : l2_policy_evict_first();
       if (c.valid) {   // the first segment's query columns: one request, ahead of the tiles
         const uint32_t qdst = sbase + kStageBytes;
         mbar_arrive_expect_tx(bar(kBarQLanded), kQBytes);
@@ -484,17 +487,17 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
         if (ok && q8) {   // the codes, each box's into the upper half of its bf16 slot
           mbar_arrive_expect_tx(bar(kBarKvFull + st), kQ8StageBytes);
           for (int i = 0; i < 4; ++i)
-            tma_load_2d(dst + i * kBoxC + kBoxC / 2, &tmap_c, 256 * (int)rank + 64 * i, (int)row,
-                        bar(kBarKvFull + st));
-          tma_load_2d(dst + 4 * kBoxC + kBoxR / 2, &tmap_r, kDLatent + 32 * (int)rank, (int)row,
-                      bar(kBarKvFull + st));
+            tma_load_2d_hint(dst + i * kBoxC + kBoxC / 2, &tmap_c, 256 * (int)rank + 64 * i, (int)row,
+                             bar(kBarKvFull + st), pol);
+          tma_load_2d_hint(dst + 4 * kBoxC + kBoxR / 2, &tmap_r, kDLatent + 32 * (int)rank, (int)row,
+                           bar(kBarKvFull + st), pol);
         } else if (ok) {
           mbar_arrive_expect_tx(bar(kBarKvFull + st), kStageBytes);
           // the CTA's four 64-column c^KV boxes in one copy (3-D map: column, row, column group),
           // then its 32 k^R columns: two TMA instructions per tile keep the producer's warp
           // from crowding the softmax warps that share its SM sub-partition
-          tma_load_3d(dst, &tmap_c, 0, (int)row, 4 * (int)rank, bar(kBarKvFull + st));
-          tma_load_2d(dst + 4 * kBoxC, &tmap_r, 32 * (int)rank, (int)row, bar(kBarKvFull + st));
+          tma_load_3d_hint(dst, &tmap_c, 0, (int)row, 4 * (int)rank, bar(kBarKvFull + st), pol);
+          tma_load_2d_hint(dst + 4 * kBoxC, &tmap_r, 32 * (int)rank, (int)row, bar(kBarKvFull + st), pol);
         } else {
           mbar_arrive(bar(kBarKvFull + st));
         }
@@ -879,7 +882,8 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
         return true;
       }
       // partial O as [slot][column quad][head][4 floats]: the 32 heads of a warp write 512
-      // contiguous bytes per store
+      // contiguous bytes per store, marked to stay in L2 for the combine
+      const uint64_t keep = l2_policy_evict_last();
       const int64_t quad_stride = (int64_t)p.n_heads * 4;
       float* dst = p.part_o + ((int64_t)slot * (kDLatent / 4) + 64 * rank) * quad_stride +
                    (head_ok ? h : 0) * 4;
@@ -890,9 +894,10 @@ decode_split_tc(const __grid_constant__ CUtensorMap tmap_c, const __grid_constan
         if (head_ok) {
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<float4*>(dst + (8 * cc + q) * quad_stride) =
-                make_float4(__uint_as_float(o[4 * q]) * inv, __uint_as_float(o[4 * q + 1]) * inv,
-                            __uint_as_float(o[4 * q + 2]) * inv, __uint_as_float(o[4 * q + 3]) * inv);
+            st_global_v4_hint(dst + (8 * cc + q) * quad_stride,
+                              make_float4(__uint_as_float(o[4 * q]) * inv, __uint_as_float(o[4 * q + 1]) * inv,
+                                          __uint_as_float(o[4 * q + 2]) * inv, __uint_as_float(o[4 * q + 3]) * inv),
+                              keep);
         }
       }
       if (head_ok && rank == 0) p.part_lse[(int64_t)slot * p.n_heads + h] = lse_e;

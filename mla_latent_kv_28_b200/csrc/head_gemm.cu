@@ -181,12 +181,17 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
   // absorb: the tile's q^R rows (n_tile x 64 bf16, unswizzled) after the x boxes
   const uint32_t qrbase = xbase + kXBoxes * xbox;
   const uint32_t bars = qrbase + (MODE == kAbsorb ? xbox : 0u);
-  // barriers: [0] operands landed (FP8: x and the first four code boxes), [1..4] the MMAs of
-  // issuer q done, [5] FP8: the last four code boxes landed, [6] absorb: q^R landed; then the
-  // TMEM slot and the issuers' flags
+  // barriers: [0] operands landed (FP8: x and the first four code boxes; bf16 W_UV: issuer 0's
+  // weight and x boxes), [1..4] the MMAs of issuer q done, [5] FP8: the last four code boxes
+  // landed, [6] absorb: q^R landed, [7..9] bf16 W_UV: issuer 1..3's weight and x boxes landed;
+  // then the TMEM slot and the issuers' flags
   const uint32_t bar_hi = bars + 8 * (1 + kIssuers);
   const uint32_t bar_qr = bars + 8 * (2 + kIssuers);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (bars - sbase) + 8 * (3 + kIssuers));
+  auto bar_in = [&](int q) { return q == 0 ? bars : bars + 8 * (2 + kIssuers + q); };
+  // bf16 W_UV: each issuer starts once its own quarter of the operands is in (the absorption's
+  // issuers rotate q^R until about when the weights have landed, so it keeps one barrier)
+  constexpr bool kSplitIn = !FP8 && MODE == kUpProject;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (bars - sbase) + 8 * (6 + kIssuers));
   const int h = blockIdx.x, b0 = blockIdx.y * p.n_tile;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // accumulator block mb sits at column mb * col_stride; the epilogue reads 32 columns at a
@@ -200,6 +205,7 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
     for (int q = 0; q < kIssuers; ++q) mbar_init(bars + 8 * (1 + q), 1);  // issuer q's MMAs done
     mbar_init(bar_hi, 1);
     mbar_init(bar_qr, 1);
+    for (int q = 1; q < kIssuers; ++q) mbar_init(bar_in(q), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&tmap_w);
     prefetch_tmap(&tmap_x);
@@ -234,19 +240,29 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
       mbar_arrive_expect_tx(bar_qr, xbox);
       tma_load_2d(qrbase, &tmap_r, h * kDRope, b0, bar_qr);
     }
-    mbar_arrive_expect_tx(bars, (FP8 ? 4 * kCodeBox : kWeightBytes) + kXBoxes * xbox);
-    if (FP8) mbar_arrive_expect_tx(bar_hi, 4 * kCodeBox);
     const int xcol = h * (MODE == kAbsorb ? kDHead : kDLatent);
-    for (int i = 0; i < kXBoxes; ++i) tma_load_2d(xbase + i * xbox, &tmap_x, xcol + 64 * i, b0, bars);
-    for (int i = 0; i < 8; ++i)
-      tma_load_2d(sbase + i * kWeightBox + (FP8 ? kCodeBox : 0), &tmap_w, 64 * i, 128 * h,
-                  FP8 && i >= 4 ? bar_hi : bars);
+    if (kSplitIn) {   // quarter q: x boxes 2q, 2q+1 and weight boxes 2q, 2q+1
+      for (int q = 0; q < kIssuers; ++q) {
+        mbar_arrive_expect_tx(bar_in(q), 2 * kWeightBox + 2 * xbox);
+        for (int i = 2 * q; i < 2 * q + 2; ++i) {
+          tma_load_2d(xbase + i * xbox, &tmap_x, xcol + 64 * i, b0, bar_in(q));
+          tma_load_2d(sbase + i * kWeightBox, &tmap_w, 64 * i, 128 * h, bar_in(q));
+        }
+      }
+    } else {
+      mbar_arrive_expect_tx(bars, (FP8 ? 4 * kCodeBox : kWeightBytes) + kXBoxes * xbox);
+      if (FP8) mbar_arrive_expect_tx(bar_hi, 4 * kCodeBox);
+      for (int i = 0; i < kXBoxes; ++i) tma_load_2d(xbase + i * xbox, &tmap_x, xcol + 64 * i, b0, bars);
+      for (int i = 0; i < 8; ++i)
+        tma_load_2d(sbase + i * kWeightBox + (FP8 ? kCodeBox : 0), &tmap_w, 64 * i, 128 * h,
+                    FP8 && i >= 4 ? bar_hi : bars);
+    }
   }
   if (MODE == kAbsorb) {
     if (wait_simple(bar_qr, 0, p)) rope_rows(p, h, b0, smem + (qrbase - sbase), lens);
     else if (threadIdx.x == 0) wait_simple(bar_qr, 0, p);   // never leave with the copy in flight
   }
-  volatile int* ok_flags = reinterpret_cast<volatile int*>(smem + (bars - sbase) + 8 * (3 + kIssuers) + 4);
+  volatile int* ok_flags = reinterpret_cast<volatile int*>(smem + (bars - sbase) + 8 * (6 + kIssuers) + 4);
   // issuer q's MMAs: absorb: accumulator q = output features [128q, 128q+128), K = 128 (8
   // steps); W_UV: accumulator q = the partial sum over latent columns [128q, 128q+128). Either
   // way they read weight boxes 2q and 2q+1 only.
@@ -290,9 +306,10 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
     }
   }
   if (!FP8 && warp < kIssuers && lane == 0) {
-    issued = wait_simple(bars, 0, p);
+    const uint32_t in = kSplitIn ? bar_in(warp) : bars;
+    issued = wait_simple(in, 0, p);
     if (issued) issue(warp);
-    else wait_simple(bars, 0, p);   // never leave with copies in flight
+    else wait_simple(in, 0, p);   // never leave with copies in flight
   }
   if (warp < kIssuers && lane == 0) {
     ok = issued && wait_simple(bars + 8 * (1 + warp), 0, p);

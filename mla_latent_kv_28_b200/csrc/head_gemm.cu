@@ -10,8 +10,10 @@
 // with the weights as the M = 128 operand ("swap AB": M = output features, N = batch). A
 // single thread issues a small-N MMA only every ~80 cycles, so four warps issue in parallel
 // into separate accumulators: one 128-feature block each for the absorption, one quarter of
-// the 512-long reduction each for W_UV (the epilogue adds the four). The tile leaves tensor
-// memory through shared memory and TMA stores.
+// the 512-long reduction each for W_UV (the epilogue adds the four). In W_UV each issuer's
+// quarter of the operands lands on a barrier of its own, so its MMAs start before the rest has
+// landed. The absorption rotates q^R (brought by TMA ahead of the weights) while the weights
+// land. The tile leaves tensor memory through shared memory and TMA stores, block by block.
 //
 // FP8 weights: E4M3 codes with one power-of-two scale 2^e per 1 x 128 tile of a weight row
 // (row r of the [n_h * 128, 512] matrix, latent columns [128 t, 128 t + 128)). The codes of each

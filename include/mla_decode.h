@@ -235,6 +235,24 @@ MLA_API int mla_apply_wuv(mla_handle_t h, int32_t batch, const void* latent, con
                   void* out, mla_stream_t stream);
 
 /*
+ * One whole decode step ([V2-walk] §2.3, the absorbed inference path): mla_absorb_q, then
+ * mla_decode_attn, then mla_apply_wuv, with the same arguments and the same results, in one
+ * call. The split-KV work plan, which mla_decode_attn builds in a launch of its own, is built
+ * here by one extra block of the absorption kernel, beside the heads.
+ *   q_abs  bf16 [batch, (q_len,) n_h, 576] and latent bf16 [batch, (q_len,) n_h, 512]: device
+ *          scratch for the intermediate results, 16-byte aligned, left holding them;
+ *   out    bf16 [batch, (q_len,) n_h, 128].
+ * Every argument is checked before anything is launched (MLA_ERR_INVALID_ARG, nothing queued).
+ * Device errors (a kv_len outside 0..max_kv_len, a page-table entry out of range) are
+ * reported as for the three calls.
+ */
+MLA_API int mla_decode_step(mla_handle_t h, int32_t batch, const void* q_c, const void* q_r,
+                    const void* w_uk, const void* w_uv, const void* c_kv, const void* k_r,
+                    int64_t row_stride, int64_t seq_stride, const int32_t* kv_lens,
+                    const int32_t* page_table, int32_t max_pages, int32_t num_pages, void* q_abs,
+                    void* latent, void* out, mla_stream_t stream);
+
+/*
  * FP8 weights for the two head projections ([V3-walk] section 4.4: weights quantised in
  * 1 x 128 tiles with high-precision accumulation; section 5.5: FP8 for storage with the
  * arithmetic in BF16 is the safe first step; [V2-notes] "Inference cost": the deployed model

@@ -63,6 +63,8 @@ SIGNATURES = {
     "mla_absorb_q": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P, _P, _P]),
     "mla_decode_attn": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32, _P, _P, _P]),
     "mla_apply_wuv": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P]),
+    "mla_decode_step": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32,
+                                       _P, _P, _P, _P]),
     "mla_prefill_attn": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I64, _I64, _P, _P, _I32, _I32, _P, _P, _P]),
     "mla_absorb_q_fp8": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P, _P, _P, _P]),
     "mla_apply_wuv_fp8": (ctypes.c_int, [_P, _I32, _P, _P, _P, _P, _P]),
@@ -438,13 +440,31 @@ class MlaDecode:
 
     def step(self, q_c, q_r, w_uk, w_uv, cache, kv_lens, page_table=None, stream=None,
              bufs: Optional[dict] = None):
-        """One decode step: absorb -> split-KV attention -> W_UV. Returns the head
-        outputs [B, n_h, 128] bf16. `bufs` may hold preallocated q_abs / latent / out."""
+        """One decode step in one C call (mla_decode_step): absorb -> split-KV attention -> W_UV,
+        the same results as the three calls, with the work plan built beside the absorption.
+        Returns the head outputs [B, (T,) n_h, 128] bf16. `bufs` may hold preallocated q_abs /
+        latent / out; q_abs and latent are left holding the intermediate results."""
         bufs = bufs or {}
-        q_abs = self.absorb_q(q_c, q_r, w_uk, kv_lens, bufs.get("q_abs"), stream)
-        latent, _ = self.decode_attn(q_abs, cache, kv_lens, page_table, bufs.get("latent"),
-                                     bufs.get("lse"), want_lse=False, stream=stream)
-        return self.apply_wuv(latent, w_uv, bufs.get("out"), stream)
+        B = q_c.shape[0]
+        for t, n in ((q_c, "q_c"), (q_r, "q_r"), (w_uk, "w_uk"), (w_uv, "w_uv")):
+            _need(t, torch.bfloat16, n)
+        _need(kv_lens, torch.int32, "kv_lens")
+        row_stride, seq_stride, c_kv, k_r, max_pages, num_pages = self._cache_view(cache, page_table)
+        lead = tuple(q_c.shape[:-1])
+        q_abs, latent, out = bufs.get("q_abs"), bufs.get("latent"), bufs.get("out")
+        if q_abs is None:
+            q_abs = torch.empty(lead + (ROW,), dtype=torch.bfloat16, device=q_c.device)
+        if latent is None:
+            latent = torch.empty(lead + (D_LATENT,), dtype=torch.bfloat16, device=q_c.device)
+        if out is None:
+            out = torch.empty(lead + (128,), dtype=torch.bfloat16, device=q_c.device)
+        for t, n in ((q_abs, "q_abs"), (latent, "latent"), (out, "out")):
+            _need(t, torch.bfloat16, n)
+        _check(self._lib.mla_decode_step(
+            self._h, B, _ptr(q_c), _ptr(q_r), _ptr(w_uk), _ptr(w_uv), ctypes.c_void_p(c_kv),
+            ctypes.c_void_p(k_r), row_stride, seq_stride, _ptr(kv_lens), _ptr(page_table), max_pages,
+            num_pages, _ptr(q_abs), _ptr(latent), _ptr(out), _stream(stream)), "mla_decode_step")
+        return out
 
     def check_device_errors(self, stream=None) -> int:
         """Synchronise the stream; raise MlaError if a kernel set the device error word."""

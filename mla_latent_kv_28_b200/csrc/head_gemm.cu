@@ -33,6 +33,7 @@
 #include "e4m3_bf16.cuh"
 #include "mla_internal.cuh"
 #include "sm100.cuh"
+#include "split_plan.cuh"
 
 namespace mla {
 namespace {
@@ -58,6 +59,12 @@ struct GemmParams {
   double theta[kDRope / 2];       // absorb only: RoPE frequencies base^(-2m/d_R), 0 when off
   uint32_t* err;
   long long wait_limit;
+  // fused decode step (absorb only): one extra column of CTAs, blockIdx.x == n_heads, of which
+  // the first builds the split-KV work plan beside the heads
+  int plan_seqs;                  // sequences; 0: no plan CTA
+  int plan_units, plan_max_splits;
+  int64_t plan_max_kv_len;
+  PlanView plan;
 };
 
 __device__ __forceinline__ bool wait_simple(uint32_t bar, uint32_t parity, const GemmParams& p) {
@@ -177,6 +184,16 @@ head_gemm_tc(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
   constexpr int kXBoxes = MODE == kAbsorb ? 2 : 8;   // 64-column boxes of one x row
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (MODE == kAbsorb && p.plan_seqs > 0 && (int)blockIdx.x == p.n_heads) {
+    // the fused step's work plan (from kv_lens), built while the heads run
+    static_assert(kThreads == plan::kPlanThreads, "one block builds the plan");
+    grid_dependency_wait();   // kv_lens, and the plan arrays the previous step's kernels read
+    allow_dependent_launch();
+    if (blockIdx.y == 0)
+      plan::build_plan(p.kv_lens, p.plan_seqs, p.plan_max_kv_len, p.plan_units, p.plan_max_splits, p.plan,
+                       p.err, reinterpret_cast<int32_t*>(smem));
+    return;
+  }
   const uint32_t sbase = smem_u32(smem);
   const uint32_t xbase = sbase + kWeightBytes;
   const uint32_t xbox = (uint32_t)p.n_tile * 128;        // bytes of one x box
@@ -410,10 +427,12 @@ bool encode_codes(CUtensorMap* m, const void* base, uint64_t rows) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// plan_seqs > 0 (absorb only): also build the split-KV work plan for that many sequences, in one
+// extra CTA.
 template <int MODE, bool FP8>
 cudaError_t launch(const mla_decode_s& h, int batch, const void* w, const int8_t* w_exp,
                    const __nv_bfloat16* x, __nv_bfloat16* out, const __nv_bfloat16* q_r,
-                   const int32_t* kv_lens, cudaStream_t s) {
+                   const int32_t* kv_lens, cudaStream_t s, int plan_seqs = 0) {
   constexpr int kXBoxes = MODE == kAbsorb ? 2 : 8;
   constexpr int kCap = MODE == kAbsorb ? 128 : 64;  // weights + x boxes fit in shared memory
   const int n_tile = std::min(kCap, (batch + 15) / 16 * 16);
@@ -455,8 +474,14 @@ cudaError_t launch(const mla_decode_s& h, int batch, const void* w, const int8_t
     p.theta[m] = h.theta[m];
   p.err = h.ws.err;
   p.wait_limit = 2000000000LL;
+  p.plan_seqs = MODE == kAbsorb ? plan_seqs : 0;
+  p.plan_units = h.units;
+  p.plan_max_splits = h.cfg.max_splits;
+  p.plan_max_kv_len = h.cfg.max_kv_len;
+  p.plan = h.ws.plan;
   const uint32_t smem = kWeightBytes + kBoxes * n_tile * 128 + 128 + 1024;
-  dim3 grid(h.cfg.n_heads, (batch + n_tile - 1) / n_tile);
+  static_assert(kWeightBytes >= plan::kPlanScratchInts * 4, "the plan CTA's scratch fits");
+  dim3 grid(h.cfg.n_heads + (p.plan_seqs > 0 ? 1 : 0), (batch + n_tile - 1) / n_tile);
   return launch_pdl(head_gemm_tc<MODE, FP8>, grid, dim3(kThreads), smem, s, tw, tx, to, tr, p);
 }
 
@@ -466,6 +491,12 @@ cudaError_t launch_absorb_q(const mla_decode_s& h, int batch, const __nv_bfloat1
                             const __nv_bfloat16* q_r, const __nv_bfloat16* w_uk,
                             const int32_t* kv_lens, __nv_bfloat16* q_abs, cudaStream_t s) {
   return launch<kAbsorb, false>(h, batch, w_uk, nullptr, q_c, q_abs, q_r, kv_lens, s);
+}
+
+cudaError_t launch_absorb_q_with_plan(const mla_decode_s& h, int rows, int n_seqs, const __nv_bfloat16* q_c,
+                                      const __nv_bfloat16* q_r, const __nv_bfloat16* w_uk,
+                                      const int32_t* kv_lens, __nv_bfloat16* q_abs, cudaStream_t s) {
+  return launch<kAbsorb, false>(h, rows, w_uk, nullptr, q_c, q_abs, q_r, kv_lens, s, n_seqs);
 }
 
 cudaError_t launch_apply_wuv(const mla_decode_s& h, int batch, const __nv_bfloat16* latent,

@@ -212,36 +212,33 @@ int cache_view(const mla_decode_s* h, const void* c_kv, const void* k_r, int64_t
   return MLA_OK;
 }
 
-// The shared body of mla_decode_attn (bf16 latent) and mla_decode_attn_partial (fp32).
-int decode_attn_common(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
-                       const void* k_r, int64_t row_stride, int64_t seq_stride,
-                       const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
-                       int32_t num_pages, void* out_latent, bool out_f32, float* lse,
-                       mla_stream_t stream) {
+// The arguments of the attention calls, checked; the cache as a view.
+int attention_args(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
+                   const void* k_r, int64_t row_stride, int64_t seq_stride, const int32_t* kv_lens,
+                   const int32_t* page_table, int32_t max_pages, int32_t num_pages,
+                   const void* out_latent, const float* lse, mla::CacheView* cv) {
   if (h == nullptr || q_abs == nullptr || c_kv == nullptr || k_r == nullptr ||
       kv_lens == nullptr || out_latent == nullptr)
     return MLA_ERR_INVALID_ARG;
   if (batch < 1 || batch > h->cfg.max_batch) return MLA_ERR_INVALID_ARG;
-  if (!aligned16(q_abs) || !aligned16(c_kv) || !aligned16(k_r) || !aligned16(out_latent) ||
+  if (!aligned16(q_abs) || !aligned16(out_latent) ||
       (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3) != 0))
     return MLA_ERR_INVALID_ARG;
-  if (row_stride < kDLatent || row_stride % 8 != 0) return MLA_ERR_INVALID_ARG;
+  return cache_view(h, c_kv, k_r, row_stride, seq_stride, page_table, max_pages, num_pages, cv);
+}
+
+// The shared body of mla_decode_attn (bf16 latent), mla_decode_attn_partial (fp32) and the
+// fused step (plan_built: the absorption kernel has built the work plan already).
+int decode_attn_common(mla_handle_t h, int32_t batch, const void* q_abs, const void* c_kv,
+                       const void* k_r, int64_t row_stride, int64_t seq_stride,
+                       const int32_t* kv_lens, const int32_t* page_table, int32_t max_pages,
+                       int32_t num_pages, void* out_latent, bool out_f32, float* lse,
+                       mla_stream_t stream, bool plan_built = false) {
   mla::CacheView cv{};
-  cv.c_kv = static_cast<const __nv_bfloat16*>(c_kv);
-  cv.k_r = static_cast<const __nv_bfloat16*>(k_r);
-  cv.row_stride = row_stride;
-  cv.page_size = h->cfg.page_size;
-  if (h->cfg.page_size == 0) {
-    if (page_table != nullptr || seq_stride < h->cfg.max_kv_len) return MLA_ERR_INVALID_ARG;
-    cv.seq_stride = seq_stride;
-  } else {
-    const int64_t need = (h->cfg.max_kv_len + h->cfg.page_size - 1) / h->cfg.page_size;
-    if (page_table == nullptr || max_pages < need || num_pages < 1) return MLA_ERR_INVALID_ARG;
-    cv.page_table = page_table;
-    cv.max_pages = max_pages;
-    cv.num_pages = num_pages;
-  }
-  cudaError_t e = mla::launch_split_plan(*h, batch, kv_lens, stream);
+  const int st = attention_args(h, batch, q_abs, c_kv, k_r, row_stride, seq_stride, kv_lens,
+                                page_table, max_pages, num_pages, out_latent, lse, &cv);
+  if (st != MLA_OK) return st;
+  cudaError_t e = plan_built ? cudaSuccess : mla::launch_split_plan(*h, batch, kv_lens, stream);
   // more than 128 attention rows per sequence (several new tokens): one decode + combine per
   // group of 128 rows, each over the same cache and plan
   for (int rb = 0; e == cudaSuccess && rb < h->n_rows; rb += h->group_rows) {
@@ -423,6 +420,37 @@ int mla_apply_wuv(mla_handle_t h, int32_t batch, const void* latent, const void*
   const cudaError_t e = mla::launch_apply_wuv(
       *h, batch * h->q_len, static_cast<const __nv_bfloat16*>(latent),
       static_cast<const __nv_bfloat16*>(w_uv), static_cast<__nv_bfloat16*>(out), stream);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_decode_step(mla_handle_t h, int32_t batch, const void* q_c, const void* q_r,
+                    const void* w_uk, const void* w_uv, const void* c_kv, const void* k_r,
+                    int64_t row_stride, int64_t seq_stride, const int32_t* kv_lens,
+                    const int32_t* page_table, int32_t max_pages, int32_t num_pages, void* q_abs,
+                    void* latent, void* out, mla_stream_t stream) {
+  // every argument is checked before anything is launched
+  if (h == nullptr || q_c == nullptr || q_r == nullptr || w_uk == nullptr || w_uv == nullptr ||
+      out == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_c) || !aligned16(q_r) || !aligned16(w_uk) || !aligned16(w_uv) || !aligned16(out))
+    return MLA_ERR_INVALID_ARG;
+  mla::CacheView cv{};
+  const int st = attention_args(h, batch, q_abs, c_kv, k_r, row_stride, seq_stride, kv_lens,
+                                page_table, max_pages, num_pages, latent, nullptr, &cv);
+  if (st != MLA_OK) return st;
+  // the absorption, with the work plan built beside it; one GEMM row per (sequence, new token)
+  cudaError_t e = mla::launch_absorb_q_with_plan(
+      *h, batch * h->q_len, batch, static_cast<const __nv_bfloat16*>(q_c),
+      static_cast<const __nv_bfloat16*>(q_r), static_cast<const __nv_bfloat16*>(w_uk), kv_lens,
+      static_cast<__nv_bfloat16*>(q_abs), stream);
+  if (e != cudaSuccess) return MLA_ERR_CUDA;
+  const int st2 = decode_attn_common(h, batch, q_abs, c_kv, k_r, row_stride, seq_stride, kv_lens,
+                                     page_table, max_pages, num_pages, latent, false, nullptr,
+                                     stream, true);
+  if (st2 != MLA_OK) return st2;
+  e = mla::launch_apply_wuv(*h, batch * h->q_len, static_cast<const __nv_bfloat16*>(latent),
+                            static_cast<const __nv_bfloat16*>(w_uv), static_cast<__nv_bfloat16*>(out),
+                            stream);
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

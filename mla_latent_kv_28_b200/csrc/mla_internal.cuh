@@ -106,6 +106,11 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 cudaError_t launch_absorb_q(const mla_decode_s& h, int batch, const __nv_bfloat16* q_c,
                             const __nv_bfloat16* q_r, const __nv_bfloat16* w_uk,
                             const int32_t* kv_lens, __nv_bfloat16* q_abs, cudaStream_t s);
+// launch_absorb_q plus, in one extra CTA beside the heads, the split-KV work plan of n_seqs
+// sequences (what launch_split_plan builds), for the fused decode step.
+cudaError_t launch_absorb_q_with_plan(const mla_decode_s& h, int rows, int n_seqs, const __nv_bfloat16* q_c,
+                                      const __nv_bfloat16* q_r, const __nv_bfloat16* w_uk,
+                                      const int32_t* kv_lens, __nv_bfloat16* q_abs, cudaStream_t s);
 
 cudaError_t launch_split_plan(const mla_decode_s& h, int batch, const int32_t* kv_lens,
                               cudaStream_t s);
